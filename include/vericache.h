@@ -1,0 +1,208 @@
+/*
+ * vericache.h -- C ABI of the VeriCache draft/verify hot path for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow two web summaries:
+ *   [VC]  "Riepilogo Tecnico: VeriCache" (gist.science/it/paper/2605.17613; Arabic
+ *         translation gist.science/ar/paper/2605.17613): draft over the compressed
+ *         cache, verify all drafts in one pass over the full cache, greedy acceptance
+ *         with a bonus token, and streaming of the full cache from CPU memory over
+ *         PCIe overlapped with other requests' drafting.
+ *   [CKV] "Riassunto Tecnico: CentroidKV" (gist.science/it/paper/2506.11418): per-slot
+ *         degree n_t that enters the softmax as a logarithmic term.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, except the host
+ *     source of vc_stage_full_kv.  The library allocates nothing; scratch space is a
+ *     caller-provided workspace whose size the matching *_workspace_size call gives.
+ *   - bf16 tensors are IEEE bfloat16 (2 bytes), fp16 tensors IEEE half.  Shapes are
+ *     row-major and contiguous unless a capacity (…_cap) gives the row stride.
+ *   - Calls only enqueue work on the given stream and return at once.  The return
+ *     code covers argument validation and launch errors; errors found on the device
+ *     (out-of-range slot indices, NaN logits) are written to caller-provided flags
+ *     that the caller reads after synchronising.
+ *   - Every pointer passed to a kernel must be 16-byte aligned.
+ *   - There is no fallback path: an unsupported shape returns VC_ERR_UNSUPPORTED.
+ */
+#ifndef VERICACHE_H
+#define VERICACHE_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VC_ABI_VERSION 1
+
+typedef enum {
+  VC_OK = 0,
+  VC_ERR_INVALID = 1,      /* bad argument: NULL, negative size, misaligned, … */
+  VC_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. head dim 96) */
+  VC_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  VC_ERR_TIMEOUT = 4       /* a bounded host wait ran out */
+} vc_status;
+
+typedef enum {
+  VC_CACHE_INDEXED = 0,    /* bf16 rows picked by a slot index list, with degrees */
+  VC_CACHE_INT4 = 1        /* 4-bit group-quantised rows (see the layout below) */
+} vc_cache_kind;
+
+/* Human-readable name of a status code (static string). */
+const char* vc_status_string(int status);
+/* Detail of the last failing call in this thread (static thread-local buffer). */
+const char* vc_last_error(void);
+/* VC_ABI_VERSION of the loaded library. */
+int vc_abi_version(void);
+
+/* ------------------------------------------------------------------------------
+ * Compressed cache KV_comp of one attention layer ([VC] "Algoritmo Principale",
+ * step 1; [VC] "Supporto Architetturale": one interface for eviction and
+ * quantisation compressors).
+ *
+ * Common:  B batch, Hq query heads, Hkv kv heads (Hq % Hkv == 0, g = Hq/Hkv <= 8),
+ *          D head dim in {64, 128}.  Query head h reads kv head h / g.
+ * Tail:    k_tail, v_tail bf16 [B, Hkv, R_cap, D]; the first n_tail rows are live
+ *          (tokens appended while drafting), each of degree 1.  May be NULL when
+ *          n_tail == 0.
+ *
+ * VC_CACHE_INDEXED (token eviction, optionally merged centroids):
+ *   k, v      bf16 [B, Hkv, T_cap, D]  base rows (a full cache viewed through idx,
+ *                                      or compact slot rows when idx == NULL)
+ *   idx       int32 [B, Hkv, S_cap]    base row of slot s, 0 <= idx < T_cap; NULL
+ *                                      means slot s is row s (needs S <= T_cap)
+ *   deg       int32 [B, Hkv, S_cap]    degree n_s >= 1 of slot s ([CKV] item 4:
+ *                                      score += ln n_s); NULL means all 1
+ *   S         live slots per (batch, kv head), same for all
+ *   err_flag  int32 [1] or NULL: set to 1 when an idx entry is out of range (the
+ *             entry is clamped and the result is then meaningless) or a degree < 1
+ *
+ * VC_CACHE_INT4 (asymmetric 4-bit groups; x_hat = q * scale + zero):
+ *   Per (batch, kv head) the S quantised tokens (S % 32 == 0, capacity T_cap tokens,
+ *   T_cap % 32 == 0) form blocks of 32.  Words are little-endian uint32 of 8 nibbles
+ *   (nibble p at bits 4p..4p+3); pair j (0..3) of a word keeps its first element in
+ *   nibble j and its second in nibble j + 4.
+ *   kq        uint32 [B, Hkv, T_cap/32, 32, 4, D/32]: pair j of word (token t, c, w)
+ *             holds channels e, e+1 of token t, e = 2c + 32w + 16*(j/2) + 8*(j%2)
+ *   k_scale, k_zero  fp16 [B, Hkv, T_cap/32, D]: one group per (block, channel)
+ *   vq        uint32 [B, Hkv, T_cap/32, D, 4]: pair j of word (channel d, c) holds
+ *             channel d of tokens 2c + 8j and 2c + 8j + 1 of the block
+ *   v_scale, v_zero  fp16 [B, Hkv, T_cap/32, D/32, 32]: one group per (token,
+ *             32 consecutive channels), stored block, channel group, token
+ *   All quantised tokens have degree 1.
+ * ---------------------------------------------------------------------------- */
+typedef struct vc_comp_cache {
+  int32_t kind;                 /* vc_cache_kind */
+  int32_t B, Hq, Hkv, D;
+  int32_t S;                    /* live slots (indexed) or quantised tokens (int4) */
+  int32_t S_cap;                /* row stride of idx / deg (indexed) */
+  int64_t T_cap;                /* base rows (indexed) or token capacity (int4) */
+  /* VC_CACHE_INDEXED */
+  const void* k;
+  const void* v;
+  const int32_t* idx;
+  const int32_t* deg;
+  /* VC_CACHE_INT4 */
+  const uint32_t* kq;
+  const void* k_scale;
+  const void* k_zero;
+  const uint32_t* vq;
+  const void* v_scale;
+  const void* v_zero;
+  /* tail */
+  const void* k_tail;
+  const void* v_tail;
+  int32_t R_cap;
+  int32_t n_tail;
+  /* device error flag, may be NULL */
+  int32_t* err_flag;
+} vc_comp_cache;
+
+/* ------------------------------------------------------------------------------
+ * Draft attention: one decode step of every query head over KV_comp plus the tail
+ * ([VC] "Algoritmo Principale", step 1, with the [CKV] log-degree term):
+ *   s_t = (q . k_t) * scale + ln n_t ;  o = sum_t softmax(s)_t v_t
+ *   q    bf16 [B, Hq, D]            out  bf16 [B, Hq, D]
+ *   lse  fp32 [B, Hq] or NULL: ln sum_t exp(s_t)
+ *   scale <= 0 selects D^-1/2.
+ * Split-K over slots: ws must hold vc_draft_workspace_size(cache) bytes (device).
+ * S + n_tail must be >= 1.
+ * ---------------------------------------------------------------------------- */
+size_t vc_draft_workspace_size(const vc_comp_cache* cache);
+vc_status vc_draft_attn(const void* q, const vc_comp_cache* cache, float scale,
+                        void* out, float* lse, void* ws, size_t ws_bytes,
+                        cudaStream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * Verify attention ([VC] "Algoritmo Principale", step 2: one pass over KV_full checks
+ * all drafted tokens in parallel).  Row i (0 <= i < n_q, n_q = k + 1: the pending
+ * token and the k drafts) sits at absolute position P + i and attends every key at
+ * position <= P + i: the prefix plus the block, causal inside the block.  No degree
+ * term.
+ *   q     bf16 [B, n_q, Hq, D]
+ *   k, v  bf16 [B, Hkv, L_cap, D]: row r holds the key / value at absolute position
+ *         kv_start + r, for r < kv_len (kv_len <= L_cap).  The block's own keys
+ *         (positions P .. P+n_q-1) must already be written where they fall.
+ *   Single pass (m == l == acc == NULL): kv_start == 0, kv_len == P + n_q; writes out
+ *         bf16 [B, n_q, Hq, D].
+ *   Chunked (long context with KV_full streamed from host memory, [VC] "Supporto
+ *         Architetturale"): m, l fp32 [B, n_q, Hq] and acc fp32 [B, n_q, Hq, D] carry
+ *         the softmax state (max, sum, weighted values, natural-log domain) between
+ *         calls over consecutive key ranges in increasing kv_start.  VC_VERIFY_FIRST
+ *         resets the state before adding this range; VC_VERIFY_LAST writes out after
+ *         adding it.  Ranges must tile [0, P + n_q) exactly, in order.
+ *   Results do not depend on n_q or on other rows: key tiles and split boundaries sit
+ *   at fixed absolute positions, and splits are merged in a fixed order.
+ *   ws: vc_verify_workspace_size(...) bytes of device memory.
+ *   Supported: D in {64, 128}, g <= 8, n_q * g <= 1024.
+ * ---------------------------------------------------------------------------- */
+#define VC_VERIFY_FIRST 1
+#define VC_VERIFY_LAST 2
+size_t vc_verify_workspace_size(int B, int n_q, int Hq, int Hkv, int D,
+                                int64_t kv_start, int64_t kv_len);
+vc_status vc_verify_attn(const void* q, int B, int n_q, int Hq, int Hkv, int D,
+                         const void* k, const void* v, int64_t L_cap,
+                         int64_t kv_start, int64_t kv_len, int64_t P,
+                         float* m, float* l, float* acc, int flags, float scale,
+                         void* out, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * Greedy acceptance ([VC] "Algoritmo Principale", step 3).
+ *   logits  fp32 [B, n_q, V]; drafts int32 [B, n_q - 1] or NULL
+ *   target[b, i] = argmax_v logits[b, i, v] (ties: lowest v; a NaN counts as larger
+ *                  than any number, the first NaN wins)           int32 [B, n_q]
+ *   accept_len[b] = a = first i < n_q-1 with target[b,i] != drafts[b,i], else n_q-1
+ *   commit[b, :] = target[b, 0..a], then -1                        int32 [B, n_q]
+ *   n_commit[b] = a + 1 (a == n_q-1: every draft plus the bonus token)
+ *   err_flag[b] = 1 if row b had a NaN, else 0                    int32 [B] or NULL
+ * With accept_len == commit == n_commit == NULL only target (and err_flag) are written
+ * (the argmax of each draft step) and drafts is not read.  Otherwise all three must be
+ * set and drafts must be non-NULL unless n_q == 1 (no drafts: a = 0).
+ * ---------------------------------------------------------------------------- */
+vc_status vc_accept(const float* logits, const int32_t* drafts, int B, int n_q, int V,
+                    int32_t* target, int32_t* accept_len, int32_t* commit,
+                    int32_t* n_commit, int32_t* err_flag, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * Staging of KV_full from pinned host memory to HBM over PCIe on a side stream
+ * ([VC] "Scaglionamento tra Risorse (P1)" and "Supporto Architetturale": the full
+ * cache lives in CPU memory and verification loads it over PCIe while other
+ * requests draft).  Copies [0, bytes) of src to dst in chunks of chunk_bytes with
+ * one cudaMemcpyAsync each (copy engine, no SMs) and records chunk_done[i] after
+ * chunk i, so a verify call on another stream can wait on exactly its chunk.
+ *   src_host must be page-locked (cudaHostAlloc / cudaHostRegister): checked.
+ *   chunk_done may be NULL (n_events == 0); otherwise n_events >= number of chunks.
+ * ---------------------------------------------------------------------------- */
+vc_status vc_stage_full_kv(void* dst_dev, const void* src_host, size_t bytes,
+                           size_t chunk_bytes, cudaStream_t copy_stream,
+                           cudaEvent_t* chunk_done, int n_events);
+
+/* Host wait on an event with a time limit (polls cudaEventQuery).  Returns VC_OK,
+ * VC_ERR_TIMEOUT after timeout_s seconds, or VC_ERR_CUDA. */
+vc_status vc_event_wait(cudaEvent_t ev, double timeout_s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VERICACHE_H */

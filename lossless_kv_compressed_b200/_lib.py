@@ -1,0 +1,95 @@
+"""ctypes view of libvericache.so (the C ABI in include/vericache.h).
+
+Loading fails loudly: there is no Python or CPU implementation behind these
+names, so a missing library is an ImportError, never a silent fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvericache.so")
+
+VC_OK, VC_ERR_INVALID, VC_ERR_UNSUPPORTED, VC_ERR_CUDA, VC_ERR_TIMEOUT = 0, 1, 2, 3, 4
+VC_CACHE_INDEXED, VC_CACHE_INT4 = 0, 1
+VC_VERIFY_FIRST, VC_VERIFY_LAST = 1, 2
+
+# Every exported symbol, in header order.
+EXPORTS = (
+    "vc_status_string", "vc_last_error", "vc_abi_version",
+    "vc_draft_workspace_size", "vc_draft_attn",
+    "vc_verify_workspace_size", "vc_verify_attn",
+    "vc_accept", "vc_stage_full_kv", "vc_event_wait",
+)
+
+_p = ctypes.c_void_p
+_i32 = ctypes.c_int32
+_i64 = ctypes.c_int64
+_sz = ctypes.c_size_t
+
+
+class CompCache(ctypes.Structure):
+    """Mirror of ``vc_comp_cache``."""
+
+    _fields_ = [
+        ("kind", _i32), ("B", _i32), ("Hq", _i32), ("Hkv", _i32), ("D", _i32),
+        ("S", _i32), ("S_cap", _i32), ("T_cap", _i64),
+        ("k", _p), ("v", _p), ("idx", _p), ("deg", _p),
+        ("kq", _p), ("k_scale", _p), ("k_zero", _p),
+        ("vq", _p), ("v_scale", _p), ("v_zero", _p),
+        ("k_tail", _p), ("v_tail", _p), ("R_cap", _i32), ("n_tail", _i32),
+        ("err_flag", _p),
+    ]
+
+
+class VCError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: {status_name(status)}: {detail}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m lossless_kv_compressed_b200.csrc.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        L.vc_status_string.restype = ctypes.c_char_p
+        L.vc_status_string.argtypes = [ctypes.c_int]
+        L.vc_last_error.restype = ctypes.c_char_p
+        L.vc_last_error.argtypes = []
+        L.vc_abi_version.restype = ctypes.c_int
+        L.vc_draft_workspace_size.restype = _sz
+        L.vc_draft_workspace_size.argtypes = [ctypes.POINTER(CompCache)]
+        L.vc_draft_attn.restype = ctypes.c_int
+        L.vc_draft_attn.argtypes = [_p, ctypes.POINTER(CompCache), ctypes.c_float, _p, _p, _p,
+                                    _sz, _p]
+        L.vc_verify_workspace_size.restype = _sz
+        L.vc_verify_workspace_size.argtypes = [ctypes.c_int] * 5 + [_i64, _i64]
+        L.vc_verify_attn.restype = ctypes.c_int
+        L.vc_verify_attn.argtypes = ([_p] + [ctypes.c_int] * 5 + [_p, _p] + [_i64] * 4
+                                     + [_p, _p, _p, ctypes.c_int, ctypes.c_float, _p, _p, _sz, _p])
+        L.vc_accept.restype = ctypes.c_int
+        L.vc_accept.argtypes = [_p, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _p, _p, _p, _p,
+                                _p, _p]
+        L.vc_stage_full_kv.restype = ctypes.c_int
+        L.vc_stage_full_kv.argtypes = [_p, _p, _sz, _sz, _p, _p, ctypes.c_int]
+        L.vc_event_wait.restype = ctypes.c_int
+        L.vc_event_wait.argtypes = [_p, ctypes.c_double]
+        _lib = L
+    return _lib
+
+
+def status_name(st: int) -> str:
+    return lib().vc_status_string(int(st)).decode()
+
+
+def check(st: int, where: str) -> None:
+    if st != VC_OK:
+        raise VCError(st, where, lib().vc_last_error().decode())

@@ -1,0 +1,41 @@
+// Host-side internals shared by the translation units of the library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "vericache.h"
+
+namespace vc {
+
+// Records a message for vc_last_error() and returns the status.
+vc_status fail(vc_status st, const char* fmt, ...);
+// Number of SMs of the current device (cached per device).
+int num_sms();
+
+#define VC_CUDA(call)                                                                \
+  do {                                                                               \
+    cudaError_t e_ = (call);                                                         \
+    if (e_ != cudaSuccess)                                                           \
+      return ::vc::fail(VC_ERR_CUDA, "%s: %s (%s:%d)", #call, cudaGetErrorString(e_), \
+                        __FILE__, __LINE__);                                         \
+  } while (0)
+
+size_t draft_workspace_bytes(const vc_comp_cache* c);
+vc_status launch_draft_indexed(const void* q, const vc_comp_cache* c, float scale, void* out,
+                               float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
+vc_status launch_draft_int4(const void* q, const vc_comp_cache* c, float scale, void* out,
+                            float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+size_t verify_workspace_bytes(int B, int n_q, int Hq, int Hkv, int D, int64_t kv_start,
+                              int64_t kv_len);
+vc_status launch_verify(const void* q, int B, int n_q, int Hq, int Hkv, int D, const void* k,
+                        const void* v, int64_t L_cap, int64_t kv_start, int64_t kv_len,
+                        int64_t P, float* m, float* l, float* acc, int flags, float scale,
+                        void* out, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+vc_status launch_accept(const float* logits, const int32_t* drafts, int B, int n_q, int V,
+                        int32_t* target, int32_t* accept_len, int32_t* commit,
+                        int32_t* n_commit, int32_t* err_flag, cudaStream_t stream);
+
+}  // namespace vc

@@ -1,0 +1,95 @@
+"""The C ABI library loads, exports every function include/vericache.h declares, and
+rejects bad arguments on the host (these paths make no CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import lossless_kv_compressed_b200 as vc
+from lossless_kv_compressed_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vericache.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vc_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_function():
+    L = vc.lib()
+    names = _declared()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in vericache.h but not exported"
+    assert set(names) == set(_lib.EXPORTS)
+
+
+def test_status_strings_and_version():
+    L = vc.lib()
+    assert L.vc_abi_version() == 1
+    assert _lib.status_name(0) == "VC_OK"
+    assert _lib.status_name(2) == "VC_ERR_UNSUPPORTED"
+    assert _lib.status_name(99) == "VC_UNKNOWN_STATUS"
+
+
+def _cache(**kw):
+    c = _lib.CompCache()
+    c.kind, c.B, c.Hq, c.Hkv, c.D, c.S, c.T_cap = 0, 1, 8, 2, 128, 16, 64
+    c.k = c.v = 1 << 20
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(D=96), _lib.VC_ERR_UNSUPPORTED),
+    (dict(Hq=7), _lib.VC_ERR_INVALID),
+    (dict(Hq=32, Hkv=2), _lib.VC_ERR_UNSUPPORTED),       # g = 16
+    (dict(S=0, n_tail=0), _lib.VC_ERR_INVALID),
+    (dict(n_tail=3), _lib.VC_ERR_INVALID),               # tail pointers missing
+    (dict(k=(1 << 20) + 8), _lib.VC_ERR_INVALID),        # misaligned
+    (dict(S=100, T_cap=64), _lib.VC_ERR_INVALID),        # compact cache larger than base
+    (dict(kind=1, S=40, T_cap=64), _lib.VC_ERR_INVALID), # int4 needs S % 32 == 0
+    (dict(kind=7), _lib.VC_ERR_INVALID),
+])
+def test_draft_rejects_bad_cache(kw, status):
+    c = _cache(**kw)
+    st = vc.lib().vc_draft_attn(1 << 20, ctypes.byref(c), 0.0, 1 << 20, None, 1 << 20, 1 << 20,
+                                None)
+    assert st == status, vc.lib().vc_last_error()
+    assert vc.lib().vc_last_error()
+
+
+def test_draft_rejects_null_cache():
+    assert vc.lib().vc_draft_attn(1 << 20, None, 0.0, 1 << 20, None, 1 << 20, 1, None) == 1
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(D=80), _lib.VC_ERR_UNSUPPORTED),
+    (dict(n_q=0), _lib.VC_ERR_INVALID),
+    (dict(Hq=64, Hkv=4), _lib.VC_ERR_UNSUPPORTED),
+    (dict(n_q=300), _lib.VC_ERR_UNSUPPORTED),           # n_q * g > 1024
+    (dict(kv_len=5000), _lib.VC_ERR_INVALID),           # single pass must cover P + n_q
+    (dict(kv_start=3), _lib.VC_ERR_INVALID),
+])
+def test_verify_rejects_bad_arguments(args, status):
+    a = dict(q=1 << 20, B=1, n_q=9, Hq=8, Hkv=2, D=128, k=1 << 20, v=1 << 20, L_cap=4096,
+             kv_start=0, kv_len=1033, P=1024, m=None, l=None, acc=None, flags=0, scale=0.0,
+             out=1 << 20, ws=1 << 20, ws_bytes=1 << 20, stream=None)
+    a.update(args)
+    st = vc.lib().vc_verify_attn(*a.values())
+    assert st == status, vc.lib().vc_last_error()
+
+
+def test_accept_and_stage_reject_bad_arguments():
+    L = vc.lib()
+    assert L.vc_accept(1 << 20, None, 0, 9, 1024, 1 << 20, None, None, None, None, None) == 1
+    assert L.vc_accept(None, None, 1, 9, 1024, 1 << 20, None, None, None, None, None) == 1
+    assert L.vc_accept(1 << 20, 1 << 20, 1, 9, 1024, 1 << 20, 1 << 20, None, None, None, None) == 1
+    assert L.vc_accept(1 << 20, None, 1, 9, 1024, 1 << 20, 1 << 20, 1 << 20, 1 << 20, None, None) == 1
+    assert L.vc_stage_full_kv(1 << 20, 1 << 20, 100, 0, None, None, 0) == 1
+    assert L.vc_stage_full_kv(None, 1 << 20, 100, 10, None, None, 0) == 1
