@@ -119,18 +119,22 @@ typedef struct vc_comp_cache {
   int32_t* err_flag;
 } vc_comp_cache;
 
+/* Output precision flag shared by the attention calls: write `out` as fp32 instead of
+ * bf16 (the fp32 value is the one the bf16 output is rounded from, to nearest even). */
+#define VC_OUT_F32 4
+
 /* ------------------------------------------------------------------------------
  * Draft attention: one decode step of every query head over KV_comp plus the tail
  * ([VC] "Algoritmo Principale", step 1, with the [CKV] log-degree term):
  *   s_t = (q . k_t) * scale + ln n_t ;  o = sum_t softmax(s)_t v_t
- *   q    bf16 [B, Hq, D]            out  bf16 [B, Hq, D]
+ *   q    bf16 [B, Hq, D]            out  bf16 [B, Hq, D] (fp32 with flags & VC_OUT_F32)
  *   lse  fp32 [B, Hq] or NULL: ln sum_t exp(s_t)
  *   scale <= 0 selects D^-1/2.
  * Split-K over slots: ws must hold vc_draft_workspace_size(cache) bytes (device).
  * S + n_tail must be >= 1.
  * ---------------------------------------------------------------------------- */
 size_t vc_draft_workspace_size(const vc_comp_cache* cache);
-vc_status vc_draft_attn(const void* q, const vc_comp_cache* cache, float scale,
+vc_status vc_draft_attn(const void* q, const vc_comp_cache* cache, float scale, int flags,
                         void* out, float* lse, void* ws, size_t ws_bytes,
                         cudaStream_t stream);
 
@@ -145,10 +149,11 @@ vc_status vc_draft_attn(const void* q, const vc_comp_cache* cache, float scale,
  *         kv_start + r, for r < kv_len (kv_len <= L_cap).  The block's own keys
  *         (positions P .. P+n_q-1) must already be written where they fall.
  *   Single pass (m == l == acc == NULL): kv_start == 0, kv_len == P + n_q; writes out
- *         bf16 [B, n_q, Hq, D].
+ *         bf16 [B, n_q, Hq, D] (fp32 with flags & VC_OUT_F32).
  *   Chunked (long context with KV_full streamed from host memory, [VC] "Supporto
  *         Architetturale"): m, l fp32 [B, n_q, Hq] and acc fp32 [B, n_q, Hq, D] carry
- *         the softmax state (max, sum, weighted values, natural-log domain) between
+ *         the softmax state (running max of s * log2(e), sum of 2^(s*log2(e) - max),
+ *         weighted values) between
  *         calls over consecutive key ranges in increasing kv_start.  VC_VERIFY_FIRST
  *         resets the state before adding this range; VC_VERIFY_LAST writes out after
  *         adding it.  Ranges must tile [0, P + n_q) exactly, in order.
@@ -201,6 +206,11 @@ vc_status vc_stage_full_kv(void* dst_dev, const void* src_host, size_t bytes,
 /* Host wait on an event with a time limit (polls cudaEventQuery).  Returns VC_OK,
  * VC_ERR_TIMEOUT after timeout_s seconds, or VC_ERR_CUDA. */
 vc_status vc_event_wait(cudaEvent_t ev, double timeout_s);
+
+/* The library's device error word on the current device (synchronous read; clear != 0
+ * resets it).  Bit 0: a bounded wait inside a verify-attention CTA expired (the call's
+ * output is then invalid; the CTA released its resources and exited). */
+vc_status vc_device_error(int32_t* value, int clear);
 
 #ifdef __cplusplus
 }

@@ -14,13 +14,14 @@ LIB_PATH = os.path.join(_HERE, "libvericache.so")
 VC_OK, VC_ERR_INVALID, VC_ERR_UNSUPPORTED, VC_ERR_CUDA, VC_ERR_TIMEOUT = 0, 1, 2, 3, 4
 VC_CACHE_INDEXED, VC_CACHE_INT4 = 0, 1
 VC_VERIFY_FIRST, VC_VERIFY_LAST = 1, 2
+VC_OUT_F32 = 4
 
 # Every exported symbol, in header order.
 EXPORTS = (
     "vc_status_string", "vc_last_error", "vc_abi_version",
     "vc_draft_workspace_size", "vc_draft_attn",
     "vc_verify_workspace_size", "vc_verify_attn",
-    "vc_accept", "vc_stage_full_kv", "vc_event_wait",
+    "vc_accept", "vc_stage_full_kv", "vc_event_wait", "vc_device_error",
 )
 
 _p = ctypes.c_void_p
@@ -68,8 +69,8 @@ def lib() -> ctypes.CDLL:
         L.vc_draft_workspace_size.restype = _sz
         L.vc_draft_workspace_size.argtypes = [ctypes.POINTER(CompCache)]
         L.vc_draft_attn.restype = ctypes.c_int
-        L.vc_draft_attn.argtypes = [_p, ctypes.POINTER(CompCache), ctypes.c_float, _p, _p, _p,
-                                    _sz, _p]
+        L.vc_draft_attn.argtypes = [_p, ctypes.POINTER(CompCache), ctypes.c_float, ctypes.c_int,
+                                    _p, _p, _p, _sz, _p]
         L.vc_verify_workspace_size.restype = _sz
         L.vc_verify_workspace_size.argtypes = [ctypes.c_int] * 5 + [_i64, _i64]
         L.vc_verify_attn.restype = ctypes.c_int
@@ -82,6 +83,8 @@ def lib() -> ctypes.CDLL:
         L.vc_stage_full_kv.argtypes = [_p, _p, _sz, _sz, _p, _p, ctypes.c_int]
         L.vc_event_wait.restype = ctypes.c_int
         L.vc_event_wait.argtypes = [_p, ctypes.c_double]
+        L.vc_device_error.restype = ctypes.c_int
+        L.vc_device_error.argtypes = [ctypes.POINTER(_i32), ctypes.c_int]
         _lib = L
     return _lib
 

@@ -132,19 +132,28 @@ def draft_workspace_size(cache) -> int:
     return int(n)
 
 
+def _out_flag(out: torch.Tensor) -> int:
+    if out.dtype == torch.float32:
+        return _lib.VC_OUT_F32
+    if out.dtype != torch.bfloat16:
+        raise TypeError("out must be bfloat16 or float32")
+    return 0
+
+
 def draft_attn(q: torch.Tensor, cache, out: Optional[torch.Tensor] = None,
                lse: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
                scale: float = 0.0, stream=None) -> torch.Tensor:
-    """o[b, h] = softmax_t(q.k_t * scale + ln n_t) . v over KV_comp plus the tail."""
+    """o[b, h] = softmax_t(q.k_t * scale + ln n_t) . v over KV_comp plus the tail.
+    ``out`` may be bfloat16 (default) or float32."""
     _need(q, torch.bfloat16, "q")
     s = cache.struct()
     if out is None:
         out = torch.empty_like(q)
     if ws is None:
         ws = torch.empty(draft_workspace_size(cache), dtype=torch.uint8, device=q.device)
-    check(lib().vc_draft_attn(q.data_ptr(), ctypes.byref(s), float(scale), out.data_ptr(),
-                              _ptr(lse), ws.data_ptr(), ws.numel(), _stream(stream)),
-          "vc_draft_attn")
+    check(lib().vc_draft_attn(q.data_ptr(), ctypes.byref(s), float(scale), _out_flag(out),
+                              out.data_ptr(), _ptr(lse), ws.data_ptr(), ws.numel(),
+                              _stream(stream)), "vc_draft_attn")
     return out
 
 
@@ -158,7 +167,8 @@ def verify_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, P: int, kv_st
                 out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
                 scale: float = 0.0, stream=None) -> torch.Tensor:
     """Verify attention of q [B, n_q, Hq, D] over keys [kv_start, kv_start+kv_len) held
-    in k, v [B, Hkv, L_cap, D]; ``state`` = (m, l, acc) for the chunked form."""
+    in k, v [B, Hkv, L_cap, D]; ``state`` = (m, l, acc) for the chunked form.
+    ``out`` may be bfloat16 (default) or float32."""
     _need(q, torch.bfloat16, "q")
     _need(k, torch.bfloat16, "k")
     _need(v, torch.bfloat16, "v")
@@ -176,6 +186,8 @@ def verify_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, P: int, kv_st
     if ws is None:
         ws = torch.empty(max(1, verify_workspace_size(B, n_q, Hq, Hkv, D, kv_start, kv_len)),
                          dtype=torch.uint8, device=q.device)
+    if out is not None:
+        flags |= _out_flag(out)
     check(lib().vc_verify_attn(q.data_ptr(), B, n_q, Hq, Hkv, D, k.data_ptr(), v.data_ptr(),
                                L_cap, kv_start, kv_len, P, _ptr(m), _ptr(l), _ptr(acc),
                                int(flags), float(scale), _ptr(out), ws.data_ptr(), ws.numel(),
@@ -238,3 +250,10 @@ def stage_full_kv(dst: torch.Tensor, src_pinned: torch.Tensor, chunk_bytes: int,
 
 def event_wait(event, timeout_s: float) -> None:
     check(lib().vc_event_wait(event.cuda_event, float(timeout_s)), "vc_event_wait")
+
+
+def device_error(clear: bool = True) -> int:
+    """The library's device error word (bit 0: a bounded wait in verify expired)."""
+    v = ctypes.c_int32(0)
+    check(lib().vc_device_error(ctypes.byref(v), int(clear)), "vc_device_error")
+    return int(v.value)

@@ -109,17 +109,18 @@ size_t vc_draft_workspace_size(const vc_comp_cache* cache) {
   return draft_workspace_bytes(cache);
 }
 
-vc_status vc_draft_attn(const void* q, const vc_comp_cache* cache, float scale, void* out,
-                        float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+vc_status vc_draft_attn(const void* q, const vc_comp_cache* cache, float scale, int flags,
+                        void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
   vc_status st = check_cache(cache);
   if (st != VC_OK) return st;
   if (!q || !out || !ws) return fail(VC_ERR_INVALID, "draft: q / out / ws NULL");
   if (!aligned16(q) || !aligned16(out) || !aligned16(ws))
     return fail(VC_ERR_INVALID, "draft: q / out / ws misaligned");
   if (scale <= 0.f) scale = 1.0f / sqrtf((float)cache->D);
+  if (flags & ~VC_OUT_F32) return fail(VC_ERR_INVALID, "draft: unknown flags");
   if (cache->kind == VC_CACHE_INDEXED)
-    return launch_draft_indexed(q, cache, scale, out, lse, ws, ws_bytes, stream);
-  return launch_draft_int4(q, cache, scale, out, lse, ws, ws_bytes, stream);
+    return launch_draft_indexed(q, cache, scale, flags, out, lse, ws, ws_bytes, stream);
+  return launch_draft_int4(q, cache, scale, flags, out, lse, ws, ws_bytes, stream);
 }
 
 size_t vc_verify_workspace_size(int B, int n_q, int Hq, int Hkv, int D, int64_t kv_start,
@@ -143,6 +144,8 @@ vc_status vc_verify_attn(const void* q, int B, int n_q, int Hq, int Hkv, int D, 
     return fail(VC_ERR_INVALID, "verify: misaligned pointer");
   if (kv_start < 0 || kv_len <= 0 || kv_len > L_cap || P < 0)
     return fail(VC_ERR_INVALID, "verify: bad key range");
+  if (flags & ~(VC_VERIFY_FIRST | VC_VERIFY_LAST | VC_OUT_F32))
+    return fail(VC_ERR_INVALID, "verify: unknown flags");
   const bool chunked = m || l || acc;
   if (chunked) {
     if (!m || !l || !acc) return fail(VC_ERR_INVALID, "verify: m, l, acc must all be set");
@@ -156,7 +159,7 @@ vc_status vc_verify_attn(const void* q, int B, int n_q, int Hq, int Hkv, int D, 
     if (kv_start != 0 || kv_len != P + n_q)
       return fail(VC_ERR_INVALID, "verify: single pass needs kv_start 0, kv_len P + n_q");
     if (!out) return fail(VC_ERR_INVALID, "verify: out NULL");
-    flags = VC_VERIFY_FIRST | VC_VERIFY_LAST;
+    flags = (flags & VC_OUT_F32) | VC_VERIFY_FIRST | VC_VERIFY_LAST;
   }
   if (out && !aligned16(out)) return fail(VC_ERR_INVALID, "verify: out misaligned");
   if (scale <= 0.f) scale = 1.0f / sqrtf((float)D);
@@ -184,5 +187,7 @@ vc_status vc_stage_full_kv(void* dst_dev, const void* src_host, size_t bytes, si
 }
 
 vc_status vc_event_wait(cudaEvent_t ev, double timeout_s) { return event_wait(ev, timeout_s); }
+
+vc_status vc_device_error(int32_t* value, int clear) { return read_device_error(value, clear); }
 
 }  // extern "C"

@@ -258,11 +258,11 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
 }
 
 // Fixed-order merge of the split partials of every head -> bf16 output (+ lse).
-template <int D>
+template <int D, typename OutT>
 __global__ void __launch_bounds__(256) draft_combine_kernel(const float* __restrict__ ws_o,
                                                             const float* __restrict__ ws_ml,
                                                             int n_split, int g, int Hkv, int Hq,
-                                                            __nv_bfloat16* __restrict__ out,
+                                                            OutT* __restrict__ out,
                                                             float* __restrict__ lse) {
   const int pair = blockIdx.x;
   const int b = pair / Hkv, j = pair - b * Hkv;
@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(256) draft_combine_kernel(const float* __restr
       O = fmaf(ws_o[pr * D + d], f, O);
     }
     const int64_t h = (int64_t)b * Hq + j * g + r;
-    out[h * D + d] = __float2bfloat16_rn(O / L);
+    store_out(out + h * D + d, O / L);
     if (lse && d == 0) lse[h] = (M + __log2f(L)) * kLn2;
   }
 }
@@ -314,8 +314,20 @@ size_t draft_workspace_bytes(const vc_comp_cache* c) {
   return (size_t)pairs * n_split * g * ((size_t)c->D + 2) * sizeof(float) + 256;
 }
 
-vc_status launch_draft_indexed(const void* q, const vc_comp_cache* c, float scale, void* out,
-                               float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+template <int D>
+static void launch_draft_combine(const DraftIndexedParams& p, int pairs, int flags, void* out,
+                                 float* lse, cudaStream_t stream) {
+  if (flags & VC_OUT_F32)
+    draft_combine_kernel<D, float><<<pairs, 256, 0, stream>>>(
+        p.ws_o, p.ws_ml, p.n_split, p.g, p.Hkv, p.Hq, static_cast<float*>(out), lse);
+  else
+    draft_combine_kernel<D, __nv_bfloat16><<<pairs, 256, 0, stream>>>(
+        p.ws_o, p.ws_ml, p.n_split, p.g, p.Hkv, p.Hq, static_cast<__nv_bfloat16*>(out), lse);
+}
+
+vc_status launch_draft_indexed(const void* q, const vc_comp_cache* c, float scale, int flags,
+                               void* out, float* lse, void* ws, size_t ws_bytes,
+                               cudaStream_t stream) {
   const int pairs = c->B * c->Hkv;
   const int total = c->S + c->n_tail;
   DraftIndexedParams p;
@@ -348,16 +360,14 @@ vc_status launch_draft_indexed(const void* q, const vc_comp_cache* c, float scal
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
     draft_indexed_kernel<128, kNStage><<<grid, 128, sm, stream>>>(p);
     VC_CUDA(cudaGetLastError());
-    draft_combine_kernel<128><<<pairs, 256, 0, stream>>>(
-        p.ws_o, p.ws_ml, p.n_split, p.g, p.Hkv, p.Hq, static_cast<__nv_bfloat16*>(out), lse);
+    launch_draft_combine<128>(p, pairs, flags, out, lse, stream);
   } else {
     const size_t sm = draft_indexed_smem<64>(p.chunk);
     VC_CUDA(cudaFuncSetAttribute(draft_indexed_kernel<64, kNStage>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
     draft_indexed_kernel<64, kNStage><<<grid, 128, sm, stream>>>(p);
     VC_CUDA(cudaGetLastError());
-    draft_combine_kernel<64><<<pairs, 256, 0, stream>>>(
-        p.ws_o, p.ws_ml, p.n_split, p.g, p.Hkv, p.Hq, static_cast<__nv_bfloat16*>(out), lse);
+    launch_draft_combine<64>(p, pairs, flags, out, lse, stream);
   }
   VC_CUDA(cudaGetLastError());
   return VC_OK;
@@ -366,8 +376,8 @@ vc_status launch_draft_indexed(const void* q, const vc_comp_cache* c, float scal
 }  // namespace vc
 
 namespace vc {
-vc_status launch_draft_int4(const void*, const vc_comp_cache*, float, void*, float*, void*, size_t,
-                            cudaStream_t) {
+vc_status launch_draft_int4(const void*, const vc_comp_cache*, float, int, void*, float*, void*,
+                            size_t, cudaStream_t) {
   return fail(VC_ERR_UNSUPPORTED, "int4 draft attention not built yet");
 }
 }  // namespace vc

@@ -22,10 +22,12 @@ int num_sms();
   } while (0)
 
 size_t draft_workspace_bytes(const vc_comp_cache* c);
-vc_status launch_draft_indexed(const void* q, const vc_comp_cache* c, float scale, void* out,
-                               float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
-vc_status launch_draft_int4(const void* q, const vc_comp_cache* c, float scale, void* out,
-                            float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
+vc_status launch_draft_indexed(const void* q, const vc_comp_cache* c, float scale, int flags,
+                               void* out, float* lse, void* ws, size_t ws_bytes,
+                               cudaStream_t stream);
+vc_status launch_draft_int4(const void* q, const vc_comp_cache* c, float scale, int flags,
+                            void* out, float* lse, void* ws, size_t ws_bytes,
+                            cudaStream_t stream);
 
 size_t verify_workspace_bytes(int B, int n_q, int Hq, int Hkv, int D, int64_t kv_start,
                               int64_t kv_len);
@@ -33,6 +35,8 @@ vc_status launch_verify(const void* q, int B, int n_q, int Hq, int Hkv, int D, c
                         const void* v, int64_t L_cap, int64_t kv_start, int64_t kv_len,
                         int64_t P, float* m, float* l, float* acc, int flags, float scale,
                         void* out, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+vc_status read_device_error(int32_t* value, int clear);
 
 vc_status launch_accept(const float* logits, const int32_t* drafts, int B, int n_q, int V,
                         int32_t* target, int32_t* accept_len, int32_t* commit,

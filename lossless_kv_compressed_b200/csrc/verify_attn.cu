@@ -1,14 +1,546 @@
-// Verify attention (placeholder until the tcgen05 kernel lands).
+// Verify attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// VeriCache summary ("Riepilogo Tecnico: VeriCache", section "Algoritmo Principale",
+// step 2): one forward pass over the full cache KV_full checks all k drafted tokens in
+// parallel.  Query row (i, h) of a (batch, kv head) pair -- block position i in
+// [0, n_q), head h of the GQA group -- sits at absolute position P + i and attends every
+// key at position <= P + i: the whole prefix plus the block, causal inside the block.
+//
+// Decomposition.  A CTA owns one pair, one group of <= 256 query rows (two M = 128
+// UMMA tiles; row r = i * g + h) and one split of the keys: the intersection of the
+// call's key range with an absolute window [s * 4096, (s + 1) * 4096).  Split windows
+// and 64-key tiles sit at fixed absolute positions, so a row's result does not depend
+// on n_q or on the other rows (a verify row equals the same token decoded alone).
+//
+// Per CTA (384 threads):
+//   warp 0      TMA producer: K and V tiles [64 keys x D] (128-byte swizzle) into a
+//               2-stage ring, one mbarrier per stage with the transaction byte count.
+//   warp 1      TMEM allocator and UMMA issuer (one thread): S = Q K^T into TMEM per
+//               M-tile, then O += P V with P from shared memory and V as an N-major B.
+//   warps 4-7   softmax of M-tile 0, warps 8-11 of M-tile 1: one thread per query row
+//               (TMEM lane), scores in the log2 domain, running max kept unless it grows
+//               by more than 2^8 (then O in TMEM is rescaled after the previous P.V),
+//               P written as bf16 into a double-buffered 128-byte-swizzled tile.
+// TMEM columns: S0 [0,64), S1 [64,128), O0 [128,128+D), O1 [128+D,128+2D).
+// Every mbarrier wait is bounded in time; on expiry the CTA raises the library's device
+// error word, releases TMEM and exits.
+// The split partials (max, sum, unnormalised O) are merged by a second kernel in
+// split order, optionally together with a carried state for chunked (streamed) keys.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "tc05.cuh"
+#include "vc_common.cuh"
 #include "vc_internal.h"
 
 namespace vc {
 
-size_t verify_workspace_bytes(int, int, int, int, int, int64_t, int64_t) { return 256; }
+__device__ int g_vc_dev_error;   // bit 0: a bounded wait in the verify kernel expired
 
-vc_status launch_verify(const void*, int, int, int, int, int, const void*, const void*, int64_t,
-                        int64_t, int64_t, int64_t, float*, float*, float*, int, float, void*,
-                        void*, size_t, cudaStream_t) {
-  return fail(VC_ERR_UNSUPPORTED, "verify attention not built yet");
+constexpr int kSplitKeys = 4096;
+constexpr int kBN = 64;
+constexpr int kVThreads = 384;
+constexpr int kNSt = 2;
+constexpr float kRescaleLog2 = 8.f;
+
+struct VerifyParams {
+  const __nv_bfloat16* q;   // [B, n_q, Hq, D]
+  int n_q, Hq, Hkv, g, R;   // R = n_q * g rows per pair
+  int64_t kv_start, kv_len, P;
+  int split0, n_split;
+  float qk_scale2;          // scale * log2(e)
+  float* ws_o;              // [pairs, n_split, R, D]
+  float* ws_ml;             // [pairs, n_split, R, 2]
+};
+
+template <int D>
+struct VLayout {
+  static constexpr int kQTile = 128 * D * 2;
+  static constexpr int kKVTile = kBN * D * 2;
+  static constexpr int kPTile = 128 * kBN * 2;
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + 2 * kQTile;
+  static constexpr int kV = kK + kNSt * kKVTile;
+  static constexpr int kP = kV + kNSt * kKVTile;
+  static constexpr int kBar = kP + 4 * kPTile;
+  static constexpr int kNBar = 2 * kNSt + 2 + 2 + 4 + 4 + 1;
+  static constexpr int kTmemSlot = kBar + kNBar * 8;
+  static constexpr int kAbort = kTmemSlot + 4;
+  static constexpr int kTotal = kAbort + 4;
+  static constexpr int kAlloc = kTotal + 1024;
+  static constexpr uint32_t kTmemCols = (128 + 2 * D) <= 256 ? 256 : 512;
+  static_assert(kQTile % 1024 == 0 && kKVTile % 1024 == 0 && kPTile % 1024 == 0, "align");
+};
+
+template <int D>
+__global__ void __launch_bounds__(kVThreads, 1)
+    verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const VerifyParams p) {
+  using L = VLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int s_local = blockIdx.x, rg = blockIdx.y, pair = blockIdx.z;
+  const int b = pair / p.Hkv, kvh = pair - b * p.Hkv;
+  const int row0 = rg * 256;
+  const int rows_here = min(256, p.R - row0);
+  const int n_mt = (rows_here + 127) >> 7;
+  const int64_t part = (int64_t)pair * p.n_split + s_local;
+
+  // key range of this split seen by this row group
+  const int64_t win = (int64_t)(p.split0 + s_local) * kSplitKeys;
+  const int64_t a0 = max(p.kv_start, win);
+  int64_t a1 = min(p.kv_start + p.kv_len, win + kSplitKeys);
+  a1 = min(a1, p.P + (row0 + rows_here - 1) / p.g + 1);
+  const int n_tiles = a1 > a0 ? (int)((a1 - 1) / kBN - a0 / kBN + 1) : 0;
+  const int64_t tile0 = a0 / kBN;
+
+  if (n_tiles == 0) {  // nothing visible: empty partials
+    for (int rr = threadIdx.x; rr < rows_here; rr += blockDim.x) {
+      const int64_t o = part * p.R + row0 + rr;
+      p.ws_ml[o * 2] = -INFINITY;
+      p.ws_ml[o * 2 + 1] = 0.f;
+      for (int d = 0; d < D; ++d) p.ws_o[o * D + d] = 0.f;
+    }
+    return;
+  }
+
+  auto bar = [&](int i) -> uint32_t { return sb + L::kBar + 8 * i; };
+  auto b_kv_full = [&](int st) { return bar(st); };
+  auto b_kv_empty = [&](int st) { return bar(kNSt + st); };
+  auto b_s_full = [&](int mt) { return bar(2 * kNSt + mt); };
+  auto b_s_free = [&](int mt) { return bar(2 * kNSt + 2 + mt); };
+  auto b_p_full = [&](int mt, int buf) { return bar(2 * kNSt + 4 + mt * 2 + buf); };
+  auto b_o_done = [&](int mt, int buf) { return bar(2 * kNSt + 8 + mt * 2 + buf); };
+  const uint32_t b_teardown = bar(2 * kNSt + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+
+  auto nw_active = [&](int mt) {
+    const int v = min(128, rows_here - mt * 128);
+    return v > 0 ? (v + 31) >> 5 : 0;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kNSt; ++st) {
+      tc::mbar_init(b_kv_full(st), 1);
+      tc::mbar_init(b_kv_empty(st), 1);
+    }
+    for (int mt = 0; mt < 2; ++mt) {
+      tc::mbar_init(b_s_full(mt), 1);
+      tc::mbar_init(b_s_free(mt), max(1, nw_active(mt)));
+      for (int buf = 0; buf < 2; ++buf) {
+        tc::mbar_init(b_p_full(mt, buf), max(1, nw_active(mt)));
+        tc::mbar_init(b_o_done(mt, buf), 1);
+      }
+    }
+    tc::mbar_init(b_teardown, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) tc::tmem_alloc(sb + L::kTmemSlot, L::kTmemCols);
+
+  // Q rows of this group -> shared memory (K-major, 128-byte swizzle); padding rows 0.
+  for (int c = threadIdx.x; c < n_mt * 128 * (D / 8); c += kVThreads) {
+    const int rr = c / (D / 8), ch = c - rr * (D / 8);
+    const int mt = rr >> 7, r = rr & 127;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (rr < rows_here) {
+      const int grow = row0 + rr;
+      const int i = grow / p.g, hl = grow - i * p.g;
+      const uint4* src = reinterpret_cast<const uint4*>(
+          p.q + (((int64_t)b * p.n_q + i) * p.Hq + kvh * p.g + hl) * D);
+      val = __ldg(src + ch);
+    }
+    const int cb = ch >> 3, cc = ch & 7;
+    *reinterpret_cast<uint4*>(smem + L::kQ + mt * L::kQTile + cb * (128 * 128) + r * 128 +
+                              ((cc ^ (r & 7)) << 4)) = val;
+  }
+  tc::fence_proxy_async();
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlot);
+
+  auto raise = [&]() {
+    *abort_flag = 1;
+    atomicOr(&g_vc_dev_error, 1);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tc::prefetch_tmap(&tmK);
+      tc::prefetch_tmap(&tmV);
+      int issued = 0;
+      for (int t = 0; t < n_tiles; ++t) {
+        const int st = t % kNSt;
+        if (t >= kNSt && !tc::mbar_wait(b_kv_empty(st), ((t / kNSt) - 1) & 1, abort_flag)) {
+          raise();
+          break;
+        }
+        const uint32_t fb = b_kv_full(st);
+        tc::mbar_expect_tx(fb, 2 * L::kKVTile);
+        const int y = (int)((tile0 + t) * kBN - p.kv_start);
+#pragma unroll
+        for (int cb = 0; cb < D / 64; ++cb) {
+          tc::tma_load_3d(sb + L::kK + st * L::kKVTile + cb * (kBN * 128), &tmK, fb, cb * 64, y,
+                          pair);
+          tc::tma_load_3d(sb + L::kV + st * L::kKVTile + cb * (kBN * 128), &tmV, fb, cb * 64, y,
+                          pair);
+        }
+        issued = t + 1;
+      }
+      // loads still in flight must land before shared memory is released
+      for (int t = max(0, issued - kNSt); t < issued; ++t)
+        tc::mbar_wait(b_kv_full(t % kNSt), (t / kNSt) & 1, nullptr, 1000000000ull);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      const uint32_t id_qk = tc::idesc_bf16_f32(128, kBN, false);
+      const uint32_t id_pv = tc::idesc_bf16_f32(128, D, true);
+      auto qk = [&](int t, int mt) {
+        const int st = t % kNSt;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t a = sb + L::kQ + mt * L::kQTile + (ks >> 2) * (128 * 128) + (ks & 3) * 32;
+          const uint32_t bb = sb + L::kK + st * L::kKVTile + (ks >> 2) * (kBN * 128) + (ks & 3) * 32;
+          tc::umma_ss(tmem + mt * kBN, tc::sdesc_sw128(a, 16, 1024), tc::sdesc_sw128(bb, 16, 1024),
+                      id_qk, ks > 0 ? 1u : 0u);
+        }
+      };
+      auto pv = [&](int t, int mt) {
+        const int st = t % kNSt, buf = t & 1;
+#pragma unroll
+        for (int ks = 0; ks < kBN / 16; ++ks) {
+          const uint32_t a = sb + L::kP + (mt * 2 + buf) * L::kPTile + ks * 32;
+          const uint32_t bb = sb + L::kV + st * L::kKVTile + ks * 16 * 128;
+          tc::umma_ss(tmem + 128 + mt * D, tc::sdesc_sw128(a, 16, 1024),
+                      tc::sdesc_sw128(bb, kBN * 128, 1024), id_pv, (t > 0 || ks > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = tc::mbar_wait(b_kv_full(0), 0, abort_flag);
+      if (ok) {
+        tc::tc_fence_after();
+        for (int mt = 0; mt < n_mt; ++mt) {
+          qk(0, mt);
+          tc::umma_commit(b_s_full(mt));
+        }
+      }
+      for (int t = 0; ok && t < n_tiles; ++t) {
+        const bool next = t + 1 < n_tiles;
+        if (next && !(ok = tc::mbar_wait(b_kv_full((t + 1) % kNSt), ((t + 1) / kNSt) & 1,
+                                         abort_flag)))
+          break;
+        for (int mt = 0; mt < n_mt && ok; ++mt) {
+          if (next) {
+            if (!(ok = tc::mbar_wait(b_s_free(mt), t & 1, abort_flag))) break;
+            tc::tc_fence_after();
+            qk(t + 1, mt);
+            tc::umma_commit(b_s_full(mt));
+          }
+          if (!(ok = tc::mbar_wait(b_p_full(mt, t & 1), (t >> 1) & 1, abort_flag))) break;
+          tc::tc_fence_after();
+          pv(t, mt);
+          tc::umma_commit(b_o_done(mt, t & 1));
+        }
+        if (!ok) break;
+        tc::umma_commit(b_kv_empty(t % kNSt));
+      }
+      if (!ok) raise();
+      // every UMMA issued must retire before TMEM is released
+      tc::umma_commit(b_teardown);
+      tc::mbar_wait(b_teardown, 0, nullptr, 1000000000ull);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax
+    const int mt = (warp - 4) >> 2, q4 = warp & 3;
+    const int valid_mt = min(128, rows_here - mt * 128);
+    if (mt < n_mt && 32 * q4 < valid_mt) {
+      const int r = 32 * q4 + lane;
+      const int grow = row0 + mt * 128 + r;
+      const bool row_ok = grow < p.R;
+      const int64_t limit = row_ok ? p.P + grow / p.g : (int64_t)-1;
+      const uint32_t s_t = tmem + ((uint32_t)(32 * q4) << 16) + mt * kBN;
+      const uint32_t o_t = tmem + ((uint32_t)(32 * q4) << 16) + 128 + mt * D;
+      float m_used = -INFINITY, lsum = 0.f;
+      bool ok = true;
+      for (int t = 0; t < n_tiles; ++t) {
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(b_s_full(mt), t & 1, abort_flag));
+        if (!ok) break;
+        tc::tc_fence_after();
+        uint32_t sr[64];
+        tc::tmem_ld32(s_t, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tc::tmem_ld32(s_t + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tc::tmem_wait_ld();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(b_s_free(mt));
+        const int64_t key0 = (tile0 + t) * kBN;
+        const int64_t lo = a0 - key0, hi = min(a1 - 1, limit) - key0;   // visible j in [lo, hi]
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const float v = (j >= lo && j <= hi) ? __uint_as_float(sr[j]) * p.qk_scale2 : -INFINITY;
+          sr[j] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+        const float m_new = fmaxf(m_used, mx);
+        const bool resc = m_new > m_used + kRescaleLog2;
+        if (t > 0 && __any_sync(0xffffffffu, resc)) {
+          ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt, (t - 1) & 1),
+                                                     ((t - 1) >> 1) & 1, abort_flag));
+          if (!ok) break;
+          tc::tc_fence_after();
+          const float alpha = resc ? ex2(m_used - m_new) : 1.f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tc::tmem_ld32(o_t + 32 * c, o);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tc::tmem_st32(o_t + 32 * c, o);
+          }
+          tc::tmem_wait_st();
+          lsum *= alpha;
+        }
+        if (resc) m_used = m_new;
+        const float m_safe = m_used == -INFINITY ? 0.f : m_used;
+        if (t >= 2) {
+          ok = __all_sync(0xffffffffu,
+                          tc::mbar_wait(b_o_done(mt, t & 1), ((t - 2) >> 1) & 1, abort_flag));
+          if (!ok) break;
+        }
+        uint8_t* prow = smem + L::kP + (mt * 2 + (t & 1)) * L::kPTile + r * 128;
+        float rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float e[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            e[u] = ex2(__uint_as_float(sr[8 * c + u]) - m_safe);
+            rs += e[u];
+          }
+          uint4 pk;
+          pk.x = pack_bf16x2(e[0], e[1]);
+          pk.y = pack_bf16x2(e[2], e[3]);
+          pk.z = pack_bf16x2(e[4], e[5]);
+          pk.w = pack_bf16x2(e[6], e[7]);
+          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = pk;
+        }
+        lsum += rs;
+        tc::fence_proxy_async();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(b_p_full(mt, t & 1));
+      }
+      if (ok) {
+        const int tl = n_tiles - 1;
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt, tl & 1), (tl >> 1) & 1,
+                                                   abort_flag));
+      }
+      if (!ok) {
+        raise();
+      } else {
+        tc::tc_fence_after();
+        const int64_t o_row = part * p.R + grow;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tc::tmem_ld32(o_t + 32 * c, o);
+          tc::tmem_wait_ld();
+          if (row_ok) {
+            float4* dst = reinterpret_cast<float4*>(p.ws_o + o_row * D + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                   __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+          }
+        }
+        if (row_ok) {
+          p.ws_ml[o_row * 2] = m_used;
+          p.ws_ml[o_row * 2 + 1] = lsum;
+        }
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// Merge split partials in split order (plus the carried state) for one query row.
+template <int D, typename OutT>
+__global__ void __launch_bounds__(D) verify_combine_kernel(
+    const float* __restrict__ ws_o, const float* __restrict__ ws_ml, int n_split, int R, int g,
+    int n_q, int Hq, int Hkv, int flags, float* m_state, float* l_state, float* acc_state,
+    OutT* __restrict__ out) {
+  const int pair = blockIdx.x / R, row = blockIdx.x - pair * R;
+  const int d = threadIdx.x;
+  const int i = row / g, hl = row - i * g;
+  const int b = pair / Hkv, kvh = pair - b * Hkv;
+  const int64_t sidx = ((int64_t)b * n_q + i) * Hq + kvh * g + hl;
+  const bool carry = m_state != nullptr && !(flags & VC_VERIFY_FIRST);
+  float cm = -INFINITY, cl = 0.f, co = 0.f;
+  if (carry) {
+    cm = m_state[sidx];
+    cl = l_state[sidx];
+    co = acc_state[sidx * D + d];
+  }
+  __syncthreads();
+  float M = cm;
+  for (int s = 0; s < n_split; ++s)
+    M = fmaxf(M, ws_ml[(((int64_t)pair * n_split + s) * R + row) * 2]);
+  float Ls = 0.f, O = 0.f;
+  if (cm > -INFINITY) {
+    const float f = ex2(cm - M);
+    Ls = cl * f;
+    O = co * f;
+  }
+  for (int s = 0; s < n_split; ++s) {
+    const int64_t pr = ((int64_t)pair * n_split + s) * R + row;
+    const float ms = ws_ml[pr * 2];
+    if (ms > -INFINITY) {
+      const float f = ex2(ms - M);
+      Ls = fmaf(ws_ml[pr * 2 + 1], f, Ls);
+      O = fmaf(ws_o[pr * D + d], f, O);
+    }
+  }
+  if (flags & VC_VERIFY_LAST) {
+    store_out(out + sidx * D + d, O / Ls);
+  } else {
+    acc_state[sidx * D + d] = O;
+    if (d == 0) {
+      m_state[sidx] = M;
+      l_state[sidx] = Ls;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// [pairs][L_cap][D] bf16 viewed as a 3-D tensor whose key extent is kv_len, so rows past
+// the live range (and negative rows) read as zero.
+bool make_kv_map(CUtensorMap* m, const void* base, int D, int64_t kv_len, int64_t L_cap,
+                 int pairs) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)kv_len, (cuuint64_t)pairs};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)L_cap * D * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)kBN, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Plan {
+  int pairs, g, R, split0, n_split, n_rg;
+  size_t ws_bytes;
+};
+
+Plan plan(int B, int n_q, int Hq, int Hkv, int D, int64_t kv_start, int64_t kv_len) {
+  Plan pl;
+  pl.pairs = B * Hkv;
+  pl.g = Hq / Hkv;
+  pl.R = n_q * pl.g;
+  pl.split0 = (int)(kv_start / kSplitKeys);
+  pl.n_split = (int)((kv_start + kv_len - 1) / kSplitKeys) - pl.split0 + 1;
+  pl.n_rg = (pl.R + 255) / 256;
+  pl.ws_bytes = (size_t)pl.pairs * pl.n_split * pl.R * ((size_t)D + 2) * sizeof(float);
+  return pl;
+}
+
+}  // namespace
+
+size_t verify_workspace_bytes(int B, int n_q, int Hq, int Hkv, int D, int64_t kv_start,
+                              int64_t kv_len) {
+  return plan(B, n_q, Hq, Hkv, D, kv_start, kv_len).ws_bytes + 256;
+}
+
+template <int D>
+static vc_status run_verify(const Plan& pl, const VerifyParams& vp, const CUtensorMap& mk,
+                            const CUtensorMap& mv, int flags, float* m, float* l, float* acc,
+                            void* out, cudaStream_t stream) {
+  using L = VLayout<D>;
+  VC_CUDA(cudaFuncSetAttribute(verify_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               L::kAlloc));
+  dim3 grid(pl.n_split, pl.n_rg, pl.pairs);
+  verify_kernel<D><<<grid, kVThreads, L::kAlloc, stream>>>(mk, mv, vp);
+  VC_CUDA(cudaGetLastError());
+  if (flags & VC_OUT_F32)
+    verify_combine_kernel<D, float><<<pl.pairs * pl.R, D, 0, stream>>>(
+        vp.ws_o, vp.ws_ml, pl.n_split, pl.R, pl.g, vp.n_q, vp.Hq, vp.Hkv, flags, m, l, acc,
+        static_cast<float*>(out));
+  else
+    verify_combine_kernel<D, __nv_bfloat16><<<pl.pairs * pl.R, D, 0, stream>>>(
+        vp.ws_o, vp.ws_ml, pl.n_split, pl.R, pl.g, vp.n_q, vp.Hq, vp.Hkv, flags, m, l, acc,
+        static_cast<__nv_bfloat16*>(out));
+  VC_CUDA(cudaGetLastError());
+  return VC_OK;
+}
+
+vc_status launch_verify(const void* q, int B, int n_q, int Hq, int Hkv, int D, const void* k,
+                        const void* v, int64_t L_cap, int64_t kv_start, int64_t kv_len,
+                        int64_t P, float* m, float* l, float* acc, int flags, float scale,
+                        void* out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const Plan pl = plan(B, n_q, Hq, Hkv, D, kv_start, kv_len);
+  if (ws_bytes < pl.ws_bytes) return fail(VC_ERR_INVALID, "verify workspace too small");
+  if (P + n_q > (int64_t)1 << 31) return fail(VC_ERR_UNSUPPORTED, "verify: positions >= 2^31");
+  CUtensorMap mk, mv;
+  if (!make_kv_map(&mk, k, D, kv_len, L_cap, pl.pairs) ||
+      !make_kv_map(&mv, v, D, kv_len, L_cap, pl.pairs))
+    return fail(VC_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  VerifyParams vp;
+  vp.q = static_cast<const __nv_bfloat16*>(q);
+  vp.n_q = n_q;
+  vp.Hq = Hq;
+  vp.Hkv = Hkv;
+  vp.g = pl.g;
+  vp.R = pl.R;
+  vp.kv_start = kv_start;
+  vp.kv_len = kv_len;
+  vp.P = P;
+  vp.split0 = pl.split0;
+  vp.n_split = pl.n_split;
+  vp.qk_scale2 = scale * kLog2e;
+  vp.ws_o = static_cast<float*>(ws);
+  vp.ws_ml = vp.ws_o + (size_t)pl.pairs * pl.n_split * pl.R * D;
+  if (D == 128) return run_verify<128>(pl, vp, mk, mv, flags, m, l, acc, out, stream);
+  return run_verify<64>(pl, vp, mk, mv, flags, m, l, acc, out, stream);
+}
+
+vc_status read_device_error(int32_t* value, int clear) {
+  int v = 0;
+  VC_CUDA(cudaMemcpyFromSymbol(&v, g_vc_dev_error, sizeof(int)));
+  if (value) *value = v;
+  if (clear) {
+    const int z = 0;
+    VC_CUDA(cudaMemcpyToSymbol(g_vc_dev_error, &z, sizeof(int)));
+  }
+  return VC_OK;
 }
 
 }  // namespace vc

@@ -145,7 +145,7 @@ def attn_case(cfg: AttnConfig | int, **override) -> dict:
     out["k_bits"], out["v_bits"] = f32_to_bf16_bits(Kf), f32_to_bf16_bits(Vf)
     out["q_draft_bits"] = f32_to_bf16_bits(normal(r[3], (B, Hq, D)))
     out["q_verify_bits"] = f32_to_bf16_bits(normal(r[4], (B, k + 1, Hq, D)))
-    if cfg.cache == "indexed":
+    if cfg.cache == "indexed" and cfg.S > 0:
         if cfg.compact:
             ck = ar1(r[5], (B, Hkv), cfg.S, D, cfg.rho)
             cv = ar1(r[6], (B, Hkv), cfg.S, D, cfg.rho)

@@ -58,14 +58,14 @@ def _cache(**kw):
 ])
 def test_draft_rejects_bad_cache(kw, status):
     c = _cache(**kw)
-    st = vc.lib().vc_draft_attn(1 << 20, ctypes.byref(c), 0.0, 1 << 20, None, 1 << 20, 1 << 20,
-                                None)
+    st = vc.lib().vc_draft_attn(1 << 20, ctypes.byref(c), 0.0, 0, 1 << 20, None, 1 << 20,
+                                1 << 20, None)
     assert st == status, vc.lib().vc_last_error()
     assert vc.lib().vc_last_error()
 
 
 def test_draft_rejects_null_cache():
-    assert vc.lib().vc_draft_attn(1 << 20, None, 0.0, 1 << 20, None, 1 << 20, 1, None) == 1
+    assert vc.lib().vc_draft_attn(1 << 20, None, 0.0, 0, 1 << 20, None, 1 << 20, 1, None) == 1
 
 
 @pytest.mark.parametrize("args,status", [

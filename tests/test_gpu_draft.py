@@ -11,7 +11,7 @@ import torch
 import oracle
 import lossless_kv_compressed_b200 as vc
 from synth import gen
-from tests.gpu_util import assert_close_attn, dev_bf16, dev_i32, host_f64
+from tests.gpu_util import assert_close_attn, both_outputs, dev_bf16, dev_i32, host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -33,8 +33,8 @@ def _run(case, S, n_tail, use_idx=True, use_deg=True, check_lse=True):
         err_flag=torch.zeros(1, dtype=torch.int32, device="cuda"))
     q = dev_bf16(q_bits)
     lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
-    out = vc.draft_attn(q, cache, lse=lse)
-    torch.cuda.synchronize()
+    out = both_outputs(lambda dt: vc.draft_attn(q, cache, lse=lse, out=torch.empty(
+        q.shape, dtype=dt, device="cuda")))
     assert int(cache.err_flag.item()) == 0
     f = oracle.bf16_to_f64
     o_ref, lse_ref = oracle.draft_attn(
