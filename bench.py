@@ -1,0 +1,535 @@
+"""Benchmark of the VeriCache draft/verify hot path on B200.
+
+One step = one draft-then-verify round of one attention layer (VeriCache summary,
+"Riepilogo Tecnico: VeriCache", section "Algoritmo Principale"), on the Llama-3.1-8B
+shaped workload: batch 8, 32 query / 8 KV heads of dim 128, 32768-token context, a
+token-evicted compressed cache of 8192 slots with degrees 1..16, draft length k = 32:
+
+  for j in 0..k-1:  vc_draft_attn over the compressed cache + j+1 tail rows
+                    vc_accept (argmax of that draft step's logits, vocab 128256)
+  vc_verify_attn    33 rows per sequence over the full 32801-key cache (tcgen05)
+  vc_accept         first-mismatch acceptance + bonus over [8, 33, 128256] logits
+
+Metric: attention GB/s = algorithmic bytes of the draft and verify calls per round /
+device time of the round.  Inputs are synthetic (seeded, see synth/), resident in HBM;
+four copies of the layer's cache rotate across calls so no call re-reads another's
+data from the 126 MB L2, and L2 is flushed (256 MB write) between timed steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "draft/verify attn GB/s & %roofline; accepted tokens/s on 1 B200"
+N_COPIES = 4
+
+
+# ------------------------------------------------------------------ bytes / flops
+def draft_bytes(cfg, n_tail: int) -> int:
+    """Algorithmic bytes of one draft call: the gathered K and V rows of every slot and
+    tail row, the slot indices and degrees, q in and o out."""
+    pairs = cfg.B * cfg.Hkv
+    kv = pairs * (cfg.S + n_tail) * cfg.D * 2 * 2
+    meta = pairs * cfg.S * 4 * 2
+    qo = 2 * cfg.B * cfg.Hq * cfg.D * 2
+    return kv + meta + qo
+
+
+def verify_bytes(cfg) -> int:
+    pairs = cfg.B * cfg.Hkv
+    n_q = cfg.k + 1
+    kv = pairs * (cfg.P + n_q) * cfg.D * 2 * 2
+    qo = 2 * cfg.B * n_q * cfg.Hq * cfg.D * 2
+    return kv + qo
+
+
+def verify_flops(cfg) -> int:
+    """QK^T and PV over the keys each row sees: 4 D per (row, visible key)."""
+    pairs = cfg.B * cfg.Hkv
+    keys = sum(cfg.P + i + 1 for i in range(cfg.k + 1))
+    return 4 * cfg.D * cfg.g * keys * pairs
+
+
+def round_bytes(cfg) -> int:
+    return sum(draft_bytes(cfg, j + 1) for j in range(cfg.k)) + verify_bytes(cfg)
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampled during the timed region (read-only queries)."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_uuid: str | None):
+        self.proc = None
+        self.uuid = dev_uuid
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "50"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ peaks / traffic
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d.get("hbm_gbs"), "bf16_tflops": d.get("bf16_tflops"),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def profiled_traffic(kernel: str) -> float | None:
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on the
+    kernel source as it is now (source hash recorded beside the figure)."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(kernel)
+    if not d:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return float(d["bytes_per_launch"]) if h == d.get("source_sha256_16") else None
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def dist_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ oracle baseline
+def oracle_pair_sample(case, b: int, j: int):
+    """The oracle's share of one round for one (batch, kv head) pair: the k draft calls
+    and the verify rows of that pair, plus acceptance of that batch row.  Returns
+    (algorithmic bytes, seconds)."""
+    import oracle
+    cfg = case["cfg"]
+    f = oracle.bf16_to_f64
+    g, P, n_q = cfg.g, cfg.P, cfg.k + 1
+    kb = f(case["k_bits"][b:b + 1, j:j + 1])
+    vb = f(case["v_bits"][b:b + 1, j:j + 1])
+    idx = case["idx"][b:b + 1, j:j + 1]
+    deg = case["deg"][b:b + 1, j:j + 1]
+    qd = f(case["q_draft_bits"][b:b + 1, j * g:(j + 1) * g])
+    qv = f(case["q_verify_bits"][b:b + 1, :, j * g:(j + 1) * g])
+    t0 = time.perf_counter()
+    nbytes = 0
+    for t in range(cfg.k):
+        oracle.draft_attn(qd, kb, vb, cfg.S, idx, deg, kb[:, :, P:P + t + 1], vb[:, :, P:P + t + 1])
+        nbytes += ((cfg.S + t + 1) * cfg.D * 4 + cfg.S * 8 + 2 * g * cfg.D * 2)
+    oracle.verify_attn(qv, kb[:, :, :P + n_q], vb[:, :, :P + n_q], P)
+    nbytes += (P + n_q) * cfg.D * 4 + 2 * n_q * g * cfg.D * 2
+    return nbytes, time.perf_counter() - t0
+
+
+def cpu_baseline(case, budget_s: float = 20.0) -> dict:
+    """The oracle, as it stands, on a bounded sample of the same workload."""
+    cfg = case["cfg"]
+    pairs = [(b, j) for b in range(cfg.B) for j in range(cfg.Hkv)]
+    tot_b, tot_t, n = 0, 0.0, 0
+    c0 = time.process_time()
+    w0 = time.perf_counter()
+    for b, j in pairs:
+        nb, dt = oracle_pair_sample(case, b, j)
+        tot_b += nb
+        tot_t += dt
+        n += 1
+        if tot_t > budget_s:
+            break
+    cores = max(1, round((time.process_time() - c0) / max(time.perf_counter() - w0, 1e-9)))
+    return {"value": tot_b / tot_t / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {len(pairs)} (batch, kv head) pairs of one round: all {cfg.k} "
+                      f"draft calls and the {cfg.k + 1} verify positions of each pair, fp64 "
+                      f"NumPy on {os.cpu_count()} host cores ({tot_t:.1f} s)"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    from synth import gen
+    case = gen.attn_case(2)
+    cfg = case["cfg"]
+    pairs = [(b, j) for b in range(cfg.B) for j in range(cfg.Hkv)]
+    for w in range(args.warmup):
+        oracle_pair_sample(case, *pairs[w % len(pairs)])
+    tot_b, tot_t = 0, 0.0
+    c0, w0 = time.process_time(), time.perf_counter()
+    for s in range(args.steps):
+        nb, dt = oracle_pair_sample(case, *pairs[(args.warmup + s) % len(pairs)])
+        tot_b += nb
+        tot_t += dt
+    cores = max(1, round((time.process_time() - c0) / max(time.perf_counter() - w0, 1e-9)))
+    value = tot_b / tot_t / 1e9
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": cfg.name, "batch": cfg.B, "heads": f"{cfg.Hq}/{cfg.Hkv}",
+                       "head_dim": cfg.D, "context": cfg.P, "slots": cfg.S, "draft_len": cfg.k,
+                       "step": "one (batch, kv head) pair's share of a round"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": "each step: one (batch, kv head) pair's k draft calls "
+                                       "and verify rows, fp64 NumPy"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ device workload
+class Round:
+    """Device-resident inputs and prepared C-ABI calls of one round."""
+
+    def __init__(self, case, device):
+        import torch
+        import lossless_kv_compressed_b200 as vc
+        from lossless_kv_compressed_b200._lib import CompCache, lib
+        from synth import gen
+        self.vc, self.lib = vc, lib()
+        cfg = self.cfg = case["cfg"]
+        t = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
+            torch.bfloat16).to(device)
+        k0, v0 = t(case["k_bits"]), t(case["v_bits"])
+        self.K = [k0] + [k0.clone() for _ in range(N_COPIES - 1)]
+        self.V = [v0] + [v0.clone() for _ in range(N_COPIES - 1)]
+        kt = t(gen.bf16_block_rows(case, "k", cfg.k + 1))
+        vt = t(gen.bf16_block_rows(case, "v", cfg.k + 1))
+        self.KT = [kt] + [kt.clone() for _ in range(N_COPIES - 1)]
+        self.VT = [vt] + [vt.clone() for _ in range(N_COPIES - 1)]
+        self.idx = torch.from_numpy(case["idx"]).to(device)
+        self.deg = torch.from_numpy(case["deg"]).to(device)
+        rng = gen.children(7002, 3)
+        qd = np.stack([gen.f32_to_bf16_bits(gen.normal(rng[0], (cfg.B, cfg.Hq, cfg.D)))
+                       for _ in range(cfg.k)])
+        self.q_draft = t(qd)
+        self.q_verify = t(case["q_verify_bits"])
+        V = cfg.vocab
+        self.draft_logits = torch.from_numpy(gen.normal(rng[1], (cfg.k, cfg.B, 1, V))).to(device)
+        self.logits = torch.from_numpy(case["logits"]).to(device)
+        self.drafts = torch.from_numpy(case["drafts"]).to(device)
+        i32 = dict(dtype=torch.int32, device=device)
+        self.d_out = torch.empty_like(self.q_draft)
+        self.v_out = torch.empty_like(self.q_verify)
+        self.d_target = torch.empty((cfg.k, cfg.B, 1), **i32)
+        self.d_err = torch.empty((cfg.k, cfg.B), **i32)
+        self.target = torch.empty((cfg.B, cfg.k + 1), **i32)
+        self.alen = torch.empty((cfg.B,), **i32)
+        self.commit = torch.empty((cfg.B, cfg.k + 1), **i32)
+        self.ncommit = torch.empty((cfg.B,), **i32)
+        self.err = torch.empty((cfg.B,), **i32)
+        # prepared draft caches (one per draft step)
+        self.caches = []
+        for j in range(cfg.k):
+            c = j % N_COPIES
+            cc = vc.IndexedCache(k=self.K[c], v=self.V[c], S=cfg.S, Hq=cfg.Hq, idx=self.idx,
+                                 deg=self.deg, k_tail=self.KT[c], v_tail=self.VT[c], n_tail=j + 1)
+            self.caches.append(cc)
+        self.structs = [c.struct() for c in self.caches]
+        self.ws_d = torch.empty(max(vc.draft_workspace_size(c) for c in self.caches),
+                                dtype=torch.uint8, device=device)
+        n_q = cfg.k + 1
+        self.ws_v = torch.empty(vc.verify_workspace_size(cfg.B, n_q, cfg.Hq, cfg.Hkv, cfg.D, 0,
+                                                         cfg.P + n_q), dtype=torch.uint8,
+                                device=device)
+        self.flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+        self.launches_per_step = cfg.k * (2 + 2) + 2 + 2
+
+    def step(self, stream_handle: int, draft_events=None, verify_events=None):
+        """Enqueue one round on the stream; optional event pairs around each draft call
+        and around the verify call."""
+        cfg, L = self.cfg, self.lib
+        sb = self.d_out.element_size()
+        for j in range(cfg.k):
+            if draft_events is not None:
+                draft_events[j][0].record()
+            st = L.vc_draft_attn(self.q_draft[j].data_ptr(), ctypes.byref(self.structs[j]), 0.0, 0,
+                                 self.d_out[j].data_ptr(), None, self.ws_d.data_ptr(),
+                                 self.ws_d.numel(), stream_handle)
+            if draft_events is not None:
+                draft_events[j][1].record()
+            if st:
+                self.vc._lib.check(st, "vc_draft_attn")
+            st = L.vc_accept(self.draft_logits[j].data_ptr(), None, cfg.B, 1, cfg.vocab,
+                             self.d_target[j].data_ptr(), None, None, None,
+                             self.d_err[j].data_ptr(), stream_handle)
+            if st:
+                self.vc._lib.check(st, "vc_accept")
+        c = cfg.k % N_COPIES
+        n_q = cfg.k + 1
+        if verify_events is not None:
+            verify_events[0].record()
+        st = L.vc_verify_attn(self.q_verify.data_ptr(), cfg.B, n_q, cfg.Hq, cfg.Hkv, cfg.D,
+                              self.K[c].data_ptr(), self.V[c].data_ptr(), cfg.L_cap, 0,
+                              cfg.P + n_q, cfg.P, None, None, None, 0, 0.0,
+                              self.v_out.data_ptr(), self.ws_v.data_ptr(), self.ws_v.numel(),
+                              stream_handle)
+        if verify_events is not None:
+            verify_events[1].record()
+        if st:
+            self.vc._lib.check(st, "vc_verify_attn")
+        st = L.vc_accept(self.logits.data_ptr(), self.drafts.data_ptr(), cfg.B, n_q, cfg.vocab,
+                         self.target.data_ptr(), self.alen.data_ptr(), self.commit.data_ptr(),
+                         self.ncommit.data_ptr(), self.err.data_ptr(), stream_handle)
+        if st:
+            self.vc._lib.check(st, "vc_accept")
+
+    def flush_l2(self):
+        self.flush_buf.zero_()
+
+
+def e2e_measure(rnd, steps: int, warmup: int, device) -> dict:
+    """Same metric through the public Python API, with every step's inputs copied
+    from pinned host memory and its results read back inside the timed region."""
+    import torch
+    vc = rnd.vc
+    cfg = rnd.cfg
+    pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())
+    h_qd, h_qv = pin(rnd.q_draft), pin(rnd.q_verify)
+    h_dl, h_lg, h_dr = pin(rnd.draft_logits), pin(rnd.logits), pin(rnd.drafts)
+    h_kt, h_vt = pin(rnd.KT[0]), pin(rnd.VT[0])
+    o_d = torch.empty(rnd.d_out.shape, dtype=rnd.d_out.dtype, pin_memory=True)
+    o_v = torch.empty(rnd.v_out.shape, dtype=rnd.v_out.dtype, pin_memory=True)
+    o_c = torch.empty(rnd.commit.shape, dtype=torch.int32, pin_memory=True)
+    o_n = torch.empty(rnd.ncommit.shape, dtype=torch.int32, pin_memory=True)
+    h2d = sum(x.numel() * x.element_size() for x in (h_qd, h_qv, h_dl, h_lg, h_dr, h_kt, h_vt))
+    d2h = sum(x.numel() * x.element_size() for x in (o_d, o_v, o_c, o_n))
+    n_q = cfg.k + 1
+
+    def one():
+        rnd.q_draft.copy_(h_qd, non_blocking=True)
+        rnd.q_verify.copy_(h_qv, non_blocking=True)
+        rnd.draft_logits.copy_(h_dl, non_blocking=True)
+        rnd.logits.copy_(h_lg, non_blocking=True)
+        rnd.drafts.copy_(h_dr, non_blocking=True)
+        rnd.KT[0].copy_(h_kt, non_blocking=True)
+        rnd.VT[0].copy_(h_vt, non_blocking=True)
+        for j in range(cfg.k):
+            vc.draft_attn(rnd.q_draft[j], rnd.caches[j], out=rnd.d_out[j], ws=rnd.ws_d)
+            vc.accept(rnd.draft_logits[j], None, target=rnd.d_target[j], err_flag=rnd.d_err[j])
+        vc.verify_attn(rnd.q_verify, rnd.K[cfg.k % N_COPIES], rnd.V[cfg.k % N_COPIES], cfg.P,
+                       out=rnd.v_out, ws=rnd.ws_v)
+        vc.accept(rnd.logits, rnd.drafts, target=rnd.target, accept_len=rnd.alen,
+                  commit=rnd.commit, n_commit=rnd.ncommit, err_flag=rnd.err)
+        o_d.copy_(rnd.d_out, non_blocking=True)
+        o_v.copy_(rnd.v_out, non_blocking=True)
+        o_c.copy_(rnd.commit, non_blocking=True)
+        o_n.copy_(rnd.ncommit, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    tot = 0.0
+    for _ in range(steps):
+        rnd.flush_l2()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        one()
+        e1.record()
+        e1.synchronize()
+        tot += e0.elapsed_time(e1) * 1e-3
+    return {"value": round_bytes(cfg) / (tot / steps) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": tot / steps * 1e3}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="vc", choices=["vc", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        code = run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return code
+
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    from synth import gen
+    case = gen.attn_case(2)
+    cfg = case["cfg"]
+    rnd = Round(case, device)
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+
+    for _ in range(args.warmup):
+        rnd.step(sh)
+    torch.cuda.synchronize()
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(cfg.k)] for _ in range(args.steps)]
+    st_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
+    v_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.1)
+    for s in range(args.steps):
+        rnd.flush_l2()
+        st_ev[s][0].record()
+        rnd.step(sh, ev[s], v_ev[s])
+        st_ev[s][1].record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    step_s = sum(a.elapsed_time(b) for a, b in st_ev) * 1e-3
+    draft_s = [a.elapsed_time(b) * 1e-3 for step in ev for a, b in step]
+    verify_s = statistics.mean(a.elapsed_time(b) * 1e-3 for a, b in v_ev)
+    t_max = dist_max(step_s, world)
+
+    rb = round_bytes(cfg)
+    value = world * args.steps * rb / t_max / 1e9
+    peaks = measured_peaks()
+    d_bytes = statistics.mean(draft_bytes(cfg, j + 1) for j in range(cfg.k))
+    d_time = statistics.mean(draft_s)
+    achieved = d_bytes / d_time / 1e9
+    traffic = profiled_traffic("draft_attn")
+    roof = {"bound": "hbm", "kernel": "vc_draft_attn (split + combine)",
+            "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+            "peak_source": peaks["source"] + " hbm_gbs (copy bandwidth)",
+            "algorithmic_bytes_per_launch": d_bytes, "launch_us": d_time * 1e6}
+
+    e2e = None
+    if world == 1 or rank == 0:
+        e2e = e2e_measure(rnd, max(3, min(args.steps, 20)), 3, device)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(case)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_max / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": cfg.name, "batch": cfg.B, "heads": f"{cfg.Hq}/{cfg.Hkv}",
+                       "head_dim": cfg.D, "context": cfg.P, "slots": cfg.S,
+                       "draft_len": cfg.k, "vocab": cfg.vocab,
+                       "l2": "flushed between steps (256 MB write); 4 rotating cache copies",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "clocks": clk,
+            "gpu_launches": rnd.launches_per_step * args.steps,
+            "kernels": {
+                "vc_draft_attn": {"us": d_time * 1e6, "GB/s": achieved,
+                                  "frac_hbm": achieved / peaks["hbm_gbs"]},
+                "vc_verify_attn": {"us": verify_s * 1e6,
+                                   "TFLOP/s": verify_flops(cfg) / verify_s / 1e12,
+                                   "frac_tensor": verify_flops(cfg) / verify_s / 1e12
+                                   / peaks["bf16_tflops"],
+                                   "GB/s": verify_bytes(cfg) / verify_s / 1e9,
+                                   "frac_hbm": verify_bytes(cfg) / verify_s / 1e9
+                                   / peaks["hbm_gbs"]},
+            },
+            "round_bytes": rb,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
