@@ -138,6 +138,24 @@ vc_status vc_draft_attn(const void* q, const vc_comp_cache* cache, float scale, 
                         void* out, float* lse, void* ws, size_t ws_bytes,
                         cudaStream_t stream);
 
+/* Draft attention that allocates nothing and takes no workspace (the pages have no
+ * counterpart: this serves callers that cannot hand the library scratch memory, such as
+ * a plugin whose host runtime owns all device memory and offers no allocator, a process
+ * whose memory pool is fully reserved up front, or a path that must not call cudaMalloc
+ * because it can block and synchronise the device).  Same arguments and result as
+ * vc_draft_attn, without ws / ws_bytes: the split-K partials go to a fixed 8 MiB array in
+ * the library's device image, which every GPU that loads the library holds until exit.
+ *   - A cache whose partials need more than 8 MiB (vc_draft_workspace_size) is rejected
+ *     with VC_ERR_UNSUPPORTED before anything is launched.
+ *   - The first call on each device does a one-time set-up (it looks up the array's
+ *     device address with that device current); make that first call before any stream
+ *     capture begins.
+ *   - All calls on a device share the one array and it keeps the last call's contents
+ *     (nothing in it needs to start at zero).  Calls that overlap on the GPU -- on
+ *     different streams, or from different threads -- race on it: serialise them. */
+vc_status vc_draft_attn_noalloc(const void* q, const vc_comp_cache* cache, float scale,
+                                int flags, void* out, float* lse, cudaStream_t stream);
+
 /* ------------------------------------------------------------------------------
  * Verify attention ([VC] "Algoritmo Principale", step 2: one pass over KV_full checks
  * all drafted tokens in parallel).  Row i (0 <= i < n_q, n_q = k + 1: the pending

@@ -19,7 +19,7 @@ VC_OUT_F32 = 4
 # Every exported symbol, in header order.
 EXPORTS = (
     "vc_status_string", "vc_last_error", "vc_abi_version",
-    "vc_draft_workspace_size", "vc_draft_attn",
+    "vc_draft_workspace_size", "vc_draft_attn", "vc_draft_attn_noalloc",
     "vc_verify_workspace_size", "vc_verify_attn",
     "vc_accept", "vc_stage_full_kv", "vc_event_wait", "vc_device_error",
 )
@@ -71,6 +71,9 @@ def lib() -> ctypes.CDLL:
         L.vc_draft_attn.restype = ctypes.c_int
         L.vc_draft_attn.argtypes = [_p, ctypes.POINTER(CompCache), ctypes.c_float, ctypes.c_int,
                                     _p, _p, _p, _sz, _p]
+        L.vc_draft_attn_noalloc.restype = ctypes.c_int
+        L.vc_draft_attn_noalloc.argtypes = [_p, ctypes.POINTER(CompCache), ctypes.c_float,
+                                            ctypes.c_int, _p, _p, _p]
         L.vc_verify_workspace_size.restype = _sz
         L.vc_verify_workspace_size.argtypes = [ctypes.c_int] * 5 + [_i64, _i64]
         L.vc_verify_attn.restype = ctypes.c_int

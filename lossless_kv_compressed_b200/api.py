@@ -157,6 +157,22 @@ def draft_attn(q: torch.Tensor, cache, out: Optional[torch.Tensor] = None,
     return out
 
 
+def draft_attn_noalloc(q: torch.Tensor, cache, out: Optional[torch.Tensor] = None,
+                       lse: Optional[torch.Tensor] = None, scale: float = 0.0,
+                       stream=None) -> torch.Tensor:
+    """draft_attn for callers that cannot provide a workspace: the library keeps the
+    split-K partials in a fixed 8 MiB per-device array (see vc_draft_attn_noalloc).
+    Calls that overlap on the GPU share that array and must be serialised."""
+    _need(q, torch.bfloat16, "q")
+    s = cache.struct()
+    if out is None:
+        out = torch.empty_like(q)
+    check(lib().vc_draft_attn_noalloc(q.data_ptr(), ctypes.byref(s), float(scale),
+                                      _out_flag(out), out.data_ptr(), _ptr(lse),
+                                      _stream(stream)), "vc_draft_attn_noalloc")
+    return out
+
+
 # ------------------------------------------------------------------ verify
 def verify_workspace_size(B, n_q, Hq, Hkv, D, kv_start, kv_len) -> int:
     return int(lib().vc_verify_workspace_size(B, n_q, Hq, Hkv, D, kv_start, kv_len))

@@ -381,3 +381,60 @@ vc_status launch_draft_int4(const void*, const vc_comp_cache*, float, int, void*
   return fail(VC_ERR_UNSUPPORTED, "int4 draft attention not built yet");
 }
 }  // namespace vc
+
+// ------------------------------------------------------------------ fixed-scratch variant
+// Some callers hand this library only their input and output buffers and cannot give it
+// scratch memory: a plugin inside a host runtime that owns every byte of device memory
+// and exposes no allocator, a fixed-budget serving process whose pool is fully reserved
+// up front, or a latency-critical path that must not call cudaMalloc (which can block
+// and synchronise the device).  For them vc_draft_attn_noalloc runs the same draft
+// attention with its split-K partials in the array below, which lives in the library's
+// own device image: every GPU that loads the library holds these bytes until the
+// process exits, and no call allocates anything.
+#include <mutex>
+#include <vector>
+
+namespace {
+constexpr size_t kNoAllocScratchBytes = 8u << 20;   // 8 MiB per device
+static __device__ __align__(256) unsigned char g_draft_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+std::vector<void*> g_noalloc_ptr;   // device address of the array, per device ordinal
+}  // namespace
+
+extern "C" vc_status vc_draft_attn_noalloc(const void* q, const vc_comp_cache* cache,
+                                           float scale, int flags, void* out, float* lse,
+                                           cudaStream_t stream) {
+  // The size check comes first and needs no device: the partials this call needs must
+  // fit the fixed array.
+  const size_t need = vc_draft_workspace_size(cache);
+  if (need == 0) return VC_ERR_INVALID;   // cache rejected; vc_last_error() says why
+  if (need > kNoAllocScratchBytes)
+    return vc::fail(VC_ERR_UNSUPPORTED,
+                    "draft_noalloc: this cache needs %zu bytes of scratch, the fixed scratch "
+                    "holds %zu (use vc_draft_attn with a caller workspace)",
+                    need, kNoAllocScratchBytes);
+  // One-time set-up per device, with that device current: in host code the array's
+  // name is only a stand-in, so its device address is looked up once and kept.
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess)
+    return vc::fail(VC_ERR_CUDA, "draft_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if ((int)g_noalloc_ptr.size() <= dev) g_noalloc_ptr.resize(dev + 1, nullptr);
+    if (!g_noalloc_ptr[dev]) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_draft_noalloc_scratch);
+      if (e != cudaSuccess || !p)
+        return vc::fail(VC_ERR_CUDA, "draft_noalloc: cudaGetSymbolAddress: %s",
+                        cudaGetErrorString(e));
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  // Nothing in the partials has to start at zero: every entry a call reads was written
+  // earlier in the same call, so the previous call's leftovers are harmless.
+  return vc_draft_attn(q, cache, scale, flags, out, lse, scratch, kNoAllocScratchBytes, stream);
+}
