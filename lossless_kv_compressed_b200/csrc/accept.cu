@@ -3,12 +3,15 @@
 // the first disagreement with the full-KV prediction, plus one bonus token when all
 // agree.
 //
-// Kernel 1: one CTA per logits row, float4 streaming argmax (ties -> lowest index;
-//           NaN larger than any number, first NaN wins).  The row's NaN bit is
-//           parked in bit 31 of its target entry.
+// Kernel 1: float4 streaming argmax of each logits row (ties -> lowest index; NaN
+//           larger than any number, first NaN wins); large vocabularies split a row
+//           over an 8-CTA cluster merged through distributed shared memory.  The
+//           row's NaN bit is parked in bit 31 of its target entry.
 // Kernel 2: one warp per batch row: clears the NaN bits into err_flag, finds the first
 //           disagreement with a ballot, and writes accept_len / commit / n_commit.
 #include <climits>
+
+#include <cooperative_groups.h>
 
 #include "vc_common.cuh"
 #include "vc_internal.h"
@@ -26,18 +29,25 @@ __device__ __forceinline__ bool better(float v, int i, const ArgBest& b) {
   return v > b.val || (v == b.val && i < b.idx);
 }
 
-template <int THREADS>
+// One row per thread-block cluster of CL CTAs: CTA c scans a contiguous slice of the
+// row, the cluster's rank-0 CTA merges the CL partials through distributed shared
+// memory (slices in order, so the lowest index still wins ties).
+template <int THREADS, int CL>
 __global__ void __launch_bounds__(THREADS) argmax_rows_kernel(const float* __restrict__ logits,
                                                               int V, int32_t* __restrict__ target) {
-  const int64_t row = blockIdx.x;
+  namespace cg = cooperative_groups;
+  const int64_t row = blockIdx.x / CL;
+  const int crank = (int)(blockIdx.x % CL);
   const float* x = logits + row * (int64_t)V;
+  // slice [lo, hi) of the row, multiples of 4 so float4 loads stay aligned
+  const int per = ((V + CL - 1) / CL + 3) & ~3;
+  const int lo = min(V, crank * per), hi = min(V, lo + per);
   ArgBest best{-INFINITY, INT_MAX};
   int first_nan = INT_MAX;
   const bool vec = ((V & 3) == 0) && ((reinterpret_cast<uintptr_t>(x) & 15) == 0);
   if (vec) {
     const float4* x4 = reinterpret_cast<const float4*>(x);
-    const int n4 = V >> 2;
-    for (int i = threadIdx.x; i < n4; i += THREADS) {
+    for (int i = (lo >> 2) + threadIdx.x; i < (hi >> 2); i += THREADS) {
       const float4 f = __ldg(x4 + i);
       const float e[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
@@ -48,13 +58,12 @@ __global__ void __launch_bounds__(THREADS) argmax_rows_kernel(const float* __res
       }
     }
   } else {
-    for (int i = threadIdx.x; i < V; i += THREADS) {
+    for (int i = lo + threadIdx.x; i < hi; i += THREADS) {
       const float e = __ldg(x + i);
       if (isnan(e)) first_nan = min(first_nan, i);
       else if (better(e, i, best)) best = {e, i};
     }
   }
-  // warp reduction
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float v = __shfl_xor_sync(0xffffffffu, best.val, o);
@@ -65,6 +74,8 @@ __global__ void __launch_bounds__(THREADS) argmax_rows_kernel(const float* __res
   __shared__ float sv[THREADS / 32];
   __shared__ int si[THREADS / 32];
   __shared__ int sn[THREADS / 32];
+  __shared__ float cv;   // this CTA's result, read by the cluster leader
+  __shared__ int ci, cn;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0) { sv[warp] = best.val; si[warp] = best.idx; sn[warp] = first_nan; }
   __syncthreads();
@@ -79,12 +90,31 @@ __global__ void __launch_bounds__(THREADS) argmax_rows_kernel(const float* __res
       if (better(v, i, best)) best = {v, i};
       first_nan = min(first_nan, __shfl_xor_sync(0xffffffffu, first_nan, o));
     }
-    if (lane == 0) {
-      // an all -inf row: every entry ties at -inf, lowest index 0 wins
-      int t = best.idx == INT_MAX ? 0 : best.idx;
-      if (first_nan != INT_MAX) t = first_nan | (int)0x80000000u;
-      target[row] = t;
+    if (lane == 0) { cv = best.val; ci = best.idx; cn = first_nan; }
+  }
+  if constexpr (CL > 1) {
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    if (crank == 0 && threadIdx.x == 0) {
+      best = {cv, ci};
+      first_nan = cn;
+      for (int r = 1; r < CL; ++r) {
+        const float v = *cluster.map_shared_rank(&cv, r);
+        const int i = *cluster.map_shared_rank(&ci, r);
+        if (better(v, i, best)) best = {v, i};
+        first_nan = min(first_nan, *cluster.map_shared_rank(&cn, r));
+      }
+      cv = best.val; ci = best.idx; cn = first_nan;
     }
+    cluster.sync();   // peers keep their shared memory until the leader has read it
+  } else {
+    __syncthreads();
+  }
+  if (crank == 0 && threadIdx.x == 0) {
+    // an all -inf row: every entry ties at -inf, lowest index 0 wins
+    int t = ci == INT_MAX ? 0 : ci;
+    if (cn != INT_MAX) t = cn | (int)0x80000000u;
+    target[row] = t;
   }
 }
 
@@ -126,8 +156,23 @@ vc_status launch_accept(const float* logits, const int32_t* drafts, int B, int n
                         int32_t* target, int32_t* accept_len, int32_t* commit,
                         int32_t* n_commit, int32_t* err_flag, cudaStream_t stream) {
   const int rows = B * n_q;
-  if (V >= 16384) argmax_rows_kernel<512><<<rows, 512, 0, stream>>>(logits, V, target);
-  else argmax_rows_kernel<128><<<rows, 128, 0, stream>>>(logits, V, target);
+  if (V >= 16384) {
+    constexpr int CL = 8;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(rows * CL);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    VC_CUDA(cudaLaunchKernelEx(&cfg, argmax_rows_kernel<256, CL>, logits, V, target));
+  } else {
+    argmax_rows_kernel<128, 1><<<rows, 128, 0, stream>>>(logits, V, target);
+  }
   VC_CUDA(cudaGetLastError());
   accept_kernel<<<B, 32, 0, stream>>>(n_q, drafts, target, accept_len, commit, n_commit,
                                       err_flag);

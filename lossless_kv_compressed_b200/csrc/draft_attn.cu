@@ -7,15 +7,23 @@
 //     s_t = (q . k_t) * scale + ln n_t,   o = sum_t softmax(s)_t v_t.
 //
 // Design (HBM-bound: every KV byte is read once per call):
-//   grid (n_split, B*Hkv); a CTA owns one (batch, kv head) and a chunk of slots, all
-//   g <= 8 query heads of the group share the KV rows it streams.  4 warps, each with
-//   its own cp.async ring of 16-slot tiles (K and V rows gathered by slot index,
-//   16-byte copies into XOR-swizzled shared rows, no CTA barrier in the main loop).
-//   q.K^T and P.V run on mma.sync m16n8k16 with the heads as the M rows (rows >= g are
-//   zero padding) so the fp32 pipes only do the softmax.  Scores live in the log2
-//   domain: s2 = s * scale * log2(e) + log2(n_t); the online softmax uses ex2.
-//   Each CTA writes one partial (max, sum, unnormalised o) per head; a second kernel
-//   merges the splits in a fixed order and writes bf16 o (and lse).
+//   The work is the list of (batch, kv head) pairs times their 16-slot tiles (the
+//   compressed slots followed by the bf16 tail rows).  A persistent grid of
+//   2 CTAs x 4 warps per SM cuts that list into equal contiguous ranges, one per warp,
+//   so every warp streams the same number of tiles (to within one) and no wave is left
+//   half empty.  Each warp runs its own cp.async ring of K and V rows gathered by slot
+//   index (16-byte copies into XOR-swizzled shared rows; no CTA barrier anywhere).  The
+//   slot -> row table and log2-degree biases of the next 16 tiles are prefetched into
+//   registers and staged into a double-buffered shared table ahead of the copies.
+//   q.K^T and P.V run on mma.sync m16n8k16 with the g <= 8 heads of the group as the M
+//   rows; rows 8-15 carry P's bf16 low part so P.V keeps ~16 mantissa bits of P.
+//   Scores live in the log2 domain: s2 = s * scale * log2(e) + log2(n_t); the online
+//   softmax uses ex2.  A warp writes one partial (max, sum, unnormalised o) per pair
+//   it touches; a second kernel merges the partials of each head in a fixed order.
+//   (Measured and rejected: L2 bulk prefetch of rows beyond the ring, 37% slower;
+//   launching the merge as a programmatic dependent, 4% slower.)
+#include <climits>
+
 #include "vc_common.cuh"
 #include "vc_internal.h"
 
@@ -32,21 +40,36 @@ struct DraftIndexedParams {
   int64_t T_cap;
   int S, S_cap, R_cap, n_tail;
   int Hq, Hkv, g;
-  int chunk, n_split;
+  int tpp;                       // 16-slot tiles per pair
+  int64_t T;                     // tiles in all: pairs * tpp
+  int W;                         // warps in the grid
+  int maxseg;                    // partial slots per pair
   float qk_scale2;               // scale * log2(e)
-  float* ws_o;                   // [pairs, n_split, g, D]
-  float* ws_ml;                  // [pairs, n_split, g, 2]
+  float* ws_o;                   // [pairs, maxseg, g, D]
+  float* ws_ml;                  // [pairs, maxseg, g, 2]
   int32_t* err_flag;
 };
 
 constexpr int kDraftWarps = 4;
-constexpr int kTile = 16;       // slots per warp tile
+constexpr int kTile = 16;       // slots per tile
+constexpr int kTB = 16;         // tiles per slot-table batch
+constexpr int kTabE = kTB * kTile;
+
+// First tile of warp w, and the warp whose range holds tile x (ranges are the
+// equal split of [0, T) into W parts).
+__host__ __device__ __forceinline__ int64_t warp_begin(int64_t w, int64_t T, int64_t W) {
+  return w * T / W;
+}
+__host__ __device__ __forceinline__ int64_t warp_of_tile(int64_t x, int64_t T, int64_t W) {
+  return ((x + 1) * W - 1) / T;
+}
 
 template <int D>
 struct DraftSmem {
   static constexpr int kRowB = D * 2;
-  static constexpr int kTileB = kTile * kRowB;       // one of K or V
+  static constexpr int kTileB = kTile * kRowB;        // one of K or V
   static constexpr int kStageB = 2 * kTileB;          // K then V
+  static constexpr int kTableB = 2 * kTabE * 8;       // 2 batches x (row code, bias)
 };
 
 template <int D, int NST>
@@ -54,65 +77,106 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
   using SM = DraftSmem<D>;
   constexpr int CH = D / 8;                 // 16-byte chunks per row
   constexpr int NT = D / 8;                 // n-tiles of the output
+  constexpr int32_t kNone = INT_MIN;        // row code of a slot past the end
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x, pair = blockIdx.y;
-  const int b = pair / p.Hkv, j = pair - b * p.Hkv;
-  const int total = p.S + p.n_tail;
-  const int s0 = split * p.chunk;
-  const int n_here = min(p.chunk, total - s0);
-
-  int32_t* srow = reinterpret_cast<int32_t*>(smem + kDraftWarps * NST * SM::kStageB);
-  float* sbias = reinterpret_cast<float*>(srow + p.chunk);
-
-  // ---- slot -> row table and log2-degree bias for this chunk
-  {
-    const int32_t* idx = p.idx ? p.idx + (int64_t)pair * p.S_cap : nullptr;
-    const int32_t* deg = p.deg ? p.deg + (int64_t)pair * p.S_cap : nullptr;
-    int bad = 0;
-    for (int i = threadIdx.x; i < n_here; i += blockDim.x) {
-      const int s = s0 + i;
-      int32_t r;
-      float bias = 0.f;
-      if (s < p.S) {
-        r = idx ? idx[s] : s;
-        if (r < 0 || (int64_t)r >= p.T_cap) { bad = 1; r = 0; }
-        int dg = deg ? deg[s] : 1;
-        if (dg < 1) { bad = 1; dg = 1; }
-        bias = log2f((float)dg);
-      } else {
-        r = -(s - p.S) - 1;
-      }
-      srow[i] = r;
-      sbias[i] = bias;
-    }
-    if (bad && p.err_flag) atomicExch(p.err_flag, 1);
-  }
-  __syncthreads();
-
-  const __nv_bfloat16* kb = p.k + (int64_t)pair * p.T_cap * D;
-  const __nv_bfloat16* vb = p.v + (int64_t)pair * p.T_cap * D;
-  const __nv_bfloat16* kt = p.k_tail ? p.k_tail + (int64_t)pair * p.R_cap * D : kb;
-  const __nv_bfloat16* vt = p.v_tail ? p.v_tail + (int64_t)pair * p.R_cap * D : vb;
+  const int64_t gw = (int64_t)blockIdx.x * kDraftWarps + warp;
+  const int64_t x0 = warp_begin(gw, p.T, p.W);
+  const int n = (int)(warp_begin(gw + 1, p.T, p.W) - x0);
+  if (n <= 0) return;
 
   uint8_t* wbuf = smem + warp * NST * SM::kStageB;
   const uint32_t wbuf_s = smem_u32(wbuf);
-  const int n_tiles = (n_here + kTile - 1) / kTile;
-  const int my_tiles = n_tiles > warp ? (n_tiles - warp + kDraftWarps - 1) / kDraftWarps : 0;
+  int32_t* trow = reinterpret_cast<int32_t*>(smem + kDraftWarps * NST * SM::kStageB +
+                                             warp * SM::kTableB);
+  float* tbias = reinterpret_cast<float*>(trow + 2 * kTabE);
+  const int total = p.S + p.n_tail;
 
+  // ---- slot table: raw idx / degree of one batch prefetched into registers, then
+  //      validated and staged into shared memory when the copies reach that batch.
+  int32_t ri[kTabE / 32], rd[kTabE / 32];
+  auto slot_of = [&](int b, int e, int64_t& pair) -> int {
+    const int local = b * kTB + e / kTile;
+    if (local >= n) return -1;
+    const int64_t x = x0 + local;
+    pair = x / p.tpp;
+    return (int)(x - pair * p.tpp) * kTile + (e % kTile);
+  };
+  auto load_batch = [&](int b) {
+#pragma unroll
+    for (int i = 0; i < kTabE / 32; ++i) {
+      int64_t pair = 0;
+      const int s = slot_of(b, lane + 32 * i, pair);
+      ri[i] = 0;
+      rd[i] = 1;
+      if (s >= 0 && s < p.S) {
+        const int64_t o = pair * p.S_cap + s;
+        ri[i] = p.idx ? __ldg(p.idx + o) : s;
+        rd[i] = p.deg ? __ldg(p.deg + o) : 1;
+      }
+    }
+  };
+  auto store_batch = [&](int b) {
+    const int buf = b & 1;
+    int bad = 0;
+#pragma unroll
+    for (int i = 0; i < kTabE / 32; ++i) {
+      const int e = lane + 32 * i;
+      int64_t pair = 0;
+      const int s = slot_of(b, e, pair);
+      int32_t code = kNone;
+      float bias = -INFINITY;
+      if (s >= 0 && s < p.S) {
+        code = ri[i];
+        if (code < 0 || (int64_t)code >= p.T_cap) { bad = 1; code = 0; }
+        int dg = rd[i];
+        if (dg < 1) { bad = 1; dg = 1; }
+        bias = log2f((float)dg);
+      } else if (s >= 0 && s < total) {
+        code = -(s - p.S) - 1;
+        bias = 0.f;
+      }
+      trow[buf * kTabE + e] = code;
+      tbias[buf * kTabE + e] = bias;
+    }
+    if (bad && p.err_flag) atomicExch(p.err_flag, 1);
+    __syncwarp();
+  };
+
+  const int nb = (n + kTB - 1) / kTB;
+  load_batch(0);
+  store_batch(0);
+  int pending = 1;                                   // batch whose raw values are in ri/rd
+  if (nb > 1) load_batch(1);
+
+  // The table of batch b is staged when the copies first reach it; the compute trails
+  // by fewer than kTB tiles, so the other buffer still holds what it reads.
   auto issue = [&](int it, int st) {
-    const int ts = (warp + it * kDraftWarps) * kTile;
+    const int b = it / kTB;
+    if (b == pending) {
+      store_batch(b);
+      ++pending;
+      if (pending < nb) load_batch(pending);
+    }
+    const int64_t x = x0 + it;
+    const int64_t pair = x / p.tpp;
+    const __nv_bfloat16* kb = p.k + pair * p.T_cap * D;
+    const __nv_bfloat16* vb = p.v + pair * p.T_cap * D;
+    const __nv_bfloat16* kt = p.k_tail ? p.k_tail + pair * p.R_cap * D : kb;
+    const __nv_bfloat16* vt = p.v_tail ? p.v_tail + pair * p.R_cap * D : vb;
+    const int e0 = (b & 1) * kTabE + (it % kTB) * kTile;
     const uint32_t kd = wbuf_s + st * SM::kStageB;
     const uint32_t vd = kd + SM::kTileB;
 #pragma unroll
     for (int i = 0; i < kTile * CH / 32; ++i) {
       const int lin = lane + 32 * i;
       const int r = lin / CH, c = lin % CH;
-      const int sl = ts + r;
-      const bool ok = sl < n_here;
-      const int32_t row = ok ? srow[sl] : 0;
-      const __nv_bfloat16* kp = row >= 0 ? kb + (int64_t)row * D : kt + (int64_t)(-row - 1) * D;
-      const __nv_bfloat16* vp = row >= 0 ? vb + (int64_t)row * D : vt + (int64_t)(-row - 1) * D;
+      const int32_t code = trow[e0 + r];
+      const bool ok = code != kNone;
+      const __nv_bfloat16* kp =
+          code >= 0 ? kb + (int64_t)code * D : (ok ? kt + (int64_t)(-code - 1) * D : kb);
+      const __nv_bfloat16* vp =
+          code >= 0 ? vb + (int64_t)code * D : (ok ? vt + (int64_t)(-code - 1) * D : vb);
       const uint32_t off = r * SM::kRowB + ((c ^ (r & 7)) << 4);
       cp_async16(kd + off, kp + c * 8, ok ? 16u : 0u);
       cp_async16(vd + off, vp + c * 8, ok ? 16u : 0u);
@@ -121,38 +185,72 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
 
   // ---- query fragments (A operand rows = heads of the group; rows >= g are zero)
   const int qr = lane >> 2, qc = lane & 3;
-  uint32_t qa[D / 16][2];
-  {
+  uint32_t qa[D / 16][2], qn[D / 16][2];
+  auto load_q = [&](int64_t pair, uint32_t (&dst)[D / 16][2]) {
+    const int64_t b = pair / p.Hkv, j = pair - b * p.Hkv;
     const bool ok = qr < p.g;
-    const uint32_t* qp = reinterpret_cast<const uint32_t*>(
-        p.q + ((int64_t)b * p.Hq + j * p.g + (ok ? qr : 0)) * D);
+    const uint32_t* qp =
+        reinterpret_cast<const uint32_t*>(p.q + (b * p.Hq + j * p.g + (ok ? qr : 0)) * D);
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
-      qa[ks][0] = ok ? qp[(16 * ks + 2 * qc) / 2] : 0u;
-      qa[ks][1] = ok ? qp[(16 * ks + 8 + 2 * qc) / 2] : 0u;
+      dst[ks][0] = ok ? __ldg(qp + (16 * ks + 2 * qc) / 2) : 0u;
+      dst[ks][1] = ok ? __ldg(qp + (16 * ks + 8 + 2 * qc) / 2) : 0u;
     }
-  }
+  };
+  const int64_t pair_first = x0 / p.tpp;
+  const int64_t pair_last = (x0 + n - 1) / p.tpp;
+  load_q(pair_first, qa);
+  if (pair_last > pair_first) load_q(pair_first + 1, qn);
 
   float o[NT][4];
+  float m_run, l_run;
+  auto reset = [&]() {
 #pragma unroll
-  for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;
+    for (int nn = 0; nn < NT; ++nn) o[nn][0] = o[nn][1] = o[nn][2] = o[nn][3] = 0.f;
+    m_run = -INFINITY;
+    l_run = 0.f;
+  };
+  auto flush = [&](int64_t pair) {
+    float l = l_run + __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    const int64_t seg = gw - warp_of_tile(pair * p.tpp, p.T, p.W);
+    const int64_t part = (pair * p.maxseg + seg) * p.g;
+    if (qr < p.g) {
+      float* dst = p.ws_o + (part + qr) * D;
+#pragma unroll
+      for (int nn = 0; nn < NT; ++nn)
+        *reinterpret_cast<float2*>(dst + nn * 8 + 2 * qc) =
+            make_float2(o[nn][0] + o[nn][2], o[nn][1] + o[nn][3]);
+      if (qc == 0) *reinterpret_cast<float2*>(p.ws_ml + (part + qr) * 2) = make_float2(m_run, l);
+    }
+  };
+  reset();
+  int64_t cur = pair_first;
 
 #pragma unroll
   for (int st = 0; st < NST - 1; ++st) {
-    if (st < my_tiles) issue(st, st);
+    if (st < n) issue(st, st);
     cp_async_commit();
   }
 
-  for (int it = 0; it < my_tiles; ++it) {
-    if (it + NST - 1 < my_tiles) issue(it + NST - 1, (it + NST - 1) % NST);
+  for (int it = 0; it < n; ++it) {
+    if (it + NST - 1 < n) issue(it + NST - 1, (it + NST - 1) % NST);
     cp_async_commit();
     cp_async_wait<NST - 1>();
     __syncwarp();
+    const int64_t pair = (x0 + it) / p.tpp;
+    if (pair != cur) {                               // segment boundary
+      flush(cur);
+      reset();
+      cur = pair;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) { qa[ks][0] = qn[ks][0]; qa[ks][1] = qn[ks][1]; }
+      if (pair < pair_last) load_q(pair + 1, qn);
+    }
     const int st = it % NST;
     const uint32_t ks_base = wbuf_s + st * SM::kStageB;
     const uint32_t vs_base = ks_base + SM::kTileB;
-    const int ts = (warp + it * kDraftWarps) * kTile;
+    const int e0 = ((it / kTB) & 1) * kTabE + (it % kTB) * kTile;
 
     // S = Q K^T over two n-tiles of 8 slots
     float s[2][4];
@@ -170,14 +268,13 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
         mma_bf16(s[nt], qa[2 * kk + 1][0], 0u, qa[2 * kk + 1][1], 0u, b2, b3);
       }
     }
-    // log2-domain scores with degree bias and the ragged-tile mask
+    // log2-domain scores; the bias of a slot past the end is -inf (masked)
     float mx = -INFINITY;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int sl = ts + nt * 8 + 2 * qc + e;
-        const float v2 = sl < n_here ? fmaf(s[nt][e], p.qk_scale2, sbias[sl]) : -INFINITY;
+        const float v2 = fmaf(s[nt][e], p.qk_scale2, tbias[e0 + nt * 8 + 2 * qc + e]);
         s[nt][e] = v2;
         mx = fmaxf(mx, v2);
       }
@@ -196,8 +293,8 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
       }
     l_run = fmaf(l_run, alpha, psum);
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      o[n][0] *= alpha; o[n][1] *= alpha; o[n][2] *= alpha; o[n][3] *= alpha;
+    for (int nn = 0; nn < NT; ++nn) {
+      o[nn][0] *= alpha; o[nn][1] *= alpha; o[nn][2] *= alpha; o[nn][3] *= alpha;
     }
     // P as bf16 high part (A rows 0-7, the heads) plus bf16 low part (A rows 8-15,
     // otherwise padding): the two accumulator halves sum to P.V with P kept to
@@ -206,7 +303,6 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
     const uint32_t ph2 = pack_bf16x2(s[1][0], s[1][1]);
     const uint32_t pl0 = pack_bf16x2(s[0][0] - bf16_lo(ph0), s[0][1] - bf16_hi(ph0));
     const uint32_t pl2 = pack_bf16x2(s[1][0] - bf16_lo(ph2), s[1][1] - bf16_hi(ph2));
-    // O += P V
 #pragma unroll
     for (int n2 = 0; n2 < NT / 2; ++n2) {
       const int mi = lane >> 3;
@@ -220,109 +316,94 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
     __syncwarp();
   }
   cp_async_wait<0>();
-
-  // ---- merge the 4 warps of the CTA through shared memory
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-  __syncthreads();
-  float* red = reinterpret_cast<float*>(smem);          // [4][8][D + 2]
-  constexpr int RS = D + 2;
-  float* mine = red + (warp * 8 + qr) * RS;
-#pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    mine[n * 8 + 2 * qc] = o[n][0] + o[n][2];
-    mine[n * 8 + 2 * qc + 1] = o[n][1] + o[n][3];
-  }
-  if (qc == 0) { mine[D] = m_run; mine[D + 1] = l_run; }
-  __syncthreads();
-  const int64_t part = (int64_t)pair * p.n_split + split;
-  for (int t = threadIdx.x; t < p.g * D; t += blockDim.x) {
-    const int r = t / D, d = t - r * D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kDraftWarps; ++w) M = fmaxf(M, red[(w * 8 + r) * RS + D]);
-    float L = 0.f, O = 0.f;
-#pragma unroll
-    for (int w = 0; w < kDraftWarps; ++w) {
-      const float* row = red + (w * 8 + r) * RS;
-      const float f = ex2(row[D] - M);
-      L = fmaf(row[D + 1], f, L);
-      O = fmaf(row[d], f, O);
-    }
-    p.ws_o[(part * p.g + r) * D + d] = O;
-    if (d == 0) {
-      p.ws_ml[(part * p.g + r) * 2] = M;
-      p.ws_ml[(part * p.g + r) * 2 + 1] = L;
-    }
-  }
+  flush(cur);
 }
 
-// Fixed-order merge of the split partials of every head -> bf16 output (+ lse).
+// Fixed-order merge of the partials of one head: block (pair, head), D threads.
 template <int D, typename OutT>
-__global__ void __launch_bounds__(256) draft_combine_kernel(const float* __restrict__ ws_o,
-                                                            const float* __restrict__ ws_ml,
-                                                            int n_split, int g, int Hkv, int Hq,
-                                                            OutT* __restrict__ out,
-                                                            float* __restrict__ lse) {
-  const int pair = blockIdx.x;
-  const int b = pair / Hkv, j = pair - b * Hkv;
-  for (int t = threadIdx.x; t < g * D; t += blockDim.x) {
-    const int r = t / D, d = t - r * D;
-    float M = -INFINITY;
-    for (int s = 0; s < n_split; ++s)
-      M = fmaxf(M, ws_ml[(((int64_t)pair * n_split + s) * g + r) * 2]);
-    float L = 0.f, O = 0.f;
-    for (int s = 0; s < n_split; ++s) {
-      const int64_t pr = ((int64_t)pair * n_split + s) * g + r;
-      const float f = ex2(ws_ml[pr * 2] - M);
-      L = fmaf(ws_ml[pr * 2 + 1], f, L);
-      O = fmaf(ws_o[pr * D + d], f, O);
-    }
-    const int64_t h = (int64_t)b * Hq + j * g + r;
-    store_out(out + h * D + d, O / L);
-    if (lse && d == 0) lse[h] = (M + __log2f(L)) * kLn2;
+__global__ void __launch_bounds__(D) draft_combine_kernel(const DraftIndexedParams p,
+                                                          OutT* __restrict__ out,
+                                                          float* __restrict__ lse) {
+  const int64_t pair = blockIdx.x / p.g;
+  const int r = blockIdx.x - (int)(pair * p.g);
+  const int d = threadIdx.x;
+  const int64_t w0 = warp_of_tile(pair * p.tpp, p.T, p.W);
+  const int64_t w1 = warp_of_tile((pair + 1) * p.tpp - 1, p.T, p.W);
+  float M = -INFINITY, L = 0.f, O = 0.f;
+#pragma unroll 4
+  for (int64_t w = w0; w <= w1; ++w) {
+    if (warp_begin(w, p.T, p.W) >= warp_begin(w + 1, p.T, p.W)) continue;   // empty range
+    const int64_t pr = (pair * p.maxseg + (w - w0)) * p.g + r;
+    const float2 ml = *reinterpret_cast<const float2*>(p.ws_ml + pr * 2);
+    const float os = p.ws_o[pr * D + d];
+    const float Mn = fmaxf(M, ml.x);
+    const float a = ex2(M - Mn), c = ex2(ml.x - Mn);
+    L = fmaf(L, a, ml.y * c);
+    O = fmaf(O, a, os * c);
+    M = Mn;
   }
+  const int64_t b = pair / p.Hkv, j = pair - b * p.Hkv;
+  const int64_t h = b * p.Hq + j * p.g + r;
+  store_out(out + h * D + d, O / L);
+  if (lse && d == 0) lse[h] = (M + __log2f(L)) * kLn2;
 }
 
 // ------------------------------------------------------------------ host side
 namespace {
 constexpr int kNStage = 3;
 
-int draft_chunk(int pairs, int total, int* n_split_out) {
-  const int target = 4 * num_sms();
-  int n_split = (target + pairs - 1) / pairs;
-  int chunk = (total + n_split - 1) / n_split;
-  chunk = ((chunk + 63) / 64) * 64;
-  if (chunk < 64) chunk = 64;
-  if (chunk > 2048) chunk = 2048;
-  *n_split_out = (total + chunk - 1) / chunk;
-  return chunk;
+struct DraftPlan {
+  int tpp, W, maxseg;
+  int64_t T;
+};
+
+DraftPlan draft_plan(int pairs, int total) {
+  DraftPlan pl;
+  pl.tpp = (total + kTile - 1) / kTile;
+  pl.T = (int64_t)pairs * pl.tpp;
+  const int64_t ctas = std::min<int64_t>(2 * (int64_t)num_sms(),
+                                         std::max<int64_t>(1, pl.T / kDraftWarps));
+  pl.W = (int)(ctas * kDraftWarps);
+  int ms = 1;
+  for (int64_t pr = 0; pr < pairs; ++pr) {
+    const int64_t a = warp_of_tile(pr * pl.tpp, pl.T, pl.W);
+    const int64_t b = warp_of_tile((pr + 1) * pl.tpp - 1, pl.T, pl.W);
+    ms = std::max<int>(ms, (int)(b - a + 1));
+  }
+  pl.maxseg = ms;
+  return pl;
 }
 
 template <int D>
-size_t draft_indexed_smem(int chunk) {
-  return (size_t)kDraftWarps * kNStage * DraftSmem<D>::kStageB + (size_t)chunk * 8;
+size_t draft_indexed_smem() {
+  return (size_t)kDraftWarps * (kNStage * DraftSmem<D>::kStageB + DraftSmem<D>::kTableB);
 }
 }  // namespace
 
 size_t draft_workspace_bytes(const vc_comp_cache* c) {
   const int pairs = c->B * c->Hkv;
   const int total = c->S + c->n_tail;
-  int n_split = 1;
-  draft_chunk(pairs, total > 0 ? total : 1, &n_split);
+  const DraftPlan pl = draft_plan(pairs, total > 0 ? total : 1);
   const int g = c->Hq / c->Hkv;
-  return (size_t)pairs * n_split * g * ((size_t)c->D + 2) * sizeof(float) + 256;
+  return (size_t)pairs * pl.maxseg * g * ((size_t)c->D + 2) * sizeof(float) + 256;
 }
 
 template <int D>
-static void launch_draft_combine(const DraftIndexedParams& p, int pairs, int flags, void* out,
-                                 float* lse, cudaStream_t stream) {
+static vc_status launch_draft_d(const DraftIndexedParams& p, int flags, void* out, float* lse,
+                                cudaStream_t stream) {
+  const size_t sm = draft_indexed_smem<D>();
+  VC_CUDA(cudaFuncSetAttribute(draft_indexed_kernel<D, kNStage>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+  draft_indexed_kernel<D, kNStage><<<p.W / kDraftWarps, 128, sm, stream>>>(p);
+  VC_CUDA(cudaGetLastError());
+  const int blocks = (int)(p.T / p.tpp) * p.g;   // one per (pair, head)
   if (flags & VC_OUT_F32)
-    draft_combine_kernel<D, float><<<pairs, 256, 0, stream>>>(
-        p.ws_o, p.ws_ml, p.n_split, p.g, p.Hkv, p.Hq, static_cast<float*>(out), lse);
+    draft_combine_kernel<D, float><<<blocks, D, 0, stream>>>(p, static_cast<float*>(out), lse);
   else
-    draft_combine_kernel<D, __nv_bfloat16><<<pairs, 256, 0, stream>>>(
-        p.ws_o, p.ws_ml, p.n_split, p.g, p.Hkv, p.Hq, static_cast<__nv_bfloat16*>(out), lse);
+    draft_combine_kernel<D, __nv_bfloat16><<<blocks, D, 0, stream>>>(
+        p, static_cast<__nv_bfloat16*>(out), lse);
+  VC_CUDA(cudaGetLastError());
+  return VC_OK;
 }
 
 vc_status launch_draft_indexed(const void* q, const vc_comp_cache* c, float scale, int flags,
@@ -330,6 +411,7 @@ vc_status launch_draft_indexed(const void* q, const vc_comp_cache* c, float scal
                                cudaStream_t stream) {
   const int pairs = c->B * c->Hkv;
   const int total = c->S + c->n_tail;
+  const DraftPlan pl = draft_plan(pairs, total);
   DraftIndexedParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k = static_cast<const __nv_bfloat16*>(c->k);
@@ -346,31 +428,18 @@ vc_status launch_draft_indexed(const void* q, const vc_comp_cache* c, float scal
   p.Hq = c->Hq;
   p.Hkv = c->Hkv;
   p.g = c->Hq / c->Hkv;
-  p.chunk = draft_chunk(pairs, total, &p.n_split);
+  p.tpp = pl.tpp;
+  p.T = pl.T;
+  p.W = pl.W;
+  p.maxseg = pl.maxseg;
   p.qk_scale2 = scale * kLog2e;
-  const size_t ws_need = (size_t)pairs * p.n_split * p.g * ((size_t)c->D + 2) * sizeof(float);
+  const size_t ws_need = (size_t)pairs * pl.maxseg * p.g * ((size_t)c->D + 2) * sizeof(float);
   if (ws_bytes < ws_need) return fail(VC_ERR_INVALID, "draft workspace too small");
   p.ws_o = static_cast<float*>(ws);
-  p.ws_ml = p.ws_o + (size_t)pairs * p.n_split * p.g * c->D;
+  p.ws_ml = p.ws_o + (size_t)pairs * pl.maxseg * p.g * c->D;
   p.err_flag = c->err_flag;
-  dim3 grid(p.n_split, pairs);
-  if (c->D == 128) {
-    const size_t sm = draft_indexed_smem<128>(p.chunk);
-    VC_CUDA(cudaFuncSetAttribute(draft_indexed_kernel<128, kNStage>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-    draft_indexed_kernel<128, kNStage><<<grid, 128, sm, stream>>>(p);
-    VC_CUDA(cudaGetLastError());
-    launch_draft_combine<128>(p, pairs, flags, out, lse, stream);
-  } else {
-    const size_t sm = draft_indexed_smem<64>(p.chunk);
-    VC_CUDA(cudaFuncSetAttribute(draft_indexed_kernel<64, kNStage>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-    draft_indexed_kernel<64, kNStage><<<grid, 128, sm, stream>>>(p);
-    VC_CUDA(cudaGetLastError());
-    launch_draft_combine<64>(p, pairs, flags, out, lse, stream);
-  }
-  VC_CUDA(cudaGetLastError());
-  return VC_OK;
+  if (c->D == 128) return launch_draft_d<128>(p, flags, out, lse, stream);
+  return launch_draft_d<64>(p, flags, out, lse, stream);
 }
 
 }  // namespace vc

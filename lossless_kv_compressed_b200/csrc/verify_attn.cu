@@ -14,13 +14,14 @@
 //
 // Per CTA (384 threads):
 //   warp 0      TMA producer: K and V tiles [64 keys x D] (128-byte swizzle) into a
-//               2-stage ring, one mbarrier per stage with the transaction byte count.
+//               4-stage ring, one mbarrier per stage with the transaction byte count.
 //   warp 1      TMEM allocator and UMMA issuer (one thread): S = Q K^T into TMEM per
 //               M-tile, then O += P V with P from shared memory and V as an N-major B.
 //   warps 4-7   softmax of M-tile 0, warps 8-11 of M-tile 1: one thread per query row
 //               (TMEM lane), scores in the log2 domain, running max kept unless it grows
 //               by more than 2^8 (then O in TMEM is rescaled after the previous P.V),
-//               P written as bf16 into a double-buffered 128-byte-swizzled tile.
+//               P written as bf16 into a 128-byte-swizzled tile per M-tile (free
+//               again once the previous P.V has retired).
 // TMEM columns: S0 [0,64), S1 [64,128), O0 [128,128+D), O1 [128+D,128+2D).
 // Every mbarrier wait is bounded in time; on expiry the CTA raises the library's device
 // error word, releases TMEM and exits.
@@ -40,7 +41,7 @@ __device__ int g_vc_dev_error;   // bit 0: a bounded wait in the verify kernel e
 constexpr int kSplitKeys = 4096;
 constexpr int kBN = 64;
 constexpr int kVThreads = 384;
-constexpr int kNSt = 2;
+constexpr int kNSt = 4;
 constexpr float kRescaleLog2 = 8.f;
 
 struct VerifyParams {
@@ -62,8 +63,8 @@ struct VLayout {
   static constexpr int kK = kQ + 2 * kQTile;
   static constexpr int kV = kK + kNSt * kKVTile;
   static constexpr int kP = kV + kNSt * kKVTile;
-  static constexpr int kBar = kP + 4 * kPTile;
-  static constexpr int kNBar = 2 * kNSt + 2 + 2 + 4 + 4 + 1;
+  static constexpr int kBar = kP + 2 * kPTile;
+  static constexpr int kNBar = 2 * kNSt + 2 + 2 + 2 + 2 + 1;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kTotal = kAbort + 4;
@@ -112,9 +113,9 @@ __global__ void __launch_bounds__(kVThreads, 1)
   auto b_kv_empty = [&](int st) { return bar(kNSt + st); };
   auto b_s_full = [&](int mt) { return bar(2 * kNSt + mt); };
   auto b_s_free = [&](int mt) { return bar(2 * kNSt + 2 + mt); };
-  auto b_p_full = [&](int mt, int buf) { return bar(2 * kNSt + 4 + mt * 2 + buf); };
-  auto b_o_done = [&](int mt, int buf) { return bar(2 * kNSt + 8 + mt * 2 + buf); };
-  const uint32_t b_teardown = bar(2 * kNSt + 12);
+  auto b_p_full = [&](int mt) { return bar(2 * kNSt + 4 + mt); };
+  auto b_o_done = [&](int mt) { return bar(2 * kNSt + 6 + mt); };
+  const uint32_t b_teardown = bar(2 * kNSt + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
 
   auto nw_active = [&](int mt) {
@@ -130,10 +131,8 @@ __global__ void __launch_bounds__(kVThreads, 1)
     for (int mt = 0; mt < 2; ++mt) {
       tc::mbar_init(b_s_full(mt), 1);
       tc::mbar_init(b_s_free(mt), max(1, nw_active(mt)));
-      for (int buf = 0; buf < 2; ++buf) {
-        tc::mbar_init(b_p_full(mt, buf), max(1, nw_active(mt)));
-        tc::mbar_init(b_o_done(mt, buf), 1);
-      }
+      tc::mbar_init(b_p_full(mt), max(1, nw_active(mt)));
+      tc::mbar_init(b_o_done(mt), 1);
     }
     tc::mbar_init(b_teardown, 1);
     *abort_flag = 0;
@@ -212,10 +211,10 @@ __global__ void __launch_bounds__(kVThreads, 1)
         }
       };
       auto pv = [&](int t, int mt) {
-        const int st = t % kNSt, buf = t & 1;
+        const int st = t % kNSt;
 #pragma unroll
         for (int ks = 0; ks < kBN / 16; ++ks) {
-          const uint32_t a = sb + L::kP + (mt * 2 + buf) * L::kPTile + ks * 32;
+          const uint32_t a = sb + L::kP + mt * L::kPTile + ks * 32;
           const uint32_t bb = sb + L::kV + st * L::kKVTile + ks * 16 * 128;
           tc::umma_ss(tmem + 128 + mt * D, tc::sdesc_sw128(a, 16, 1024),
                       tc::sdesc_sw128(bb, kBN * 128, 1024), id_pv, (t > 0 || ks > 0) ? 1u : 0u);
@@ -241,10 +240,10 @@ __global__ void __launch_bounds__(kVThreads, 1)
             qk(t + 1, mt);
             tc::umma_commit(b_s_full(mt));
           }
-          if (!(ok = tc::mbar_wait(b_p_full(mt, t & 1), (t >> 1) & 1, abort_flag))) break;
+          if (!(ok = tc::mbar_wait(b_p_full(mt), t & 1, abort_flag))) break;
           tc::tc_fence_after();
           pv(t, mt);
-          tc::umma_commit(b_o_done(mt, t & 1));
+          tc::umma_commit(b_o_done(mt));
         }
         if (!ok) break;
         tc::umma_commit(b_kv_empty(t % kNSt));
@@ -279,20 +278,29 @@ __global__ void __launch_bounds__(kVThreads, 1)
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(b_s_free(mt));
+        // visible columns j in [lo, hi] of this tile for this row (int32, clamped)
         const int64_t key0 = (tile0 + t) * kBN;
-        const int64_t lo = a0 - key0, hi = min(a1 - 1, limit) - key0;   // visible j in [lo, hi]
-        float mx = -INFINITY;
+        const int lo = (int)max((int64_t)0, min((int64_t)kBN, a0 - key0));
+        const int hi = (int)max((int64_t)-1, min((int64_t)(kBN - 1), min(a1 - 1, limit) - key0));
+        // Row max on the raw scores (the scale is positive, so it commutes with max);
+        // a tile every row of the warp sees whole skips the per-column mask.
+        float mraw = -INFINITY;
+        if (__all_sync(0xffffffffu, lo == 0 && hi == kBN - 1)) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const float v = (j >= lo && j <= hi) ? __uint_as_float(sr[j]) * p.qk_scale2 : -INFINITY;
-          sr[j] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
+          for (int j = 0; j < 64; ++j) mraw = fmaxf(mraw, __uint_as_float(sr[j]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            const float v = (j >= lo && j <= hi) ? __uint_as_float(sr[j]) : -INFINITY;
+            sr[j] = __float_as_uint(v);
+            mraw = fmaxf(mraw, v);
+          }
         }
+        const float mx = mraw * p.qk_scale2;
         const float m_new = fmaxf(m_used, mx);
         const bool resc = m_new > m_used + kRescaleLog2;
         if (t > 0 && __any_sync(0xffffffffu, resc)) {
-          ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt, (t - 1) & 1),
-                                                     ((t - 1) >> 1) & 1, abort_flag));
+          ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt), (t - 1) & 1, abort_flag));
           if (!ok) break;
           tc::tc_fence_after();
           const float alpha = resc ? ex2(m_used - m_new) : 1.f;
@@ -310,19 +318,19 @@ __global__ void __launch_bounds__(kVThreads, 1)
         }
         if (resc) m_used = m_new;
         const float m_safe = m_used == -INFINITY ? 0.f : m_used;
-        if (t >= 2) {
-          ok = __all_sync(0xffffffffu,
-                          tc::mbar_wait(b_o_done(mt, t & 1), ((t - 2) >> 1) & 1, abort_flag));
+        // the single P tile of this M-tile is free once the previous P.V has retired
+        if (t >= 1) {
+          ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt), (t - 1) & 1, abort_flag));
           if (!ok) break;
         }
-        uint8_t* prow = smem + L::kP + (mt * 2 + (t & 1)) * L::kPTile + r * 128;
+        uint8_t* prow = smem + L::kP + mt * L::kPTile + r * 128;
         float rs = 0.f;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           float e[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            e[u] = ex2(__uint_as_float(sr[8 * c + u]) - m_safe);
+            e[u] = ex2(fmaf(__uint_as_float(sr[8 * c + u]), p.qk_scale2, -m_safe));
             rs += e[u];
           }
           uint4 pk;
@@ -336,12 +344,11 @@ __global__ void __launch_bounds__(kVThreads, 1)
         tc::fence_proxy_async();
         tc::tc_fence_before();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(b_p_full(mt, t & 1));
+        if (lane == 0) tc::mbar_arrive(b_p_full(mt));
       }
       if (ok) {
         const int tl = n_tiles - 1;
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt, tl & 1), (tl >> 1) & 1,
-                                                   abort_flag));
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt), tl & 1, abort_flag));
       }
       if (!ok) {
         raise();
