@@ -319,31 +319,345 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
   flush(cur);
 }
 
-// Fixed-order merge of the partials of one head: block (pair, head), D threads.
+// ------------------------------------------------------------------ int4 cache
+// Draft attention over the 4-bit cache (layout in vericache.h): the same persistent
+// per-warp ranges, over (pair, 32-token block) units.  A block's packed K and V words
+// and its fp16 scales / zeros are five contiguous runs (5 KB at D = 128) copied into a
+// per-warp cp.async ring.  The word layout matches the mma.sync fragments, so a thread
+// reads exactly its own nibbles: one 16-byte load per token for K, one word per channel
+// for V.  The nibbles stay exact (ORed into the mantissa of fp16 1024, then 1024
+// subtracted) and the scales move to the other operand, so nothing proportional to a
+// dequantised value is ever rounded to fp16:
+//   q . k_hat = sum_d (q_d s_d) n_d + sum_d q_d z_d              (K: per channel)
+//   sum_t p_t v_hat_t = sum_t (p_t s_t)(n_t - 7.5) + sum_t p_t (z_t + 7.5 s_t)
+//                                                                 (V: per token, group;
+//   centred so that neither sum is much larger than the result)
+// q_d s_d and p_t s_t are split into fp16 high and low parts placed in A rows 0-7 and
+// 8-15 (rows 8-15 are padding: g <= 8), so one f16 mma.sync carries both and the two
+// accumulator halves add up to ~22 mantissa bits.  The zero-point sum over tokens is
+// one more mma per 16 tokens; sum_d q_d z_d is an fp32 dot product.
+struct DraftInt4Params {
+  const __nv_bfloat16* q;
+  const uint32_t* kq;            // [pairs, nblk_cap, 32, 4, D/32]
+  const __half* ks;              // [pairs, nblk_cap, D]
+  const __half* kz;
+  const uint32_t* vq;            // [pairs, nblk_cap, D, 4]
+  const __half* vs;              // [pairs, nblk_cap, D/32, 32]
+  const __half* vz;
+  int64_t nblk_cap;
+  int nblk;                      // live blocks per pair
+  int Hq, Hkv, g;
+  int64_t T;                     // pairs * nblk
+  int W, maxseg;
+  float qk_scale2;
+  float* ws_o;
+  float* ws_ml;
+};
+
+template <int D>
+struct Int4Smem {
+  static constexpr int kKW = 16 * D;     // 32 tokens x D/2 bytes
+  static constexpr int kVW = 16 * D;     // D channels x 4 words
+  static constexpr int kSZ = 2 * D;      // one fp16 per channel (K) / per token-group (V)
+  static constexpr int kStageB = kKW + kVW + 4 * kSZ;
+};
+
+// Nibble pair j of word w as exact fp16x2 integers (n0, n1).
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int j) {
+  const uint32_t x = ((w >> (4 * j)) & 0x000F000Fu) | 0x64006400u;   // 1024 + n
+  uint32_t n;
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(n) : "r"(x), "r"(0x64006400u));
+  return n;
+}
+// Same, centred on the middle of the 4-bit range: (n0 - 7.5, n1 - 7.5), still exact.
+__device__ __forceinline__ uint32_t nib_pair_c(uint32_t w, int j) {
+  uint32_t c;
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(c) : "r"(nib_pair(w, j)), "r"(0x47804780u));
+  return c;
+}
+__device__ __forceinline__ float2 h2f(uint32_t h) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+// (a, b) -> fp16x2 high part and fp16x2 low part (a - hi, b - hi).
+__device__ __forceinline__ void split_f16(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack_f16x2(a, b);
+  const float2 h = h2f(hi);
+  lo = pack_f16x2(a - h.x, b - h.y);
+}
+
+template <int D, int NST>
+__global__ void __launch_bounds__(128, 2) draft_int4_kernel(const DraftInt4Params p) {
+  using SM = Int4Smem<D>;
+  constexpr int NT = D / 8;
+  constexpr int NW = D / 32;                 // K words per (token, c); channel groups of V
+  constexpr int CH = SM::kStageB / 16;       // 16-byte chunks per block
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t)blockIdx.x * kDraftWarps + warp;
+  const int64_t x0 = warp_begin(gw, p.T, p.W);
+  const int n = (int)(warp_begin(gw + 1, p.T, p.W) - x0);
+  if (n <= 0) return;
+  const uint32_t wbuf_s = smem_u32(smem + warp * NST * SM::kStageB);
+  uint8_t* wbuf = smem + warp * NST * SM::kStageB;
+
+  auto issue = [&](int it, int st) {
+    const int64_t x = x0 + it;
+    const int64_t pair = x / p.nblk;
+    const int64_t blk = pair * p.nblk_cap + (x - pair * p.nblk);
+    const uint32_t dst = wbuf_s + st * SM::kStageB;
+#pragma unroll
+    for (int i = 0; i < (CH + 31) / 32; ++i) {
+      const int c = lane + 32 * i;
+      if (c < CH) {
+        const int off = c * 16;
+        const uint8_t* src;
+        if (off < SM::kKW) {
+          src = reinterpret_cast<const uint8_t*>(p.kq + blk * (32 * 4 * NW)) + off;
+        } else if (off < SM::kKW + SM::kVW) {
+          src = reinterpret_cast<const uint8_t*>(p.vq + blk * (D * 4)) + (off - SM::kKW);
+        } else {
+          const int o2 = off - SM::kKW - SM::kVW;
+          const int part = o2 / SM::kSZ, rel = o2 - part * SM::kSZ;
+          const __half* base = part == 0 ? p.ks : part == 1 ? p.kz : part == 2 ? p.vs : p.vz;
+          src = reinterpret_cast<const uint8_t*>(base + blk * D) + rel;
+        }
+        cp_async16(dst + off, src, 16u);
+      }
+    }
+  };
+
+  const int qr = lane >> 2, qc = lane & 3;
+  uint32_t qa[D / 16][2], qn[D / 16][2];
+  auto load_q = [&](int64_t pair, uint32_t (&dst)[D / 16][2]) {
+    const int64_t b = pair / p.Hkv, j = pair - b * p.Hkv;
+    const bool ok = qr < p.g;
+    const uint32_t* qp =
+        reinterpret_cast<const uint32_t*>(p.q + (b * p.Hq + j * p.g + (ok ? qr : 0)) * D);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {       // raw bf16 pairs, widened when used
+      dst[ks][0] = ok ? __ldg(qp + (16 * ks + 2 * qc) / 2) : 0u;
+      dst[ks][1] = ok ? __ldg(qp + (16 * ks + 8 + 2 * qc) / 2) : 0u;
+    }
+  };
+  const int64_t pair_first = x0 / p.nblk;
+  const int64_t pair_last = (x0 + n - 1) / p.nblk;
+  load_q(pair_first, qa);
+  if (pair_last > pair_first) load_q(pair_first + 1, qn);
+
+  float o[NT][4];
+  float zacc[4];
+  float m_run, l_run;
+  auto reset = [&]() {
+#pragma unroll
+    for (int nn = 0; nn < NT; ++nn) o[nn][0] = o[nn][1] = o[nn][2] = o[nn][3] = 0.f;
+    zacc[0] = zacc[1] = zacc[2] = zacc[3] = 0.f;
+    m_run = -INFINITY;
+    l_run = 0.f;
+  };
+  auto flush = [&](int64_t pair) {
+    float l = l_run + __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    // zero-point term of group G for row qr: columns G of the zacc tile (lane qr*4 + G/2)
+    const float zc0 = zacc[0] + zacc[2], zc1 = zacc[1] + zacc[3];
+    float zt[NW];
+#pragma unroll
+    for (int G = 0; G < NW; ++G) {
+      const float a = __shfl_sync(0xffffffffu, zc0, qr * 4 + G / 2);
+      const float b = __shfl_sync(0xffffffffu, zc1, qr * 4 + G / 2);
+      zt[G] = (G & 1) ? b : a;
+    }
+    const int64_t seg = gw - warp_of_tile(pair * p.nblk, p.T, p.W);
+    const int64_t part = (pair * p.maxseg + seg) * p.g;
+    if (qr < p.g) {
+      float* dst = p.ws_o + (part + qr) * D;
+#pragma unroll
+      for (int nn = 0; nn < NT; ++nn)
+        *reinterpret_cast<float2*>(dst + nn * 8 + 2 * qc) =
+            make_float2(o[nn][0] + o[nn][2] + zt[nn / 4], o[nn][1] + o[nn][3] + zt[nn / 4]);
+      if (qc == 0) *reinterpret_cast<float2*>(p.ws_ml + (part + qr) * 2) = make_float2(m_run, l);
+    }
+  };
+  reset();
+  int64_t cur = pair_first;
+
+#pragma unroll
+  for (int st = 0; st < NST - 1; ++st) {
+    if (st < n) issue(st, st);
+    cp_async_commit();
+  }
+  for (int it = 0; it < n; ++it) {
+    if (it + NST - 1 < n) issue(it + NST - 1, (it + NST - 1) % NST);
+    cp_async_commit();
+    cp_async_wait<NST - 1>();
+    __syncwarp();
+    const int64_t pair = (x0 + it) / p.nblk;
+    if (pair != cur) {
+      flush(cur);
+      reset();
+      cur = pair;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) { qa[ks][0] = qn[ks][0]; qa[ks][1] = qn[ks][1]; }
+      if (pair < pair_last) load_q(pair + 1, qn);
+    }
+    const uint8_t* sbase = wbuf + (it % NST) * SM::kStageB;
+    const uint32_t* kw = reinterpret_cast<const uint32_t*>(sbase);
+    const uint32_t* vw = reinterpret_cast<const uint32_t*>(sbase + SM::kKW);
+    const uint32_t* ksc = reinterpret_cast<const uint32_t*>(sbase + SM::kKW + SM::kVW);
+    const uint32_t* kzr = ksc + SM::kSZ / 4;
+    const uint32_t* vsc = kzr + SM::kSZ / 4;
+    const uint32_t* vzr = vsc + SM::kSZ / 4;
+
+    // ---- q'_d = q_d * s_d (per channel of this block) as hi/lo A fragments, and the
+    //      zero-point term c = sum_d q_d z_d of this thread's head (fp32)
+    uint32_t ah[D / 16][2], al[D / 16][2];
+    float cz = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int d0 = 16 * ks + 8 * h + 2 * qc;
+        const float2 sc = h2f(ksc[d0 / 2]), zc = h2f(kzr[d0 / 2]);
+        const float q0 = bf16_lo(qa[ks][h]), q1 = bf16_hi(qa[ks][h]);
+        split_f16(q0 * sc.x, q1 * sc.y, ah[ks][h], al[ks][h]);
+        cz = fmaf(q0, zc.x, fmaf(q1, zc.y, cz));
+      }
+    cz += __shfl_xor_sync(0xffffffffu, cz, 1);
+    cz += __shfl_xor_sync(0xffffffffu, cz, 2);
+
+    // ---- S = Q K^T over 4 n-tiles of 8 tokens (B = exact nibbles)
+    float s[4][4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+      const int t = nt * 8 + qr;
+      uint32_t w[NW];
+      if constexpr (NW == 4) {
+        const uint4 v4 = *reinterpret_cast<const uint4*>(kw + (t * 4 + qc) * NW);
+        w[0] = v4.x; w[1] = v4.y; w[2] = v4.z; w[3] = v4.w;
+      } else {
+        const uint2 v2 = *reinterpret_cast<const uint2*>(kw + (t * 4 + qc) * NW);
+        w[0] = v2.x; w[1] = v2.y;
+      }
+#pragma unroll
+      for (int wi = 0; wi < NW; ++wi)
+#pragma unroll
+        for (int hk = 0; hk < 2; ++hk) {            // k-step 2wi + hk
+          const int ks = 2 * wi + hk;
+          mma_f16(s[nt], ah[ks][0], al[ks][0], ah[ks][1], al[ks][1], nib_pair(w[wi], 2 * hk),
+                  nib_pair(w[wi], 2 * hk + 1));
+        }
+    }
+    // rows qr (high part) + rows qr+8 (low part) + zero-point term
+    float mx = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      s[nt][0] = (s[nt][0] + s[nt][2] + cz) * p.qk_scale2;
+      s[nt][1] = (s[nt][1] + s[nt][3] + cz) * p.qk_scale2;
+      mx = fmaxf(mx, fmaxf(s[nt][0], s[nt][1]));
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    const float alpha = ex2(m_run - m_new);
+    m_run = m_new;
+    float psum = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      s[nt][0] = ex2(s[nt][0] - m_new);
+      s[nt][1] = ex2(s[nt][1] - m_new);
+      psum += s[nt][0] + s[nt][1];
+    }
+    l_run = fmaf(l_run, alpha, psum);
+#pragma unroll
+    for (int nn = 0; nn < NT; ++nn) {
+      o[nn][0] *= alpha; o[nn][1] *= alpha; o[nn][2] *= alpha; o[nn][3] *= alpha;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) zacc[e] *= alpha;
+
+    // ---- zero-point term sum_t p_t z_t: A = p (hi/lo), B = zeros [tokens x groups]
+    {
+      uint32_t ph[4], pl[4];
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) split_f16(s[nt][0], s[nt][1], ph[nt], pl[nt]);
+      // B = z + 7.5 s, the value of the middle of each group's grid (the nibbles of V
+      // enter centred, so both sums stay of the size of the result: no cancellation)
+      auto zmid = [&](int t0) -> uint32_t {
+        const int o = (qr * 32 + t0) / 2;
+        const float2 z = h2f(vzr[o]), sc = h2f(vsc[o]);
+        return pack_f16x2(fmaf(7.5f, sc.x, z.x), fmaf(7.5f, sc.y, z.y));
+      };
+#pragma unroll
+      for (int kt = 0; kt < 2; ++kt) {
+        uint32_t z0 = 0u, z1 = 0u;
+        if (qr < NW) {
+          z0 = zmid(16 * kt + 2 * qc);
+          z1 = zmid(16 * kt + 8 + 2 * qc);
+        }
+        mma_f16(zacc, ph[2 * kt], pl[2 * kt], ph[2 * kt + 1], pl[2 * kt + 1], z0, z1);
+      }
+    }
+    // ---- O += (p s) N per channel group, B = exact nibbles of V
+#pragma unroll
+    for (int G = 0; G < NW; ++G) {
+      uint32_t pah[4], pal[4];                      // [kt * 2 + half]
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {                 // token pair 2qc + 8j: n-tile j
+        const float2 sv = h2f(vsc[(G * 32 + 2 * qc + 8 * j) / 2]);
+        split_f16(s[j][0] * sv.x, s[j][1] * sv.y, pah[j], pal[j]);
+      }
+#pragma unroll
+      for (int nn = 4 * G; nn < 4 * G + 4; ++nn) {
+        const uint32_t wv = vw[(nn * 8 + qr) * 4 + qc];
+        mma_f16(o[nn], pah[0], pal[0], pah[1], pal[1], nib_pair_c(wv, 0), nib_pair_c(wv, 1));
+        mma_f16(o[nn], pah[2], pal[2], pah[3], pal[3], nib_pair_c(wv, 2), nib_pair_c(wv, 3));
+      }
+    }
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+  flush(cur);
+}
+
+// ------------------------------------------------------------------ merge
+// Partials of one launch: one (max, sum, unnormalised o) per (pair, warp segment, head).
+struct PartialSet {
+  const float* o;
+  const float* ml;
+  int upp;          // units per pair
+  int64_t T;        // pairs * upp
+  int W, maxseg;
+};
+
+// Fixed-order merge of up to two partial sets for one head: block (pair, head), D threads.
 template <int D, typename OutT>
-__global__ void __launch_bounds__(D) draft_combine_kernel(const DraftIndexedParams p,
+__global__ void __launch_bounds__(D) draft_combine_kernel(PartialSet a, PartialSet b, int nsets,
+                                                          int g, int Hkv, int Hq,
                                                           OutT* __restrict__ out,
                                                           float* __restrict__ lse) {
-  const int64_t pair = blockIdx.x / p.g;
-  const int r = blockIdx.x - (int)(pair * p.g);
+  const int64_t pair = blockIdx.x / g;
+  const int r = blockIdx.x - (int)(pair * g);
   const int d = threadIdx.x;
-  const int64_t w0 = warp_of_tile(pair * p.tpp, p.T, p.W);
-  const int64_t w1 = warp_of_tile((pair + 1) * p.tpp - 1, p.T, p.W);
   float M = -INFINITY, L = 0.f, O = 0.f;
+  for (int si = 0; si < nsets; ++si) {
+    const PartialSet& ps = si == 0 ? a : b;
+    const int64_t w0 = warp_of_tile(pair * ps.upp, ps.T, ps.W);
+    const int64_t w1 = warp_of_tile((pair + 1) * ps.upp - 1, ps.T, ps.W);
 #pragma unroll 4
-  for (int64_t w = w0; w <= w1; ++w) {
-    if (warp_begin(w, p.T, p.W) >= warp_begin(w + 1, p.T, p.W)) continue;   // empty range
-    const int64_t pr = (pair * p.maxseg + (w - w0)) * p.g + r;
-    const float2 ml = *reinterpret_cast<const float2*>(p.ws_ml + pr * 2);
-    const float os = p.ws_o[pr * D + d];
-    const float Mn = fmaxf(M, ml.x);
-    const float a = ex2(M - Mn), c = ex2(ml.x - Mn);
-    L = fmaf(L, a, ml.y * c);
-    O = fmaf(O, a, os * c);
-    M = Mn;
+    for (int64_t w = w0; w <= w1; ++w) {
+      if (warp_begin(w, ps.T, ps.W) >= warp_begin(w + 1, ps.T, ps.W)) continue;   // empty
+      const int64_t pr = (pair * ps.maxseg + (w - w0)) * g + r;
+      const float2 ml = *reinterpret_cast<const float2*>(ps.ml + pr * 2);
+      const float os = ps.o[pr * D + d];
+      const float Mn = fmaxf(M, ml.x);
+      const float fa = ex2(M - Mn), fc = ex2(ml.x - Mn);
+      L = fmaf(L, fa, ml.y * fc);
+      O = fmaf(O, fa, os * fc);
+      M = Mn;
+    }
   }
-  const int64_t b = pair / p.Hkv, j = pair - b * p.Hkv;
-  const int64_t h = b * p.Hq + j * p.g + r;
+  const int64_t bb = pair / Hkv, j = pair - bb * Hkv;
+  const int64_t h = bb * Hq + j * g + r;
   store_out(out + h * D + d, O / L);
   if (lse && d == 0) lse[h] = (M + __log2f(L)) * kLn2;
 }
@@ -351,67 +665,74 @@ __global__ void __launch_bounds__(D) draft_combine_kernel(const DraftIndexedPara
 // ------------------------------------------------------------------ host side
 namespace {
 constexpr int kNStage = 3;
+constexpr int kNStageInt4 = 4;
 
 struct DraftPlan {
-  int tpp, W, maxseg;
+  int upp, W, maxseg;
   int64_t T;
+  size_t floats(int pairs, int g, int D) const {
+    return (size_t)pairs * maxseg * g * ((size_t)D + 2);
+  }
 };
 
-DraftPlan draft_plan(int pairs, int total) {
+// Equal contiguous warp ranges over pairs x upp units (upp units per pair).
+DraftPlan draft_plan(int pairs, int upp) {
   DraftPlan pl;
-  pl.tpp = (total + kTile - 1) / kTile;
-  pl.T = (int64_t)pairs * pl.tpp;
+  pl.upp = upp;
+  pl.T = (int64_t)pairs * upp;
   const int64_t ctas = std::min<int64_t>(2 * (int64_t)num_sms(),
                                          std::max<int64_t>(1, pl.T / kDraftWarps));
   pl.W = (int)(ctas * kDraftWarps);
   int ms = 1;
   for (int64_t pr = 0; pr < pairs; ++pr) {
-    const int64_t a = warp_of_tile(pr * pl.tpp, pl.T, pl.W);
-    const int64_t b = warp_of_tile((pr + 1) * pl.tpp - 1, pl.T, pl.W);
+    const int64_t a = warp_of_tile(pr * upp, pl.T, pl.W);
+    const int64_t b = warp_of_tile((pr + 1) * upp - 1, pl.T, pl.W);
     ms = std::max<int>(ms, (int)(b - a + 1));
   }
   pl.maxseg = ms;
   return pl;
 }
 
+int tiles_of(int slots) { return (slots + kTile - 1) / kTile; }
+
 template <int D>
 size_t draft_indexed_smem() {
   return (size_t)kDraftWarps * (kNStage * DraftSmem<D>::kStageB + DraftSmem<D>::kTableB);
 }
-}  // namespace
+template <int D>
+size_t draft_int4_smem() {
+  return (size_t)kDraftWarps * kNStageInt4 * Int4Smem<D>::kStageB;
+}
 
-size_t draft_workspace_bytes(const vc_comp_cache* c) {
-  const int pairs = c->B * c->Hkv;
-  const int total = c->S + c->n_tail;
-  const DraftPlan pl = draft_plan(pairs, total > 0 ? total : 1);
-  const int g = c->Hq / c->Hkv;
-  return (size_t)pairs * pl.maxseg * g * ((size_t)c->D + 2) * sizeof(float) + 256;
+PartialSet partials(const DraftPlan& pl, float* base, int pairs, int g, int D) {
+  PartialSet ps;
+  ps.o = base;
+  ps.ml = base + (size_t)pairs * pl.maxseg * g * D;
+  ps.upp = pl.upp;
+  ps.T = pl.T;
+  ps.W = pl.W;
+  ps.maxseg = pl.maxseg;
+  return ps;
 }
 
 template <int D>
-static vc_status launch_draft_d(const DraftIndexedParams& p, int flags, void* out, float* lse,
-                                cudaStream_t stream) {
-  const size_t sm = draft_indexed_smem<D>();
-  VC_CUDA(cudaFuncSetAttribute(draft_indexed_kernel<D, kNStage>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-  draft_indexed_kernel<D, kNStage><<<p.W / kDraftWarps, 128, sm, stream>>>(p);
-  VC_CUDA(cudaGetLastError());
-  const int blocks = (int)(p.T / p.tpp) * p.g;   // one per (pair, head)
+vc_status launch_combine(const PartialSet& a, const PartialSet& b, int nsets, int pairs, int g,
+                         int Hkv, int Hq, int flags, void* out, float* lse, cudaStream_t stream) {
+  const int blocks = pairs * g;
   if (flags & VC_OUT_F32)
-    draft_combine_kernel<D, float><<<blocks, D, 0, stream>>>(p, static_cast<float*>(out), lse);
+    draft_combine_kernel<D, float><<<blocks, D, 0, stream>>>(a, b, nsets, g, Hkv, Hq,
+                                                             static_cast<float*>(out), lse);
   else
     draft_combine_kernel<D, __nv_bfloat16><<<blocks, D, 0, stream>>>(
-        p, static_cast<__nv_bfloat16*>(out), lse);
+        a, b, nsets, g, Hkv, Hq, static_cast<__nv_bfloat16*>(out), lse);
   VC_CUDA(cudaGetLastError());
   return VC_OK;
 }
 
-vc_status launch_draft_indexed(const void* q, const vc_comp_cache* c, float scale, int flags,
-                               void* out, float* lse, void* ws, size_t ws_bytes,
-                               cudaStream_t stream) {
+// Indexed-kernel parameters for the slots [0, S) and tail rows [0, n_tail) of a cache.
+DraftIndexedParams indexed_params(const void* q, const vc_comp_cache* c, int S, int n_tail,
+                                  float scale, const DraftPlan& pl, float* ws) {
   const int pairs = c->B * c->Hkv;
-  const int total = c->S + c->n_tail;
-  const DraftPlan pl = draft_plan(pairs, total);
   DraftIndexedParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k = static_cast<const __nv_bfloat16*>(c->k);
@@ -421,34 +742,138 @@ vc_status launch_draft_indexed(const void* q, const vc_comp_cache* c, float scal
   p.k_tail = static_cast<const __nv_bfloat16*>(c->k_tail);
   p.v_tail = static_cast<const __nv_bfloat16*>(c->v_tail);
   p.T_cap = c->T_cap;
-  p.S = c->S;
+  p.S = S;
   p.S_cap = c->S_cap;
   p.R_cap = c->R_cap;
-  p.n_tail = c->n_tail;
+  p.n_tail = n_tail;
   p.Hq = c->Hq;
   p.Hkv = c->Hkv;
   p.g = c->Hq / c->Hkv;
-  p.tpp = pl.tpp;
+  p.tpp = pl.upp;
   p.T = pl.T;
   p.W = pl.W;
   p.maxseg = pl.maxseg;
   p.qk_scale2 = scale * kLog2e;
-  const size_t ws_need = (size_t)pairs * pl.maxseg * p.g * ((size_t)c->D + 2) * sizeof(float);
-  if (ws_bytes < ws_need) return fail(VC_ERR_INVALID, "draft workspace too small");
-  p.ws_o = static_cast<float*>(ws);
-  p.ws_ml = p.ws_o + (size_t)pairs * pl.maxseg * p.g * c->D;
+  p.ws_o = ws;
+  p.ws_ml = ws + (size_t)pairs * pl.maxseg * p.g * c->D;
   p.err_flag = c->err_flag;
-  if (c->D == 128) return launch_draft_d<128>(p, flags, out, lse, stream);
-  return launch_draft_d<64>(p, flags, out, lse, stream);
+  return p;
 }
 
-}  // namespace vc
-
-namespace vc {
-vc_status launch_draft_int4(const void*, const vc_comp_cache*, float, int, void*, float*, void*,
-                            size_t, cudaStream_t) {
-  return fail(VC_ERR_UNSUPPORTED, "int4 draft attention not built yet");
+template <int D>
+vc_status run_indexed(const DraftIndexedParams& p, cudaStream_t stream) {
+  const size_t sm = draft_indexed_smem<D>();
+  VC_CUDA(cudaFuncSetAttribute(draft_indexed_kernel<D, kNStage>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+  draft_indexed_kernel<D, kNStage><<<p.W / kDraftWarps, 128, sm, stream>>>(p);
+  VC_CUDA(cudaGetLastError());
+  return VC_OK;
 }
+
+template <int D>
+vc_status run_int4(const DraftInt4Params& p, cudaStream_t stream) {
+  const size_t sm = draft_int4_smem<D>();
+  VC_CUDA(cudaFuncSetAttribute(draft_int4_kernel<D, kNStageInt4>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+  draft_int4_kernel<D, kNStageInt4><<<p.W / kDraftWarps, 128, sm, stream>>>(p);
+  VC_CUDA(cudaGetLastError());
+  return VC_OK;
+}
+
+// Workspace split of an int4 call: partials of the quantised blocks, then of the tail.
+struct Int4Plans {
+  DraftPlan q, t;
+  bool has_q, has_t;
+  size_t floats_q, floats_t;
+};
+Int4Plans int4_plans(const vc_comp_cache* c) {
+  const int pairs = c->B * c->Hkv, g = c->Hq / c->Hkv;
+  Int4Plans ip;
+  ip.has_q = c->S > 0;
+  ip.has_t = c->n_tail > 0;
+  ip.q = draft_plan(pairs, ip.has_q ? c->S / 32 : 1);
+  ip.t = draft_plan(pairs, ip.has_t ? tiles_of(c->n_tail) : 1);
+  ip.floats_q = ip.has_q ? ip.q.floats(pairs, g, c->D) : 0;
+  ip.floats_t = ip.has_t ? ip.t.floats(pairs, g, c->D) : 0;
+  return ip;
+}
+}  // namespace
+
+size_t draft_workspace_bytes(const vc_comp_cache* c) {
+  const int pairs = c->B * c->Hkv, g = c->Hq / c->Hkv;
+  if (c->kind == VC_CACHE_INT4) {
+    const Int4Plans ip = int4_plans(c);
+    return (ip.floats_q + ip.floats_t) * sizeof(float) + 256;
+  }
+  const int total = c->S + c->n_tail;
+  const DraftPlan pl = draft_plan(pairs, tiles_of(total > 0 ? total : 1));
+  return pl.floats(pairs, g, c->D) * sizeof(float) + 256;
+}
+
+vc_status launch_draft_indexed(const void* q, const vc_comp_cache* c, float scale, int flags,
+                               void* out, float* lse, void* ws, size_t ws_bytes,
+                               cudaStream_t stream) {
+  const int pairs = c->B * c->Hkv, g = c->Hq / c->Hkv;
+  const DraftPlan pl = draft_plan(pairs, tiles_of(c->S + c->n_tail));
+  if (ws_bytes < pl.floats(pairs, g, c->D) * sizeof(float))
+    return fail(VC_ERR_INVALID, "draft workspace too small");
+  float* w = static_cast<float*>(ws);
+  const DraftIndexedParams p = indexed_params(q, c, c->S, c->n_tail, scale, pl, w);
+  const PartialSet ps = partials(pl, w, pairs, g, c->D);
+  vc_status st = c->D == 128 ? run_indexed<128>(p, stream) : run_indexed<64>(p, stream);
+  if (st != VC_OK) return st;
+  return c->D == 128 ? launch_combine<128>(ps, ps, 1, pairs, g, c->Hkv, c->Hq, flags, out, lse, stream)
+                     : launch_combine<64>(ps, ps, 1, pairs, g, c->Hkv, c->Hq, flags, out, lse, stream);
+}
+
+vc_status launch_draft_int4(const void* q, const vc_comp_cache* c, float scale, int flags,
+                            void* out, float* lse, void* ws, size_t ws_bytes,
+                            cudaStream_t stream) {
+  const int pairs = c->B * c->Hkv, g = c->Hq / c->Hkv;
+  const Int4Plans ip = int4_plans(c);
+  if (ws_bytes < (ip.floats_q + ip.floats_t) * sizeof(float))
+    return fail(VC_ERR_INVALID, "draft workspace too small");
+  float* wq = static_cast<float*>(ws);
+  float* wt = wq + ip.floats_q;
+  PartialSet sets[2];
+  int nsets = 0;
+  if (ip.has_q) {
+    DraftInt4Params p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.kq = c->kq;
+    p.ks = static_cast<const __half*>(c->k_scale);
+    p.kz = static_cast<const __half*>(c->k_zero);
+    p.vq = c->vq;
+    p.vs = static_cast<const __half*>(c->v_scale);
+    p.vz = static_cast<const __half*>(c->v_zero);
+    p.nblk_cap = c->T_cap / 32;
+    p.nblk = c->S / 32;
+    p.Hq = c->Hq;
+    p.Hkv = c->Hkv;
+    p.g = g;
+    p.T = ip.q.T;
+    p.W = ip.q.W;
+    p.maxseg = ip.q.maxseg;
+    p.qk_scale2 = scale * kLog2e;
+    p.ws_o = wq;
+    p.ws_ml = wq + (size_t)pairs * ip.q.maxseg * g * c->D;
+    vc_status st = c->D == 128 ? run_int4<128>(p, stream) : run_int4<64>(p, stream);
+    if (st != VC_OK) return st;
+    sets[nsets++] = partials(ip.q, wq, pairs, g, c->D);
+  }
+  if (ip.has_t) {   // the bf16 tail rows through the indexed kernel (no slots)
+    const DraftIndexedParams p = indexed_params(q, c, 0, c->n_tail, scale, ip.t, wt);
+    vc_status st = c->D == 128 ? run_indexed<128>(p, stream) : run_indexed<64>(p, stream);
+    if (st != VC_OK) return st;
+    sets[nsets++] = partials(ip.t, wt, pairs, g, c->D);
+  }
+  return c->D == 128
+             ? launch_combine<128>(sets[0], sets[nsets - 1], nsets, pairs, g, c->Hkv, c->Hq, flags,
+                                   out, lse, stream)
+             : launch_combine<64>(sets[0], sets[nsets - 1], nsets, pairs, g, c->Hkv, c->Hq, flags,
+                                  out, lse, stream);
+}
+
 }  // namespace vc
 
 // ------------------------------------------------------------------ fixed-scratch variant
