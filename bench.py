@@ -414,6 +414,108 @@ def e2e_measure(rnd, steps: int, warmup: int, device) -> dict:
             "ms_per_step": tot / steps * 1e3}
 
 
+# ------------------------------------------------------------------ workload 4
+def run_config4(args) -> int:
+    """Long-context staging: one request's 1M-token full cache (4 GiB, chunk-major in
+    pinned host memory) streams through a 3-slot HBM ring for its k = 40 verify while
+    three 256K-context requests draft over their 65536-slot compressed caches."""
+    import torch
+    import lossless_kv_compressed_b200 as vc
+    from lossless_kv_compressed_b200.stagger import StagedVerify, run_alongside
+    from synth import gen
+    from synth.configs import get_config
+    cfg = get_config(4)
+    dev = torch.device("cuda", 0)
+    chunk = cfg.chunk_tokens
+    n_chunks = cfg.P // chunk
+    case = gen.staged_case(cfg)
+    host = torch.empty((n_chunks, 2, cfg.Hkv, chunk, cfg.D), dtype=torch.bfloat16,
+                       pin_memory=True)
+    b16 = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
+        torch.bfloat16)
+    for c, (kb, vb) in enumerate(zip(case["chunks_k"], case["chunks_v"])):
+        host[c, 0] = b16(kb)
+        host[c, 1] = b16(vb)
+    bk, bv = b16(case["block_k_bits"]).to(dev), b16(case["block_v_bits"]).to(dev)
+    q = b16(case["q_verify_bits"]).to(dev)
+    st = StagedVerify(host, cfg.P, bk, bv, n_slots=3)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    # drafting requests: 3 x 8 kv heads x 65536 compact slots, degrees 1..16
+    r = gen.children(cfg.seed + 200, 4)
+    S = cfg.S
+    kc = b16(gen.f32_to_bf16_bits(gen.ar1(r[0], (cfg.n_draft_requests, cfg.Hkv), S, cfg.D,
+                                          cfg.rho))).to(dev)
+    vcc = b16(gen.f32_to_bf16_bits(gen.ar1(r[1], (cfg.n_draft_requests, cfg.Hkv), S, cfg.D,
+                                           cfg.rho))).to(dev)
+    deg = torch.from_numpy(gen.slot_degrees(r[2], (cfg.n_draft_requests, cfg.Hkv), S,
+                                            cfg.n_sinks, cfg.n_recent, cfg.deg_max)).to(dev)
+    dq = b16(gen.f32_to_bf16_bits(gen.normal(r[3], (cfg.n_draft_requests, cfg.Hq,
+                                                    cfg.D)))).to(dev)
+    dcache = vc.IndexedCache(k=kc, v=vcc, S=S, Hq=cfg.Hq, deg=deg)
+    dws = torch.empty(vc.draft_workspace_size(dcache), dtype=torch.uint8, device=dev)
+    dout = torch.empty_like(dq)
+    s_draft = torch.cuda.Stream(dev)
+    d_bytes = cfg.n_draft_requests * cfg.Hkv * S * (cfg.D * 4 + 4) + 2 * dq.numel() * 2
+
+    def draft_step(stream):
+        vc.draft_attn(dq, dcache, out=dout, ws=dws, stream=stream)
+
+    full_bytes = n_chunks * st.chunk_bytes
+    # (1) bare PCIe: the 16 chunk copies alone, back to back
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for rep in range(2):
+        ev0.record(st.s_copy)
+        for c in range(n_chunks):
+            vc.stage_full_kv(st.ring[c % 3], host[c], st.chunk_bytes, st.s_copy)
+        ev1.record(st.s_copy)
+        ev1.synchronize()
+    bare_gbs = full_bytes / (ev0.elapsed_time(ev1) * 1e-3) / 1e9
+    # (2) drafts alone
+    for _ in range(5):
+        draft_step(s_draft)
+    s_draft.synchronize()
+    ev0.record(s_draft)
+    n_alone = 50
+    for _ in range(n_alone):
+        draft_step(s_draft)
+    ev1.record(s_draft)
+    ev1.synchronize()
+    draft_alone_s = ev0.elapsed_time(ev1) * 1e-3 / n_alone
+    # (3) staged verify alone, then (4) alongside drafting; warm once each
+    st.launch(q, out)
+    torch.cuda.synchronize()
+    st.launch(q, out)
+    torch.cuda.synchronize()
+    verify_alone_ms = st.t_start.elapsed_time(st.t_done)
+    staged_alone_gbs = full_bytes / (st.t_start.elapsed_time(st.t_staged) * 1e-3) / 1e9
+    ev0.record(s_draft)
+    n_drafts = run_alongside(st, q, out, draft_step, s_draft)
+    ev1.record(s_draft)
+    torch.cuda.synchronize()
+    round_ms = st.t_start.elapsed_time(st.t_done)
+    staged_gbs = full_bytes / (st.t_start.elapsed_time(st.t_staged) * 1e-3) / 1e9
+    draft_span_s = ev0.elapsed_time(ev1) * 1e-3
+    assert vc.device_error() == 0
+    line = {
+        "metric": METRIC, "value": staged_gbs, "unit": "GB/s", "n_gpus": 1,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic", "scaling": "weak",
+        "vs_baseline": None,
+        "config": {"workload": cfg.name, "context": cfg.P, "heads": f"{cfg.Hq}/{cfg.Hkv}",
+                   "head_dim": cfg.D, "verify_rows": cfg.k + 1, "chunk_tokens": chunk,
+                   "ring_slots": 3, "draft_requests": cfg.n_draft_requests,
+                   "draft_slots": S},
+        "pcie": {"bare_h2d_GBs": bare_gbs, "staged_alone_GBs": staged_alone_gbs,
+                 "staged_while_drafting_GBs": staged_gbs, "frac_of_bare": staged_gbs / bare_gbs,
+                 "bytes_per_round": full_bytes},
+        "verify_round_ms": {"alone": verify_alone_ms, "while_drafting": round_ms},
+        "draft": {"alone_us": draft_alone_s * 1e6, "alone_GBs": d_bytes / draft_alone_s / 1e9,
+                  "steps_during_round": n_drafts,
+                  "overlapped_GBs": n_drafts * d_bytes / draft_span_s / 1e9},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -421,9 +523,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="vc", choices=["vc", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--config", type=int, default=2, choices=[2, 4],
+                    help="2: the round of the 32K-context layer (default line); "
+                         "4: long-context staging while drafting")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.config == 4 and args.impl == "vc":
+        return run_config4(args)
     world, rank, local = dist_setup()
     if args.impl == "reference":
         code = run_reference(args, world, rank)

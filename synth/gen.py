@@ -198,3 +198,43 @@ def tinylm_prompt(cfg) -> np.ndarray:
     """Prompt of uniform-random token ids."""
     r = children(cfg.seed + 500, 1)[0]
     return r.integers(0, cfg.vocab, size=cfg.prompt_len, dtype=np.int64)
+
+
+def ar1_chunks(rng: Generator, lead: tuple, L: int, D: int, rho: float, chunk: int):
+    """AR(1) along the sequence in pieces of ``chunk`` rows (bf16 bits [*lead, n, D]),
+    the filter state carried across pieces, so long sequences never sit in fp32 whole.
+    Same process as ``ar1``."""
+    b0 = math.sqrt(1.0 - rho * rho)
+    state = None
+    for s0 in range(0, L, chunk):
+        n = min(chunk, L - s0)
+        e = rng.standard_normal((*lead, n, D), dtype=np.float32)
+        if rho == 0.0:
+            yield f32_to_bf16_bits(e)
+            continue
+        if state is None:
+            e[..., 0, :] /= b0
+            x = lfilter([b0], [1.0, -rho], e, axis=-2)
+        else:
+            x, _ = lfilter([b0], [1.0, -rho], e, axis=-2,
+                           zi=(rho * state)[..., None, :])
+        state = x[..., -1, :].astype(np.float64)
+        yield f32_to_bf16_bits(x.astype(np.float32))
+
+
+def staged_case(cfg=None, chunk: int | None = None, P: int | None = None):
+    """Workload-4 inputs: the full cache of one request as chunk-major bf16 bits
+    (generator of [2 (K|V), Hkv, chunk, D] pieces), its verify queries and block K/V,
+    and the compact compressed caches of the drafting requests."""
+    cfg = cfg or get_config(4)
+    chunk = chunk or cfg.chunk_tokens
+    P = P or cfg.P
+    r = children(cfg.seed + 100, 8)
+    out = {"cfg": cfg, "chunk": chunk, "P": P}
+    out["chunks_k"] = ar1_chunks(r[0], (cfg.Hkv,), P, cfg.D, cfg.rho, chunk)
+    out["chunks_v"] = ar1_chunks(r[1], (cfg.Hkv,), P, cfg.D, cfg.rho, chunk)
+    n_q = cfg.k + 1
+    out["block_k_bits"] = f32_to_bf16_bits(normal(r[2], (1, cfg.Hkv, n_q, cfg.D)))
+    out["block_v_bits"] = f32_to_bf16_bits(normal(r[3], (1, cfg.Hkv, n_q, cfg.D)))
+    out["q_verify_bits"] = f32_to_bf16_bits(normal(r[4], (1, n_q, cfg.Hq, cfg.D)))
+    return out
