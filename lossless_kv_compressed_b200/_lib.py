@@ -23,6 +23,11 @@ EXPORTS = (
     "vc_verify_workspace_size", "vc_verify_attn",
     "vc_accept", "vc_stage_full_kv", "vc_event_wait", "vc_device_error",
 )
+# Model glue of the end-to-end loop (include/vericache_glue.h).
+GLUE_EXPORTS = (
+    "vc_glue_embed", "vc_glue_rmsnorm", "vc_glue_gemm", "vc_glue_rope_store",
+    "vc_glue_swiglu", "vc_glue_append_slots",
+)
 
 _p = ctypes.c_void_p
 _i32 = ctypes.c_int32
@@ -88,6 +93,17 @@ def lib() -> ctypes.CDLL:
         L.vc_event_wait.argtypes = [_p, ctypes.c_double]
         L.vc_device_error.restype = ctypes.c_int
         L.vc_device_error.argtypes = [ctypes.POINTER(_i32), ctypes.c_int]
+        for name in GLUE_EXPORTS:
+            getattr(L, name).restype = ctypes.c_int
+        L.vc_glue_embed.argtypes = [_p, _p, ctypes.c_int, ctypes.c_int, _p, _p]
+        L.vc_glue_rmsnorm.argtypes = [_p, ctypes.c_int, ctypes.c_int, ctypes.c_float, _p, _p]
+        L.vc_glue_gemm.argtypes = [_p, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _p,
+                                   ctypes.c_int, _p]
+        L.vc_glue_rope_store.argtypes = [_p, _p, _p] + [ctypes.c_int] * 4 + [ctypes.c_float,
+                                                                             _p, _p, _p,
+                                                                             ctypes.c_int, _p]
+        L.vc_glue_swiglu.argtypes = [_p, ctypes.c_int, ctypes.c_int, _p, _p]
+        L.vc_glue_append_slots.argtypes = [_p, _p] + [ctypes.c_int] * 5 + [_p]
         _lib = L
     return _lib
 

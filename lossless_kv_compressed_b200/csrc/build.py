@@ -43,7 +43,7 @@ def _newer(src_paths, out) -> bool:
 def build(verbose: bool = False, ptxas_v: bool = False, force: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     headers = [os.path.join(HERE, f) for f in os.listdir(HERE) if f.endswith((".cuh", ".h"))]
-    headers.append(os.path.join(INCLUDE, "vericache.h"))
+    headers += [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
     jobs = []
     for s in sources():
         o = os.path.join(BUILD, os.path.basename(s)[:-3] + ".o")

@@ -1,0 +1,227 @@
+// Model glue for the end-to-end draft-then-verify loop (see vericache_glue.h).
+// Every kernel computes a row with the same instructions in the same order whatever the
+// number of rows, so a block of k+1 tokens and k+1 single tokens agree bit for bit.
+#include <math.h>
+
+#include "vc_common.cuh"
+#include "vc_internal.h"
+#include "vericache_glue.h"
+
+namespace vc {
+namespace {
+
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+__global__ void embed_kernel(const __nv_bfloat16* __restrict__ table, const int32_t* __restrict__ ids,
+                             int n, int d, float* __restrict__ x) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)n * d) return;
+  const int r = (int)(i / d), c = (int)(i - (int64_t)r * d);
+  x[i] = __bfloat162float(table[(int64_t)ids[r] * d + c]);
+}
+
+// one warp per row; lane-strided squares summed in a fixed order, butterfly reduction
+__global__ void rmsnorm_kernel(const float* __restrict__ x, int n, int d, float eps,
+                               __nv_bfloat16* __restrict__ out) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= n) return;
+  const float* xr = x + (int64_t)row * d;
+  float ss = 0.f;
+  for (int j = lane; j < d; j += 32) ss = fmaf(xr[j], xr[j], ss);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+  for (int j = lane; j < d; j += 32) out[(int64_t)row * d + j] = __float2bfloat16_rn(xr[j] * inv);
+}
+
+// c[16 x 64 tile] (+)= a[16 x K] @ w[K x 64]: 4 warps x (16 rows x 16 cols), k-steps of 16
+// in order; the w tile rows stream through a 3-stage cp.async ring (128-byte rows,
+// XOR-swizzled) and enter the mma as transposed ldmatrix fragments.
+constexpr int kGemmNst = 3;
+__global__ void __launch_bounds__(128) gemm_kernel(const __nv_bfloat16* __restrict__ a,
+                                                   const __nv_bfloat16* __restrict__ w, int M,
+                                                   int K, int N, float* __restrict__ c,
+                                                   int accumulate) {
+  __shared__ __align__(128) uint8_t sw[kGemmNst][16 * 128];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qr = lane >> 2, qc = lane & 3;
+  const int n0 = blockIdx.x * 64, m0 = blockIdx.y * 16;
+  const int ksteps = K / 16;
+  auto issue = [&](int ks, int st) {
+    const int row = threadIdx.x >> 3, ch = threadIdx.x & 7;
+    const __nv_bfloat16* src = w + (int64_t)(ks * 16 + row) * N + n0 + ch * 8;
+    cp_async16(smem_u32(&sw[st][row * 128 + ((ch ^ (row & 7)) << 4)]), src, 16u);
+  };
+  const bool r0 = m0 + qr < M, r1 = m0 + qr + 8 < M;
+  const uint32_t* a0p = reinterpret_cast<const uint32_t*>(a + (int64_t)(r0 ? m0 + qr : 0) * K);
+  const uint32_t* a1p = reinterpret_cast<const uint32_t*>(a + (int64_t)(r1 ? m0 + qr + 8 : 0) * K);
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+  for (int st = 0; st < kGemmNst - 1; ++st) {
+    if (st < ksteps) issue(st, st);
+    cp_async_commit();
+  }
+  for (int ks = 0; ks < ksteps; ++ks) {
+    if (ks + kGemmNst - 1 < ksteps) issue(ks + kGemmNst - 1, (ks + kGemmNst - 1) % kGemmNst);
+    cp_async_commit();
+    cp_async_wait<kGemmNst - 1>();
+    __syncthreads();
+    const int k0 = ks * 16;
+    const uint32_t A0 = r0 ? __ldg(a0p + (k0 + 2 * qc) / 2) : 0u;
+    const uint32_t A1 = r1 ? __ldg(a1p + (k0 + 2 * qc) / 2) : 0u;
+    const uint32_t A2 = r0 ? __ldg(a0p + (k0 + 8 + 2 * qc) / 2) : 0u;
+    const uint32_t A3 = r1 ? __ldg(a1p + (k0 + 8 + 2 * qc) / 2) : 0u;
+    const int mi = lane >> 3;
+    const int krow = (mi & 1) * 8 + (lane & 7);
+    const int ch = warp * 2 + (mi >> 1);
+    uint32_t b0, b1, b2, b3;
+    ldsm_x4_t(smem_u32(&sw[ks % kGemmNst][krow * 128 + ((ch ^ (krow & 7)) << 4)]), b0, b1, b2, b3);
+    mma_bf16(acc[0], A0, A1, A2, A3, b0, b1);
+    mma_bf16(acc[1], A0, A1, A2, A3, b2, b3);
+    __syncthreads();
+  }
+  cp_async_wait<0>();
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    const int col = n0 + warp * 16 + nt * 8 + 2 * qc;
+    if (r0) {
+      float* p = c + (int64_t)(m0 + qr) * N + col;
+      p[0] = accumulate ? p[0] + acc[nt][0] : acc[nt][0];
+      p[1] = accumulate ? p[1] + acc[nt][1] : acc[nt][1];
+    }
+    if (r1) {
+      float* p = c + (int64_t)(m0 + qr + 8) * N + col;
+      p[0] = accumulate ? p[0] + acc[nt][2] : acc[nt][2];
+      p[1] = accumulate ? p[1] + acc[nt][3] : acc[nt][3];
+    }
+  }
+}
+
+// one thread per (row, head, i < D/2): rotate-half RoPE in double precision angles
+__global__ void rope_store_kernel(const float* __restrict__ qkv, const int32_t* __restrict__ pos,
+                                  const int32_t* __restrict__ dst_row, int n, int Hq, int Hkv,
+                                  int D, float theta, __nv_bfloat16* __restrict__ q_out,
+                                  __nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc_,
+                                  int cap) {
+  const int half = D / 2;
+  const int heads = Hq + 2 * Hkv;
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= (int64_t)n * heads * half) return;
+  const int row = (int)(t / ((int64_t)heads * half));
+  const int rem = (int)(t - (int64_t)row * heads * half);
+  const int h = rem / half, i = rem - h * half;
+  const float* src = qkv + (int64_t)row * heads * D + (int64_t)h * D;
+  const float x1 = src[i], x2 = src[i + half];
+  if (h < Hq + Hkv) {
+    const double inv = pow((double)theta, -2.0 * i / (double)D);
+    double s, co;
+    sincos((double)pos[row] * inv, &s, &co);
+    const float y1 = (float)(x1 * co - x2 * s), y2 = (float)(x2 * co + x1 * s);
+    if (h < Hq) {
+      __nv_bfloat16* qo = q_out + ((int64_t)row * Hq + h) * D;
+      qo[i] = __float2bfloat16_rn(y1);
+      qo[i + half] = __float2bfloat16_rn(y2);
+    } else if (dst_row[row] >= 0) {
+      __nv_bfloat16* ko = kc + ((int64_t)(h - Hq) * cap + dst_row[row]) * D;
+      ko[i] = __float2bfloat16_rn(y1);
+      ko[i + half] = __float2bfloat16_rn(y2);
+    }
+  } else if (dst_row[row] >= 0) {
+    __nv_bfloat16* vo = vc_ + ((int64_t)(h - Hq - Hkv) * cap + dst_row[row]) * D;
+    vo[i] = __float2bfloat16_rn(x1);
+    vo[i + half] = __float2bfloat16_rn(x2);
+  }
+}
+
+__global__ void swiglu_kernel(const float* __restrict__ gu, int n, int F,
+                              __nv_bfloat16* __restrict__ out) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)n * F) return;
+  const int r = (int)(i / F), j = (int)(i - (int64_t)r * F);
+  const float g = gu[(int64_t)r * 2 * F + j], u = gu[(int64_t)r * 2 * F + F + j];
+  out[i] = __float2bfloat16_rn(g / (1.0f + expf(-g)) * u);
+}
+
+__global__ void append_slots_kernel(int32_t* idx, int32_t* deg, int Hkv, int S_cap, int S,
+                                    int start, int count) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= Hkv * count) return;
+  const int h = t / count, i = t - h * count;
+  idx[(int64_t)h * S_cap + S + i] = start + i;
+  if (deg) deg[(int64_t)h * S_cap + S + i] = 1;
+}
+
+int blocks_for(int64_t n, int t) { return (int)((n + t - 1) / t); }
+
+}  // namespace
+}  // namespace vc
+
+using namespace vc;
+
+extern "C" {
+
+vc_status vc_glue_embed(const void* table, const int32_t* ids, int n, int d, float* x,
+                        cudaStream_t stream) {
+  if (!table || !ids || !x || n <= 0 || d <= 0) return fail(VC_ERR_INVALID, "embed: args");
+  embed_kernel<<<blocks_for((int64_t)n * d, 256), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(table), ids, n, d, x);
+  VC_CUDA(cudaGetLastError());
+  return VC_OK;
+}
+
+vc_status vc_glue_rmsnorm(const float* x, int n, int d, float eps, void* out,
+                          cudaStream_t stream) {
+  if (!x || !out || n <= 0 || d <= 0) return fail(VC_ERR_INVALID, "rmsnorm: args");
+  rmsnorm_kernel<<<blocks_for(n, 4), 128, 0, stream>>>(x, n, d, eps,
+                                                       static_cast<__nv_bfloat16*>(out));
+  VC_CUDA(cudaGetLastError());
+  return VC_OK;
+}
+
+vc_status vc_glue_gemm(const void* a, const void* w, int M, int K, int N, float* c,
+                       int accumulate, cudaStream_t stream) {
+  if (!a || !w || !c || M <= 0 || K <= 0 || N <= 0) return fail(VC_ERR_INVALID, "gemm: args");
+  if (K % 16 || N % 64) return fail(VC_ERR_UNSUPPORTED, "gemm: K %% 16 and N %% 64 must be 0");
+  if (!al16(a) || !al16(w)) return fail(VC_ERR_INVALID, "gemm: misaligned");
+  dim3 grid(N / 64, (M + 15) / 16);
+  gemm_kernel<<<grid, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(a),
+                                        static_cast<const __nv_bfloat16*>(w), M, K, N, c,
+                                        accumulate);
+  VC_CUDA(cudaGetLastError());
+  return VC_OK;
+}
+
+vc_status vc_glue_rope_store(const float* qkv, const int32_t* pos, const int32_t* dst_row,
+                             int n, int Hq, int Hkv, int D, float theta, void* q_out,
+                             void* k_cache, void* v_cache, int cap, cudaStream_t stream) {
+  if (!qkv || !pos || !dst_row || !q_out || !k_cache || !v_cache || n <= 0 || D % 2)
+    return fail(VC_ERR_INVALID, "rope_store: args");
+  const int64_t total = (int64_t)n * (Hq + 2 * Hkv) * (D / 2);
+  rope_store_kernel<<<blocks_for(total, 256), 256, 0, stream>>>(
+      qkv, pos, dst_row, n, Hq, Hkv, D, theta, static_cast<__nv_bfloat16*>(q_out),
+      static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), cap);
+  VC_CUDA(cudaGetLastError());
+  return VC_OK;
+}
+
+vc_status vc_glue_swiglu(const float* gu, int n, int F, void* out, cudaStream_t stream) {
+  if (!gu || !out || n <= 0 || F <= 0) return fail(VC_ERR_INVALID, "swiglu: args");
+  swiglu_kernel<<<blocks_for((int64_t)n * F, 256), 256, 0, stream>>>(
+      gu, n, F, static_cast<__nv_bfloat16*>(out));
+  VC_CUDA(cudaGetLastError());
+  return VC_OK;
+}
+
+vc_status vc_glue_append_slots(int32_t* idx, int32_t* deg, int Hkv, int S_cap, int S, int start,
+                               int count, cudaStream_t stream) {
+  if (!idx || Hkv <= 0 || count < 0 || S < 0 || S + count > S_cap)
+    return fail(VC_ERR_INVALID, "append_slots: args");
+  if (count == 0) return VC_OK;
+  append_slots_kernel<<<blocks_for((int64_t)Hkv * count, 256), 256, 0, stream>>>(
+      idx, deg, Hkv, S_cap, S, start, count);
+  VC_CUDA(cudaGetLastError());
+  return VC_OK;
+}
+
+}  // extern "C"

@@ -10,22 +10,24 @@ import lossless_kv_compressed_b200 as vc
 from lossless_kv_compressed_b200 import _lib
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "vericache.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("vericache.h", "vericache_glue.h")]
 
 
-def _declared():
-    text = open(HEADER).read()
+def _declared(path):
+    text = open(path).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(vc_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_library_exports_every_declared_function():
     L = vc.lib()
-    names = _declared()
-    assert len(names) >= 10
-    for n in names:
-        assert hasattr(L, n), f"{n} declared in vericache.h but not exported"
-    assert set(names) == set(_lib.EXPORTS)
+    core, glue = _declared(HEADERS[0]), _declared(HEADERS[1])
+    assert len(core) >= 10 and len(glue) >= 6
+    for n in core + glue:
+        assert hasattr(L, n), f"{n} declared in a header but not exported"
+    assert set(core) == set(_lib.EXPORTS)
+    assert set(glue) == set(_lib.GLUE_EXPORTS)
+    assert sorted(os.listdir(os.path.join(ROOT, "include"))) == ["vericache.h", "vericache_glue.h"]
 
 
 def test_status_strings_and_version():

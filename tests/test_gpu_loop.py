@@ -1,0 +1,146 @@
+"""The draft-then-verify loop end to end on the GPU (VeriCache summary, "Riepilogo
+Tecnico: VeriCache", sections "Algoritmo Principale" and "Risultati Sperimentali":
+outputs identical to full-KV greedy decoding).
+
+* glue kernels: numerics against plain PyTorch fp32, and row invariance (a row's
+  result does not depend on the other rows) -- the property the exactness rests on;
+* the GPU loop's committed stream equals GPU full-KV greedy decoding bit for bit;
+* every round's acceptance is bit-exact with the oracle given the GPU's logits;
+* the GPU decoder follows the fp64 oracle decoder on its first tokens (a structural
+  pin: a wrong RoPE, norm or head layout diverges at once).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import lossless_kv_compressed_b200 as vc
+import oracle
+from lossless_kv_compressed_b200._lib import check, lib
+from lossless_kv_compressed_b200.loop import GpuTinyLM, greedy_loop, vericache_loop
+from oracle import tinylm
+from synth import gen
+from synth.configs import LoopConfig, get_config
+
+pytestmark = pytest.mark.gpu
+S = lambda: torch.cuda.current_stream().cuda_stream
+
+
+def test_gemm_matches_fp32_reference_and_is_row_invariant():
+    torch.manual_seed(0)
+    K, N = 512, 1408 * 2
+    a = torch.randn(37, K, device="cuda").bfloat16()
+    w = (torch.randn(K, N, device="cuda") * 0.02).bfloat16()
+    c = torch.empty(37, N, device="cuda")
+    check(lib().vc_glue_gemm(a.data_ptr(), w.data_ptr(), 37, K, N, c.data_ptr(), 0, S()), "gemm")
+    ref = a.float() @ w.float()
+    torch.cuda.synchronize()
+    assert (c - ref).abs().max().item() < 1e-3 * ref.abs().max().item()
+    for r in (0, 5, 16, 36):
+        c1 = torch.empty(1, N, device="cuda")
+        check(lib().vc_glue_gemm(a[r:r + 1].data_ptr(), w.data_ptr(), 1, K, N, c1.data_ptr(), 0,
+                                 S()), "gemm")
+        torch.cuda.synchronize()
+        assert torch.equal(c1[0], c[r]), f"gemm row {r} depends on the batch"
+    # accumulate mode adds into c
+    c2 = c.clone()
+    check(lib().vc_glue_gemm(a.data_ptr(), w.data_ptr(), 37, K, N, c2.data_ptr(), 1, S()), "gemm")
+    torch.cuda.synchronize()
+    assert torch.allclose(c2, 2 * c, rtol=1e-6, atol=1e-6)
+
+
+def test_rmsnorm_rope_swiglu_match_reference():
+    torch.manual_seed(1)
+    n, d, Hq, Hkv, D, F = 9, 512, 8, 2, 64, 1408
+    x = torch.randn(n, d, device="cuda")
+    h = torch.empty(n, d, dtype=torch.bfloat16, device="cuda")
+    check(lib().vc_glue_rmsnorm(x.data_ptr(), n, d, 1e-5, h.data_ptr(), S()), "rmsnorm")
+    ref = (x / torch.sqrt((x * x).mean(-1, keepdim=True) + 1e-5)).bfloat16()
+    torch.cuda.synchronize()
+    assert (h.float() - ref.float()).abs().max().item() <= 1e-2
+    qkv = torch.randn(n, (Hq + 2 * Hkv) * D, device="cuda")
+    pos = torch.arange(100, 100 + n, dtype=torch.int32, device="cuda")
+    q = torch.empty(n, Hq, D, dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros(Hkv, 200, D, dtype=torch.bfloat16, device="cuda")
+    vcc = torch.zeros_like(kc)
+    check(lib().vc_glue_rope_store(qkv.data_ptr(), pos.data_ptr(), pos.data_ptr(), n, Hq, Hkv, D,
+                                   10000.0, q.data_ptr(), kc.data_ptr(), vcc.data_ptr(), 200, S()),
+          "rope")
+    torch.cuda.synchronize()
+    qr = tinylm.rope(qkv[:, :Hq * D].view(n, Hq, D).double().cpu().numpy(),
+                     np.arange(100, 100 + n), 10000.0)
+    assert np.abs(q.float().cpu().numpy() - qr).max() < 2e-2
+    kr = tinylm.rope(qkv[:, Hq * D:(Hq + Hkv) * D].view(n, Hkv, D).double().cpu().numpy(),
+                     np.arange(100, 100 + n), 10000.0)
+    assert np.abs(kc[:, 100:100 + n].float().cpu().numpy().transpose(1, 0, 2) - kr).max() < 2e-2
+    gu = torch.randn(n, 2 * F, device="cuda")
+    out = torch.empty(n, F, dtype=torch.bfloat16, device="cuda")
+    check(lib().vc_glue_swiglu(gu.data_ptr(), n, F, out.data_ptr(), S()), "swiglu")
+    torch.cuda.synchronize()
+    g, u = gu[:, :F], gu[:, F:]
+    assert (out.float() - torch.nn.functional.silu(g) * u).abs().max().item() < 2e-2
+
+
+SMALL = LoopConfig(n_layers=2, d_model=256, Hq=8, Hkv=2, D=64, ffn=256, vocab=512,
+                   prompt_len=300, gen_tokens=64, k=8, budget=96, n_sinks=4, n_recent=16,
+                   score_window=8, init_std=0.3)
+
+
+def _model(cfg, weights):
+    max_len = cfg.prompt_len + cfg.gen_tokens + cfg.k + 2
+    return GpuTinyLM(weights, cfg, max_len, cfg.k, cfg.budget + cfg.gen_tokens + cfg.k + 2)
+
+
+@pytest.mark.parametrize("cfg", [SMALL, dataclasses.replace(SMALL, init_std=0.05, k=16)])
+def test_loop_commits_equal_greedy_and_accept_is_exact(cfg):
+    w = gen.tinylm_weights(cfg)
+    prompt = gen.tinylm_prompt(cfg)
+    greedy = greedy_loop(_model(cfg, w), prompt, cfg.gen_tokens)
+    rec = []
+    vc_tokens, alens = vericache_loop(_model(cfg, w), prompt, cfg.gen_tokens, cfg.k, cfg.budget,
+                                      cfg.n_sinks, cfg.n_recent, cfg.score_window, record=rec)
+    assert vc_tokens == greedy
+    assert len(alens) >= 2
+    for logits, drafts, got in rec:
+        want = oracle.accept(logits[None], drafts)
+        for key in ("target", "accept_len", "commit", "n_commit", "err"):
+            assert np.array_equal(got[key], want[key]), key
+    assert vc.device_error() == 0
+
+
+def test_gpu_decoder_follows_the_fp64_oracle():
+    cfg = SMALL
+    w = gen.tinylm_weights(cfg)
+    prompt = gen.tinylm_prompt(cfg)
+    n = 12
+    gpu = greedy_loop(_model(cfg, w), prompt, n)
+    ref = tinylm.greedy_loop(tinylm.TinyLM({k: oracle.bf16_to_f64(v) for k, v in w.items()}, cfg),
+                             prompt, n)
+    assert gpu == ref
+
+
+def test_no_compression_accepts_every_draft():
+    """Budget above the prompt: the drafter sees the whole context, so every round
+    accepts all k drafts plus the bonus (VeriCache summary, step 3)."""
+    cfg = dataclasses.replace(SMALL, budget=400, gen_tokens=37)
+    w = gen.tinylm_weights(cfg)
+    prompt = gen.tinylm_prompt(cfg)
+    toks, alens = vericache_loop(_model(cfg, w), prompt, cfg.gen_tokens, cfg.k, cfg.budget,
+                                 cfg.n_sinks, cfg.n_recent, cfg.score_window)
+    full = (cfg.gen_tokens - 1) // (cfg.k + 1)
+    assert alens[:full] == [cfg.k] * full
+    assert toks == greedy_loop(_model(cfg, w), prompt, cfg.gen_tokens)
+
+
+def test_workload5_full_size():
+    """Workload 5: 4 layers, d 512, 8/2 heads of 64, SwiGLU 1408, vocab 8192, N(0, 0.02)
+    weights; 8192-token prompt, 512 generated, k = 32, 2048-slot budget."""
+    cfg = get_config(5)
+    w = gen.tinylm_weights(cfg)
+    prompt = gen.tinylm_prompt(cfg)
+    greedy = greedy_loop(_model(cfg, w), prompt, cfg.gen_tokens)
+    toks, alens = vericache_loop(_model(cfg, w), prompt, cfg.gen_tokens, cfg.k, cfg.budget,
+                                 cfg.n_sinks, cfg.n_recent, cfg.score_window)
+    assert toks == greedy
+    assert sum(a + 1 for a in alens) >= cfg.gen_tokens - 1
