@@ -150,6 +150,8 @@ def profiled_traffic(kernel: str) -> float | None:
 
 # ------------------------------------------------------------------ distributed
 def dist_setup():
+    """One process per GPU (torchrun env).  NCCL on a GPU machine; gloo where there is no GPU
+    (the CPU tests of the N > 1 timing logic)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -157,18 +159,24 @@ def dist_setup():
         import datetime
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout,
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=timeout)
     return world, rank, local
 
 
 def dist_max(x: float, world: int) -> float:
+    """Max of a per-rank time over all ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -177,6 +185,13 @@ def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
+
+
+def job_throughput(units_per_rank_step: float, steps: int, world: int,
+                   t_max_s: float) -> float:
+    """Whole-job rate: the units every rank processed over the slowest rank's time
+    (replicas: each rank runs the same round on its own GPU)."""
+    return world * steps * units_per_rank_step / t_max_s
 
 
 # ------------------------------------------------------------------ oracle baseline
@@ -225,11 +240,14 @@ def cpu_baseline(case, budget_s: float = 20.0) -> dict:
                       f"NumPy on {os.cpu_count()} host cores ({tot_t:.1f} s)"}
 
 
-def run_reference(args, world, rank):
+def run_reference(args, world, rank, case=None):
+    """The oracle as this tier's reference arm: rank 0 alone runs it (other ranks of a
+    torchrun launch exit without work or a process group)."""
     if rank != 0:
         return 0
-    from synth import gen
-    case = gen.attn_case(2)
+    if case is None:
+        from synth import gen
+        case = gen.attn_case(2)
     cfg = case["cfg"]
     pairs = [(b, j) for b in range(cfg.B) for j in range(cfg.Hkv)]
     for w in range(args.warmup):
@@ -587,13 +605,10 @@ def main():
         return run_config4(args)
     if args.config == 5 and args.impl == "vc":
         return run_config5(args)
-    world, rank, local = dist_setup()
     if args.impl == "reference":
-        code = run_reference(args, world, rank)
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
-        return code
+        return run_reference(args, int(os.environ.get("WORLD_SIZE", "1")),
+                             int(os.environ.get("RANK", "0")))
+    world, rank, local = dist_setup()
 
     import torch
     torch.cuda.set_device(local)
@@ -639,7 +654,7 @@ def main():
     t_max = dist_max(step_s, world)
 
     rb = round_bytes(cfg)
-    value = world * args.steps * rb / t_max / 1e9
+    value = job_throughput(rb, args.steps, world, t_max) / 1e9
     peaks = measured_peaks()
     d_bytes = statistics.mean(draft_bytes(cfg, j + 1) for j in range(cfg.k))
     d_time = statistics.mean(draft_s)
