@@ -332,7 +332,9 @@ class Round:
                                                          cfg.P + n_q), dtype=torch.uint8,
                                 device=device)
         self.flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
-        self.launches_per_step = cfg.k * (2 + 2) + 2 + 2
+        # per draft step: split kernel + merge + argmax; verify: kernel + merge;
+        # acceptance: argmax + accept
+        self.launches_per_step = cfg.k * 3 + 2 + 2
 
     def step(self, stream_handle: int, draft_events=None, verify_events=None):
         """Enqueue one round on the stream; optional event pairs around each draft call
@@ -588,6 +590,44 @@ def run_config5(args) -> int:
     return 0
 
 
+def run_profile_case(kind: str) -> int:
+    """A short run of one call of the workload-2 round for an ncu capture: one copy of
+    the inputs (about 1.2 GB on the device), five calls of the chosen entry point."""
+    import torch
+    import lossless_kv_compressed_b200 as vc
+    from synth import gen
+    case = gen.attn_case(2)
+    cfg = case["cfg"]
+    dev = torch.device("cuda", 0)
+    t = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
+        torch.bfloat16).to(dev)
+    k, v = t(case["k_bits"]), t(case["v_bits"])
+    if kind == "draft":
+        cache = vc.IndexedCache(k=k, v=v, S=cfg.S, Hq=cfg.Hq,
+                                idx=torch.from_numpy(case["idx"]).to(dev),
+                                deg=torch.from_numpy(case["deg"]).to(dev),
+                                k_tail=t(gen.bf16_block_rows(case, "k", cfg.k + 1)),
+                                v_tail=t(gen.bf16_block_rows(case, "v", cfg.k + 1)),
+                                n_tail=cfg.k)
+        q = t(case["q_draft_bits"])
+        ws = torch.empty(vc.draft_workspace_size(cache), dtype=torch.uint8, device=dev)
+        for _ in range(5):
+            vc.draft_attn(q, cache, ws=ws)
+    elif kind == "verify":
+        q = t(case["q_verify_bits"])
+        for _ in range(5):
+            vc.verify_attn(q, k, v, cfg.P)
+    else:
+        lg = torch.from_numpy(case["logits"]).to(dev)
+        dr = torch.from_numpy(case["drafts"]).to(dev)
+        for _ in range(5):
+            vc.accept(lg, dr)
+            vc.accept(lg[:, :1].contiguous())
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": kind, "workload": cfg.name, "ok": True}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -595,12 +635,17 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="vc", choices=["vc", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=["draft", "verify", "accept"], default=None,
+                    help="run five calls of one entry point on the workload-2 inputs (one "
+                         "copy) for an ncu capture, and print no bench line")
     ap.add_argument("--config", type=int, default=2, choices=[2, 4, 5],
                     help="2: the round of the 32K-context layer (default line); "
                          "4: long-context staging while drafting; 5: the loop end to end")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.profile_case:
+        return run_profile_case(args.profile_case)
     if args.config == 4 and args.impl == "vc":
         return run_config4(args)
     if args.config == 5 and args.impl == "vc":

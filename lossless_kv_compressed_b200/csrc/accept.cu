@@ -4,11 +4,15 @@
 // agree.
 //
 // Kernel 1: float4 streaming argmax of each logits row (ties -> lowest index; NaN
-//           larger than any number, first NaN wins); large vocabularies split a row
-//           over an 8-CTA cluster merged through distributed shared memory.  The
-//           row's NaN bit is parked in bit 31 of its target entry.
-// Kernel 2: one warp per batch row: clears the NaN bits into err_flag, finds the first
-//           disagreement with a ballot, and writes accept_len / commit / n_commit.
+//           larger than any number, first NaN wins).  Each thread keeps 8 float4 loads
+//           in flight; when the rows are few (a draft step's B rows) each row is split
+//           over a cluster of up to 8 CTAs merged through distributed shared memory, so
+//           the grid still covers the SMs.  The row's NaN bit is parked in bit 31 of its
+//           target entry -- except for one-position rows (n_q == 1), whose outputs this
+//           kernel finishes itself (a single launch per draft step).
+// Kernel 2 (n_q > 1): one warp per batch row: clears the NaN bits into err_flag, finds
+//           the first disagreement with a ballot, and writes accept_len / commit /
+//           n_commit.
 #include <climits>
 
 #include <cooperative_groups.h>
@@ -29,40 +33,65 @@ __device__ __forceinline__ bool better(float v, int i, const ArgBest& b) {
   return v > b.val || (v == b.val && i < b.idx);
 }
 
+// Outputs of a one-position row (n_q == 1), written by the argmax kernel itself so that
+// the draft-time argmax is a single launch: the target without its NaN bit, the row's
+// NaN flag, and -- in acceptance mode -- accept_len 0, commit [target], n_commit 1.
+struct RowEpilogue {
+  int32_t* accept_len;
+  int32_t* commit;
+  int32_t* n_commit;
+  int32_t* err_flag;
+  int fused;
+};
+
 // One row per thread-block cluster of CL CTAs: CTA c scans a contiguous slice of the
-// row, the cluster's rank-0 CTA merges the CL partials through distributed shared
-// memory (slices in order, so the lowest index still wins ties).
-template <int THREADS, int CL>
+// row, U float4 loads in flight per thread before any is compared, stores its result
+// into the cluster leader's shared memory (one cluster barrier), and the leader merges
+// the CL results (any order gives the same winner: larger value, then lower index).
+template <int THREADS, int CL, int U>
 __global__ void __launch_bounds__(THREADS) argmax_rows_kernel(const float* __restrict__ logits,
-                                                              int V, int32_t* __restrict__ target) {
+                                                              int V, int32_t* __restrict__ target,
+                                                              RowEpilogue ep) {
   namespace cg = cooperative_groups;
   const int64_t row = blockIdx.x / CL;
   const int crank = (int)(blockIdx.x % CL);
   const float* x = logits + row * (int64_t)V;
+  // Distributed shared memory of a CTA may be written only once that CTA has started:
+  // arrive now, wait just before the remote stores (every CTA has long started by then).
+  if constexpr (CL > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
   // slice [lo, hi) of the row, multiples of 4 so float4 loads stay aligned
   const int per = ((V + CL - 1) / CL + 3) & ~3;
   const int lo = min(V, crank * per), hi = min(V, lo + per);
   ArgBest best{-INFINITY, INT_MAX};
   int first_nan = INT_MAX;
+  auto take = [&](float e, int id) {
+    if (isnan(e)) first_nan = min(first_nan, id);
+    else if (better(e, id, best)) best = {e, id};
+  };
   const bool vec = ((V & 3) == 0) && ((reinterpret_cast<uintptr_t>(x) & 15) == 0);
   if (vec) {
     const float4* x4 = reinterpret_cast<const float4*>(x);
-    for (int i = (lo >> 2) + threadIdx.x; i < (hi >> 2); i += THREADS) {
-      const float4 f = __ldg(x4 + i);
-      const float e[4] = {f.x, f.y, f.z, f.w};
+    const int lo4 = lo >> 2, hi4 = hi >> 2;
+    for (int base = lo4 + (int)threadIdx.x; base < hi4; base += THREADS * U) {
+      float4 f[U];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int id = 4 * i + u;
-        if (isnan(e[u])) first_nan = min(first_nan, id);
-        else if (better(e[u], id, best)) best = {e[u], id};
+      for (int u = 0; u < U; ++u) {
+        const int i = base + u * THREADS;
+        f[u] = i < hi4 ? __ldcs(x4 + i) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = base + u * THREADS;
+        if (i < hi4) {
+          take(f[u].x, 4 * i);
+          take(f[u].y, 4 * i + 1);
+          take(f[u].z, 4 * i + 2);
+          take(f[u].w, 4 * i + 3);
+        }
       }
     }
   } else {
-    for (int i = lo + threadIdx.x; i < hi; i += THREADS) {
-      const float e = __ldg(x + i);
-      if (isnan(e)) first_nan = min(first_nan, i);
-      else if (better(e, i, best)) best = {e, i};
-    }
+    for (int i = lo + threadIdx.x; i < hi; i += THREADS) take(__ldg(x + i), i);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -74,11 +103,12 @@ __global__ void __launch_bounds__(THREADS) argmax_rows_kernel(const float* __res
   __shared__ float sv[THREADS / 32];
   __shared__ int si[THREADS / 32];
   __shared__ int sn[THREADS / 32];
-  __shared__ float cv;   // this CTA's result, read by the cluster leader
-  __shared__ int ci, cn;
+  __shared__ float cv[CL];   // each CTA's result, gathered in the cluster leader's copy
+  __shared__ int ci[CL], cn[CL];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0) { sv[warp] = best.val; si[warp] = best.idx; sn[warp] = first_nan; }
   __syncthreads();
+  if constexpr (CL > 1) asm volatile("barrier.cluster.wait.aligned;\n" ::: "memory");
   if (warp == 0) {
     constexpr int NW = THREADS / 32;
     best = lane < NW ? ArgBest{sv[lane], si[lane]} : ArgBest{-INFINITY, INT_MAX};
@@ -90,31 +120,52 @@ __global__ void __launch_bounds__(THREADS) argmax_rows_kernel(const float* __res
       if (better(v, i, best)) best = {v, i};
       first_nan = min(first_nan, __shfl_xor_sync(0xffffffffu, first_nan, o));
     }
-    if (lane == 0) { cv = best.val; ci = best.idx; cn = first_nan; }
+    if (lane == 0) {
+      // write this CTA's result into the leader's slot `crank` (a remote store through
+      // distributed shared memory for the other CTAs of the cluster)
+      if constexpr (CL > 1) {
+        cg::cluster_group cluster = cg::this_cluster();
+        *cluster.map_shared_rank(&cv[crank], 0) = best.val;
+        *cluster.map_shared_rank(&ci[crank], 0) = best.idx;
+        *cluster.map_shared_rank(&cn[crank], 0) = first_nan;
+      } else {
+        cv[0] = best.val; ci[0] = best.idx; cn[0] = first_nan;
+      }
+    }
   }
   if constexpr (CL > 1) {
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
-    if (crank == 0 && threadIdx.x == 0) {
-      best = {cv, ci};
-      first_nan = cn;
-      for (int r = 1; r < CL; ++r) {
-        const float v = *cluster.map_shared_rank(&cv, r);
-        const int i = *cluster.map_shared_rank(&ci, r);
-        if (better(v, i, best)) best = {v, i};
-        first_nan = min(first_nan, *cluster.map_shared_rank(&cn, r));
-      }
-      cv = best.val; ci = best.idx; cn = first_nan;
-    }
-    cluster.sync();   // peers keep their shared memory until the leader has read it
+    cg::this_cluster().sync();   // release the remote stores, acquire them in the leader
   } else {
     __syncthreads();
   }
+  int res_i = INT_MAX, res_n = INT_MAX;
+  if (crank == 0 && threadIdx.x == 0) {
+    best = {cv[0], ci[0]};
+    first_nan = cn[0];
+#pragma unroll
+    for (int r = 1; r < CL; ++r) {
+      if (better(cv[r], ci[r], best)) best = {cv[r], ci[r]};
+      first_nan = min(first_nan, cn[r]);
+    }
+    res_i = best.idx;
+    res_n = first_nan;
+  }
   if (crank == 0 && threadIdx.x == 0) {
     // an all -inf row: every entry ties at -inf, lowest index 0 wins
-    int t = ci == INT_MAX ? 0 : ci;
-    if (cn != INT_MAX) t = cn | (int)0x80000000u;
-    target[row] = t;
+    int t = res_i == INT_MAX ? 0 : res_i;
+    const bool nan = res_n != INT_MAX;
+    if (nan) t = res_n;
+    if (!ep.fused) {
+      target[row] = nan ? (t | (int)0x80000000u) : t;
+    } else {
+      target[row] = t;
+      if (ep.err_flag) ep.err_flag[row] = nan ? 1 : 0;
+      if (ep.commit) {
+        ep.accept_len[row] = 0;
+        ep.commit[row] = t;
+        ep.n_commit[row] = 1;
+      }
+    }
   }
 }
 
@@ -152,15 +203,20 @@ __global__ void accept_kernel(int n_q, const int32_t* __restrict__ drafts,
   for (int i = lane; i < n_q; i += 32) commit[(int64_t)b * n_q + i] = i <= a ? tg[i] : -1;
 }
 
-vc_status launch_accept(const float* logits, const int32_t* drafts, int B, int n_q, int V,
-                        int32_t* target, int32_t* accept_len, int32_t* commit,
-                        int32_t* n_commit, int32_t* err_flag, cudaStream_t stream) {
-  const int rows = B * n_q;
-  if (V >= 16384) {
-    constexpr int CL = 8;
+namespace {
+constexpr int kArgThreads = 512;
+constexpr int kArgUnroll = 8;
+
+template <int CL>
+vc_status launch_argmax(const float* logits, int V, int rows, int32_t* target,
+                        const RowEpilogue& ep, cudaStream_t stream) {
+  if constexpr (CL == 1) {
+    argmax_rows_kernel<kArgThreads, 1, kArgUnroll><<<rows, kArgThreads, 0, stream>>>(
+        logits, V, target, ep);
+  } else {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(rows * CL);
-    cfg.blockDim = dim3(256);
+    cfg.blockDim = dim3(kArgThreads);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -169,11 +225,36 @@ vc_status launch_accept(const float* logits, const int32_t* drafts, int B, int n
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    VC_CUDA(cudaLaunchKernelEx(&cfg, argmax_rows_kernel<256, CL>, logits, V, target));
-  } else {
-    argmax_rows_kernel<128, 1><<<rows, 128, 0, stream>>>(logits, V, target);
+    VC_CUDA(cudaLaunchKernelEx(&cfg, argmax_rows_kernel<kArgThreads, CL, kArgUnroll>, logits,
+                               V, target, ep));
   }
   VC_CUDA(cudaGetLastError());
+  return VC_OK;
+}
+}  // namespace
+
+// Cluster size: split rows over more CTAs while the grid still fits in one wave of two
+// CTAs per SM and every CTA keeps at least 2048 logits.
+int argmax_cluster(int rows, int V) {
+  int cl = 1;
+  while (cl < 8 && (int64_t)rows * cl * 2 <= 2 * (int64_t)num_sms() && V / (2 * cl) >= 2048)
+    cl *= 2;
+  return cl;
+}
+
+vc_status launch_accept(const float* logits, const int32_t* drafts, int B, int n_q, int V,
+                        int32_t* target, int32_t* accept_len, int32_t* commit,
+                        int32_t* n_commit, int32_t* err_flag, cudaStream_t stream) {
+  const int rows = B * n_q;
+  RowEpilogue ep{accept_len, commit, n_commit, err_flag, n_q == 1 ? 1 : 0};
+  vc_status st;
+  switch (argmax_cluster(rows, V)) {
+    case 1: st = launch_argmax<1>(logits, V, rows, target, ep, stream); break;
+    case 2: st = launch_argmax<2>(logits, V, rows, target, ep, stream); break;
+    case 4: st = launch_argmax<4>(logits, V, rows, target, ep, stream); break;
+    default: st = launch_argmax<8>(logits, V, rows, target, ep, stream); break;
+  }
+  if (st != VC_OK || n_q == 1) return st;
   accept_kernel<<<B, 32, 0, stream>>>(n_q, drafts, target, accept_len, commit, n_commit,
                                       err_flag);
   VC_CUDA(cudaGetLastError());

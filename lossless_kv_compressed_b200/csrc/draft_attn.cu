@@ -629,37 +629,99 @@ struct PartialSet {
   int W, maxseg;
 };
 
-// Fixed-order merge of up to two partial sets for one head: block (pair, head), D threads.
+// Merge of up to two partial sets, one CTA of kCombWarps warps per (pair, head).  The
+// pair's segments are cut into one contiguous share per warp; a warp loads the (max,
+// sum) of up to 8 segments and their unnormalised outputs all at once (its lanes hold
+// D/32 channels each), so a share of <= 8 segments costs one L2 round trip, and folds
+// them into its running (m, l, o) with the weights broadcast by shuffle.  The warps'
+// states are then merged through shared memory in warp order.  Every sum runs in an
+// order fixed by the launch configuration, so results are reproducible.
+constexpr int kCombWarps = 4;
+constexpr int kCombChunk = 8;
+
 template <int D, typename OutT>
-__global__ void __launch_bounds__(D) draft_combine_kernel(PartialSet a, PartialSet b, int nsets,
-                                                          int g, int Hkv, int Hq,
-                                                          OutT* __restrict__ out,
-                                                          float* __restrict__ lse) {
+__global__ void __launch_bounds__(kCombWarps * 32) draft_combine_kernel(
+    PartialSet a, PartialSet b, int nsets, int g, int Hkv, int Hq, OutT* __restrict__ out,
+    float* __restrict__ lse) {
+  constexpr int DPL = D / 32;                 // output channels per lane
+  __shared__ float s_o[kCombWarps][D];
+  __shared__ float s_m[kCombWarps], s_l[kCombWarps];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t pair = blockIdx.x / g;
-  const int r = blockIdx.x - (int)(pair * g);
-  const int d = threadIdx.x;
-  float M = -INFINITY, L = 0.f, O = 0.f;
-  for (int si = 0; si < nsets; ++si) {
-    const PartialSet& ps = si == 0 ? a : b;
+  const int r = (int)(blockIdx.x - pair * g);
+  float m = -INFINITY, l = 0.f, o[DPL];
+#pragma unroll
+  for (int j = 0; j < DPL; ++j) o[j] = 0.f;
+  // Fold segments [s_begin, s_end) of one set into (m, l, o).  The segments of this pair
+  // are warps w0 + s; empty warp ranges wrote no partial and get weight 0.
+  auto fold = [&](const PartialSet& ps) {
     const int64_t w0 = warp_of_tile(pair * ps.upp, ps.T, ps.W);
-    const int64_t w1 = warp_of_tile((pair + 1) * ps.upp - 1, ps.T, ps.W);
-#pragma unroll 4
-    for (int64_t w = w0; w <= w1; ++w) {
-      if (warp_begin(w, ps.T, ps.W) >= warp_begin(w + 1, ps.T, ps.W)) continue;   // empty
-      const int64_t pr = (pair * ps.maxseg + (w - w0)) * g + r;
-      const float2 ml = *reinterpret_cast<const float2*>(ps.ml + pr * 2);
-      const float os = ps.o[pr * D + d];
-      const float Mn = fmaxf(M, ml.x);
-      const float fa = ex2(M - Mn), fc = ex2(ml.x - Mn);
-      L = fmaf(L, fa, ml.y * fc);
-      O = fmaf(O, fa, os * fc);
-      M = Mn;
+    const int n = (int)(warp_of_tile((pair + 1) * ps.upp - 1, ps.T, ps.W) - w0 + 1);
+    const int s_begin = warp * n / kCombWarps, s_end = (warp + 1) * n / kCombWarps;
+    for (int c0 = s_begin; c0 < s_end; c0 += kCombChunk) {
+      const int cnt = min(kCombChunk, s_end - c0);
+      float2 ml = make_float2(-INFINITY, 0.f);
+      if (lane < cnt && warp_begin(w0 + c0 + lane, ps.T, ps.W) <
+                            warp_begin(w0 + c0 + lane + 1, ps.T, ps.W))
+        ml = *reinterpret_cast<const float2*>(ps.ml + ((pair * ps.maxseg + c0 + lane) * g + r) * 2);
+      float v[kCombChunk][DPL];
+#pragma unroll
+      for (int j = 0; j < kCombChunk; ++j) {
+        const float* src = ps.o + ((pair * ps.maxseg + c0 + min(j, cnt - 1)) * g + r) * D + lane * DPL;
+        if constexpr (DPL == 4) {
+          const float4 t = *reinterpret_cast<const float4*>(src);
+          v[j][0] = t.x; v[j][1] = t.y; v[j][2] = t.z; v[j][3] = t.w;
+        } else {
+          const float2 t = *reinterpret_cast<const float2*>(src);
+          v[j][0] = t.x; v[j][1] = t.y;
+        }
+      }
+      float mc = ml.x;
+#pragma unroll
+      for (int x = 1; x < kCombChunk; x <<= 1) mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, x));
+      mc = __shfl_sync(0xffffffffu, mc, 0);
+      const float m_new = fmaxf(m, mc);
+      if (m_new == -INFINITY) continue;          // nothing live yet
+      const float alpha = m == -INFINITY ? 0.f : ex2(m - m_new);
+      const float wl = ml.x == -INFINITY ? 0.f : ex2(ml.x - m_new);
+      l *= alpha;
+#pragma unroll
+      for (int t = 0; t < DPL; ++t) o[t] *= alpha;
+#pragma unroll
+      for (int j = 0; j < kCombChunk; ++j) {
+        const float w = __shfl_sync(0xffffffffu, wl, j);
+        const float lj = __shfl_sync(0xffffffffu, ml.y, j);
+        if (j < cnt && w != 0.f) {               // warp-uniform
+          l = fmaf(w, lj, l);
+#pragma unroll
+          for (int t = 0; t < DPL; ++t) o[t] = fmaf(w, v[j][t], o[t]);
+        }
+      }
+      m = m_new;
     }
-  }
+  };
+  fold(a);
+  if (nsets > 1) fold(b);
+#pragma unroll
+  for (int t = 0; t < DPL; ++t) s_o[warp][lane * DPL + t] = o[t];
+  if (lane == 0) { s_m[warp] = m; s_l[warp] = l; }
+  __syncthreads();
   const int64_t bb = pair / Hkv, j = pair - bb * Hkv;
   const int64_t h = bb * Hq + j * g + r;
-  store_out(out + h * D + d, O / L);
-  if (lse && d == 0) lse[h] = (M + __log2f(L)) * kLn2;
+  for (int d = threadIdx.x; d < D; d += kCombWarps * 32) {
+    float M = s_m[0];
+#pragma unroll
+    for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, s_m[w]);
+    float L = 0.f, O = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCombWarps; ++w) {
+      const float f = s_m[w] == -INFINITY ? 0.f : ex2(s_m[w] - M);
+      L = fmaf(s_l[w], f, L);
+      O = fmaf(s_o[w][d], f, O);
+    }
+    store_out(out + h * D + d, O / L);
+    if (lse && d == 0) lse[h] = (M + __log2f(L)) * kLn2;
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -719,11 +781,12 @@ template <int D>
 vc_status launch_combine(const PartialSet& a, const PartialSet& b, int nsets, int pairs, int g,
                          int Hkv, int Hq, int flags, void* out, float* lse, cudaStream_t stream) {
   const int blocks = pairs * g;
+  constexpr int T = kCombWarps * 32;
   if (flags & VC_OUT_F32)
-    draft_combine_kernel<D, float><<<blocks, D, 0, stream>>>(a, b, nsets, g, Hkv, Hq,
+    draft_combine_kernel<D, float><<<blocks, T, 0, stream>>>(a, b, nsets, g, Hkv, Hq,
                                                              static_cast<float*>(out), lse);
   else
-    draft_combine_kernel<D, __nv_bfloat16><<<blocks, D, 0, stream>>>(
+    draft_combine_kernel<D, __nv_bfloat16><<<blocks, T, 0, stream>>>(
         a, b, nsets, g, Hkv, Hq, static_cast<__nv_bfloat16*>(out), lse);
   VC_CUDA(cudaGetLastError());
   return VC_OK;

@@ -384,48 +384,89 @@ __global__ void __launch_bounds__(kVThreads, 1)
   }
 }
 
-// Merge split partials in split order (plus the carried state) for one query row.
+// Merge split partials (plus the carried state) for one query row: one warp per row,
+// lanes holding D/32 output channels each.  The lanes load the splits' (max, sum) at
+// once; the unnormalised outputs of 8 splits are loaded together before any is used,
+// so a row costs a few L2 round trips, not one per split.  The sums run in split order
+// after the carried state, the same order whatever the number of rows, which keeps a
+// verify row bit-identical to the same position decoded alone.
+constexpr int kVCombWarps = 8;
+
 template <int D, typename OutT>
-__global__ void __launch_bounds__(D) verify_combine_kernel(
+__global__ void __launch_bounds__(kVCombWarps * 32) verify_combine_kernel(
     const float* __restrict__ ws_o, const float* __restrict__ ws_ml, int n_split, int R, int g,
     int n_q, int Hq, int Hkv, int flags, float* m_state, float* l_state, float* acc_state,
-    OutT* __restrict__ out) {
-  const int pair = blockIdx.x / R, row = blockIdx.x - pair * R;
-  const int d = threadIdx.x;
+    OutT* __restrict__ out, int rows) {
+  constexpr int DPL = D / 32;
+  constexpr int CH = 8;
+  const int lane = threadIdx.x & 31;
+  const int gr = blockIdx.x * kVCombWarps + (threadIdx.x >> 5);
+  if (gr >= rows) return;
+  const int pair = gr / R, row = gr - pair * R;
   const int i = row / g, hl = row - i * g;
   const int b = pair / Hkv, kvh = pair - b * Hkv;
   const int64_t sidx = ((int64_t)b * n_q + i) * Hq + kvh * g + hl;
   const bool carry = m_state != nullptr && !(flags & VC_VERIFY_FIRST);
-  float cm = -INFINITY, cl = 0.f, co = 0.f;
+  const int64_t pr0 = (int64_t)pair * n_split * R + row;   // split s: pr0 + s * R
+  float M = carry ? m_state[sidx] : -INFINITY;
+  for (int s = lane; s < n_split; s += 32) M = fmaxf(M, ws_ml[(pr0 + (int64_t)s * R) * 2]);
+  M = warp_max_xor(M, 5);
+  float Ls = 0.f, O[DPL];
+#pragma unroll
+  for (int t = 0; t < DPL; ++t) O[t] = 0.f;
   if (carry) {
-    cm = m_state[sidx];
-    cl = l_state[sidx];
-    co = acc_state[sidx * D + d];
+    const float cm = m_state[sidx];
+    if (cm > -INFINITY) {
+      const float f = ex2(cm - M);
+      Ls = l_state[sidx] * f;
+#pragma unroll
+      for (int t = 0; t < DPL; ++t) O[t] = acc_state[sidx * D + lane * DPL + t] * f;
+    }
   }
-  __syncthreads();
-  float M = cm;
-  for (int s = 0; s < n_split; ++s)
-    M = fmaxf(M, ws_ml[(((int64_t)pair * n_split + s) * R + row) * 2]);
-  float Ls = 0.f, O = 0.f;
-  if (cm > -INFINITY) {
-    const float f = ex2(cm - M);
-    Ls = cl * f;
-    O = co * f;
-  }
-  for (int s = 0; s < n_split; ++s) {
-    const int64_t pr = ((int64_t)pair * n_split + s) * R + row;
-    const float ms = ws_ml[pr * 2];
-    if (ms > -INFINITY) {
-      const float f = ex2(ms - M);
-      Ls = fmaf(ws_ml[pr * 2 + 1], f, Ls);
-      O = fmaf(ws_o[pr * D + d], f, O);
+  for (int s0 = 0; s0 < n_split; s0 += 32) {
+    const int cnt32 = min(32, n_split - s0);
+    float wl = 0.f, ll = 0.f;
+    if (lane < cnt32) {
+      const float2 ml = *reinterpret_cast<const float2*>(ws_ml + (pr0 + (int64_t)(s0 + lane) * R) * 2);
+      if (ml.x > -INFINITY) {
+        wl = ex2(ml.x - M);
+        ll = ml.y;
+      }
+    }
+    for (int c0 = 0; c0 < cnt32; c0 += CH) {
+      float v[CH][DPL];
+#pragma unroll
+      for (int j = 0; j < CH; ++j) {
+        const int s = s0 + min(c0 + j, cnt32 - 1);
+        const float* src = ws_o + (pr0 + (int64_t)s * R) * D + lane * DPL;
+        if constexpr (DPL == 4) {
+          const float4 t = *reinterpret_cast<const float4*>(src);
+          v[j][0] = t.x; v[j][1] = t.y; v[j][2] = t.z; v[j][3] = t.w;
+        } else {
+          const float2 t = *reinterpret_cast<const float2*>(src);
+          v[j][0] = t.x; v[j][1] = t.y;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < CH; ++j) {
+        const float w = __shfl_sync(0xffffffffu, wl, c0 + j);
+        const float lj = __shfl_sync(0xffffffffu, ll, c0 + j);
+        if (c0 + j < cnt32 && w != 0.f) {         // warp-uniform
+          Ls = fmaf(lj, w, Ls);
+#pragma unroll
+          for (int t = 0; t < DPL; ++t) O[t] = fmaf(v[j][t], w, O[t]);
+        }
+      }
     }
   }
   if (flags & VC_VERIFY_LAST) {
-    store_out(out + sidx * D + d, O / Ls);
+    const float inv = 1.f / Ls;
+#pragma unroll
+    for (int t = 0; t < DPL; ++t) store_out(out + sidx * D + lane * DPL + t, O[t] * inv);
   } else {
-    acc_state[sidx * D + d] = O;
-    if (d == 0) {
+#pragma unroll
+    for (int t = 0; t < DPL; ++t) acc_state[sidx * D + lane * DPL + t] = O[t];
+    if (lane == 0) {
       m_state[sidx] = M;
       l_state[sidx] = Ls;
     }
@@ -497,14 +538,16 @@ static vc_status run_verify(const Plan& pl, const VerifyParams& vp, const CUtens
   dim3 grid(pl.n_split, pl.n_rg, pl.pairs);
   verify_kernel<D><<<grid, kVThreads, L::kAlloc, stream>>>(mk, mv, vp);
   VC_CUDA(cudaGetLastError());
+  const int rows = pl.pairs * pl.R;
+  const int cblocks = (rows + kVCombWarps - 1) / kVCombWarps;
   if (flags & VC_OUT_F32)
-    verify_combine_kernel<D, float><<<pl.pairs * pl.R, D, 0, stream>>>(
+    verify_combine_kernel<D, float><<<cblocks, kVCombWarps * 32, 0, stream>>>(
         vp.ws_o, vp.ws_ml, pl.n_split, pl.R, pl.g, vp.n_q, vp.Hq, vp.Hkv, flags, m, l, acc,
-        static_cast<float*>(out));
+        static_cast<float*>(out), rows);
   else
-    verify_combine_kernel<D, __nv_bfloat16><<<pl.pairs * pl.R, D, 0, stream>>>(
+    verify_combine_kernel<D, __nv_bfloat16><<<cblocks, kVCombWarps * 32, 0, stream>>>(
         vp.ws_o, vp.ws_ml, pl.n_split, pl.R, pl.g, vp.n_q, vp.Hq, vp.Hkv, flags, m, l, acc,
-        static_cast<__nv_bfloat16*>(out));
+        static_cast<__nv_bfloat16*>(out), rows);
   VC_CUDA(cudaGetLastError());
   return VC_OK;
 }
