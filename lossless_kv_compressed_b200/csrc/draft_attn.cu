@@ -92,21 +92,39 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
   float* tbias = reinterpret_cast<float*>(trow + 2 * kTabE);
   const int total = p.S + p.n_tail;
 
+  // Tile x0 + i lies in pair (x0 + i) / tpp.  The pair and the tile's place in it are
+  // carried forward as the tiles advance, so the loop divides nothing in 64 bits.
+  const int tpp = p.tpp;
+  const int64_t pair_first = x0 / tpp;
+  const int rem_first = (int)(x0 - pair_first * tpp);
+  auto advance = [&](int64_t& pair, int& rem, int by) {
+    rem += by;
+    if (rem >= tpp) {
+      const int q = rem / tpp;
+      pair += q;
+      rem -= q * tpp;
+    }
+  };
+
   // ---- slot table: raw idx / degree of one batch prefetched into registers, then
   //      validated and staged into shared memory when the copies reach that batch.
+  //      Entry e of a batch is slot e % 16 of the batch's tile e / 16.
   int32_t ri[kTabE / 32], rd[kTabE / 32];
-  auto slot_of = [&](int b, int e, int64_t& pair) -> int {
-    const int local = b * kTB + e / kTile;
-    if (local >= n) return -1;
-    const int64_t x = x0 + local;
-    pair = x / p.tpp;
-    return (int)(x - pair * p.tpp) * kTile + (e % kTile);
+  int64_t lb_pair = pair_first, sb_pair = pair_first;   // first tile of the batch being
+  int lb_rem = rem_first, sb_rem = rem_first;           // loaded / stored
+  auto slot_of = [&](int b, int e, int64_t bpair, int brem, int64_t& pair) -> int {
+    const int t = e / kTile;
+    if (b * kTB + t >= n) return -1;
+    pair = bpair;
+    int rem = brem;
+    advance(pair, rem, t);
+    return rem * kTile + (e % kTile);
   };
   auto load_batch = [&](int b) {
 #pragma unroll
     for (int i = 0; i < kTabE / 32; ++i) {
       int64_t pair = 0;
-      const int s = slot_of(b, lane + 32 * i, pair);
+      const int s = slot_of(b, lane + 32 * i, lb_pair, lb_rem, pair);
       ri[i] = 0;
       rd[i] = 1;
       if (s >= 0 && s < p.S) {
@@ -115,6 +133,7 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
         rd[i] = p.deg ? __ldg(p.deg + o) : 1;
       }
     }
+    advance(lb_pair, lb_rem, kTB);
   };
   auto store_batch = [&](int b) {
     const int buf = b & 1;
@@ -123,7 +142,7 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
     for (int i = 0; i < kTabE / 32; ++i) {
       const int e = lane + 32 * i;
       int64_t pair = 0;
-      const int s = slot_of(b, e, pair);
+      const int s = slot_of(b, e, sb_pair, sb_rem, pair);
       int32_t code = kNone;
       float bias = -INFINITY;
       if (s >= 0 && s < p.S) {
@@ -139,6 +158,7 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
       trow[buf * kTabE + e] = code;
       tbias[buf * kTabE + e] = bias;
     }
+    advance(sb_pair, sb_rem, kTB);
     if (bad && p.err_flag) atomicExch(p.err_flag, 1);
     __syncwarp();
   };
@@ -151,6 +171,12 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
 
   // The table of batch b is staged when the copies first reach it; the compute trails
   // by fewer than kTB tiles, so the other buffer still holds what it reads.
+  // Lane l copies chunk l % CH of rows (l / CH) * NI + i, i < NI: its NI row codes are
+  // contiguous in the table (two 16-byte shared loads at D = 128).
+  constexpr int NI = kTile * CH / 32;
+  const int c_ln = lane % CH, r_ln = (lane / CH) * NI;
+  int64_t is_pair = pair_first;
+  int is_rem = rem_first;
   auto issue = [&](int it, int st) {
     const int b = it / kTB;
     if (b == pending) {
@@ -158,28 +184,31 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
       ++pending;
       if (pending < nb) load_batch(pending);
     }
-    const int64_t x = x0 + it;
-    const int64_t pair = x / p.tpp;
-    const __nv_bfloat16* kb = p.k + pair * p.T_cap * D;
-    const __nv_bfloat16* vb = p.v + pair * p.T_cap * D;
-    const __nv_bfloat16* kt = p.k_tail ? p.k_tail + pair * p.R_cap * D : kb;
-    const __nv_bfloat16* vt = p.v_tail ? p.v_tail + pair * p.R_cap * D : vb;
+    const int64_t pair = is_pair;
+    advance(is_pair, is_rem, 1);
+    const uint64_t kb = reinterpret_cast<uint64_t>(p.k + pair * p.T_cap * D);
+    const uint64_t vb = reinterpret_cast<uint64_t>(p.v + pair * p.T_cap * D);
+    const uint64_t kt = p.k_tail ? reinterpret_cast<uint64_t>(p.k_tail + pair * p.R_cap * D) : kb;
+    const uint64_t vt = p.v_tail ? reinterpret_cast<uint64_t>(p.v_tail + pair * p.R_cap * D) : vb;
     const int e0 = (b & 1) * kTabE + (it % kTB) * kTile;
+    int32_t code[NI];
+#pragma unroll
+    for (int i = 0; i < NI; i += 4) {
+      const int4 c4 = *reinterpret_cast<const int4*>(trow + e0 + r_ln + i);
+      code[i] = c4.x; code[i + 1] = c4.y; code[i + 2] = c4.z; code[i + 3] = c4.w;
+    }
     const uint32_t kd = wbuf_s + st * SM::kStageB;
     const uint32_t vd = kd + SM::kTileB;
 #pragma unroll
-    for (int i = 0; i < kTile * CH / 32; ++i) {
-      const int lin = lane + 32 * i;
-      const int r = lin / CH, c = lin % CH;
-      const int32_t code = trow[e0 + r];
-      const bool ok = code != kNone;
-      const __nv_bfloat16* kp =
-          code >= 0 ? kb + (int64_t)code * D : (ok ? kt + (int64_t)(-code - 1) * D : kb);
-      const __nv_bfloat16* vp =
-          code >= 0 ? vb + (int64_t)code * D : (ok ? vt + (int64_t)(-code - 1) * D : vb);
-      const uint32_t off = r * SM::kRowB + ((c ^ (r & 7)) << 4);
-      cp_async16(kd + off, kp + c * 8, ok ? 16u : 0u);
-      cp_async16(vd + off, vp + c * 8, ok ? 16u : 0u);
+    for (int i = 0; i < NI; ++i) {
+      const int r = r_ln + i;
+      const bool ok = code[i] != kNone;
+      const bool tail = code[i] < 0;
+      // byte offset of the chunk in its row (a masked slot reads nothing: size 0)
+      const uint64_t bo = ok ? ((uint64_t)(tail ? -code[i] - 1 : code[i]) * D + c_ln * 8) * 2 : 0;
+      const uint32_t off = r * SM::kRowB + ((c_ln ^ (r & 7)) << 4);
+      cp_async16(kd + off, reinterpret_cast<const void*>((tail ? kt : kb) + bo), ok ? 16u : 0u);
+      cp_async16(vd + off, reinterpret_cast<const void*>((tail ? vt : vb) + bo), ok ? 16u : 0u);
     }
   };
 
@@ -197,8 +226,7 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
       dst[ks][1] = ok ? __ldg(qp + (16 * ks + 8 + 2 * qc) / 2) : 0u;
     }
   };
-  const int64_t pair_first = x0 / p.tpp;
-  const int64_t pair_last = (x0 + n - 1) / p.tpp;
+  const int64_t pair_last = (x0 + n - 1) / tpp;
   load_q(pair_first, qa);
   if (pair_last > pair_first) load_q(pair_first + 1, qn);
 
@@ -233,30 +261,34 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
     cp_async_commit();
   }
 
+  int c_rem = rem_first;
   for (int it = 0; it < n; ++it) {
     if (it + NST - 1 < n) issue(it + NST - 1, (it + NST - 1) % NST);
     cp_async_commit();
     cp_async_wait<NST - 1>();
     __syncwarp();
-    const int64_t pair = (x0 + it) / p.tpp;
-    if (pair != cur) {                               // segment boundary
+    if (c_rem == tpp) {                              // segment boundary
+      c_rem = 0;
       flush(cur);
       reset();
-      cur = pair;
+      ++cur;
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) { qa[ks][0] = qn[ks][0]; qa[ks][1] = qn[ks][1]; }
-      if (pair < pair_last) load_q(pair + 1, qn);
+      if (cur < pair_last) load_q(cur + 1, qn);
     }
+    ++c_rem;
     const int st = it % NST;
     const uint32_t ks_base = wbuf_s + st * SM::kStageB;
     const uint32_t vs_base = ks_base + SM::kTileB;
     const int e0 = ((it / kTB) & 1) * kTabE + (it % kTB) * kTile;
 
-    // S = Q K^T over two n-tiles of 8 slots
-    float s[2][4];
+    // S = Q K^T over two n-tiles of 8 slots; the two k-halves of each 32-wide step go
+    // to separate accumulators (two short MMA chains per n-tile instead of one long one)
+    float s[2][4], s2[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+      s2[nt][0] = s2[nt][1] = s2[nt][2] = s2[nt][3] = 0.f;
       const int r = nt * 8 + (lane & 7);
       const int mi = lane >> 3;
 #pragma unroll
@@ -265,7 +297,7 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
         uint32_t b0, b1, b2, b3;
         ldsm_x4(ks_base + r * SM::kRowB + ((c ^ (r & 7)) << 4), b0, b1, b2, b3);
         mma_bf16(s[nt], qa[2 * kk][0], 0u, qa[2 * kk][1], 0u, b0, b1);
-        mma_bf16(s[nt], qa[2 * kk + 1][0], 0u, qa[2 * kk + 1][1], 0u, b2, b3);
+        mma_bf16(s2[nt], qa[2 * kk + 1][0], 0u, qa[2 * kk + 1][1], 0u, b2, b3);
       }
     }
     // log2-domain scores; the bias of a slot past the end is -inf (masked)
@@ -274,15 +306,24 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const float v2 = fmaf(s[nt][e], p.qk_scale2, tbias[e0 + nt * 8 + 2 * qc + e]);
+        const float v2 =
+            fmaf(s[nt][e] + s2[nt][e], p.qk_scale2, tbias[e0 + nt * 8 + 2 * qc + e]);
         s[nt][e] = v2;
         mx = fmaxf(mx, v2);
       }
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     const float m_new = fmaxf(m_run, mx);
-    const float alpha = ex2(m_run - m_new);
-    m_run = m_new;
+    // rescale only when some row's running maximum moved (rare after the first tiles)
+    if (__any_sync(0xffffffffu, m_new != m_run)) {
+      const float alpha = ex2(m_run - m_new);
+      l_run *= alpha;
+#pragma unroll
+      for (int nn = 0; nn < NT; ++nn) {
+        o[nn][0] *= alpha; o[nn][1] *= alpha; o[nn][2] *= alpha; o[nn][3] *= alpha;
+      }
+      m_run = m_new;
+    }
     float psum = 0.f;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
@@ -291,11 +332,7 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
         s[nt][e] = ex2(s[nt][e] - m_new);
         psum += s[nt][e];
       }
-    l_run = fmaf(l_run, alpha, psum);
-#pragma unroll
-    for (int nn = 0; nn < NT; ++nn) {
-      o[nn][0] *= alpha; o[nn][1] *= alpha; o[nn][2] *= alpha; o[nn][3] *= alpha;
-    }
+    l_run += psum;
     // P as bf16 high part (A rows 0-7, the heads) plus bf16 low part (A rows 8-15,
     // otherwise padding): the two accumulator halves sum to P.V with P kept to
     // about 16 mantissa bits, at no extra MMA.
