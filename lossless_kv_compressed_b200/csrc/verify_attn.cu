@@ -14,15 +14,18 @@
 //
 // Per CTA (384 threads):
 //   warp 0      TMA producer: K and V tiles [64 keys x D] (128-byte swizzle) into a
-//               4-stage ring, one mbarrier per stage with the transaction byte count.
-//   warp 1      TMEM allocator and UMMA issuer (one thread): S = Q K^T into TMEM per
-//               M-tile, then O += P V with P from shared memory and V as an N-major B.
+//               6-stage ring, one mbarrier per stage with the transaction byte count.
+//   warp 1      TMEM allocator and UMMA issuer (one thread), both products with the A
+//               operand in TMEM: S = Q K^T (Q in TMEM, K from shared memory), then
+//               O += P V (P in TMEM, V from shared memory as an N-major B).
 //   warps 4-7   softmax of M-tile 0, warps 8-11 of M-tile 1: one thread per query row
-//               (TMEM lane), scores in the log2 domain, running max kept unless it grows
-//               by more than 2^8 (then O in TMEM is rescaled after the previous P.V),
-//               P written as bf16 into a 128-byte-swizzled tile per M-tile (free
-//               again once the previous P.V has retired).
-// TMEM columns: S0 [0,64), S1 [64,128), O0 [128,128+D), O1 [128+D,128+2D).
+//               (TMEM lane); they first store the rows' Q into TMEM.  Scores in the log2
+//               domain, running max kept unless it grows by more than 2^8 (then O in
+//               TMEM is rescaled after the previous P.V), P written back as bf16 over
+//               the first 32 columns of the row's S (the next Q K^T into that S is issued
+//               after this P.V, and UMMAs from one thread run in order).
+// Shared memory then carries only K and V; TMEM columns: O0 [0,D), O1 [D,2D),
+// S0 [2D,2D+64), S1 [2D+64,2D+128), Q0 and Q1 (D/2 columns each) after them.
 // Every mbarrier wait is bounded in time; on expiry the CTA raises the library's device
 // error word, releases TMEM and exits.
 // The split partials (max, sum, unnormalised O) are merged by a second kernel in
@@ -41,7 +44,7 @@ __device__ int g_vc_dev_error;   // bit 0: a bounded wait in the verify kernel e
 constexpr int kSplitKeys = 4096;
 constexpr int kBN = 64;
 constexpr int kVThreads = 384;
-constexpr int kNSt = 4;
+constexpr int kNSt = 6;
 constexpr float kRescaleLog2 = 8.f;
 
 struct VerifyParams {
@@ -56,21 +59,21 @@ struct VerifyParams {
 
 template <int D>
 struct VLayout {
-  static constexpr int kQTile = 128 * D * 2;
   static constexpr int kKVTile = kBN * D * 2;
-  static constexpr int kPTile = 128 * kBN * 2;
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + 2 * kQTile;
+  static constexpr int kK = 0;
   static constexpr int kV = kK + kNSt * kKVTile;
-  static constexpr int kP = kV + kNSt * kKVTile;
-  static constexpr int kBar = kP + 2 * kPTile;
-  static constexpr int kNBar = 2 * kNSt + 2 + 2 + 2 + 2 + 1;
+  static constexpr int kBar = kV + kNSt * kKVTile;
+  static constexpr int kNBar = 2 * kNSt + 2 + 2 + 2 + 1;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kTotal = kAbort + 4;
   static constexpr int kAlloc = kTotal + 1024;
-  static constexpr uint32_t kTmemCols = (128 + 2 * D) <= 256 ? 256 : 512;
-  static_assert(kQTile % 1024 == 0 && kKVTile % 1024 == 0 && kPTile % 1024 == 0, "align");
+  static constexpr uint32_t kColO = 0;
+  static constexpr uint32_t kColS = 2 * D;
+  static constexpr uint32_t kColQ = 2 * D + 2 * kBN;
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(kColQ + D <= kTmemCols, "TMEM columns");
+  static_assert(kKVTile % 1024 == 0, "align");
 };
 
 template <int D>
@@ -112,12 +115,10 @@ __global__ void __launch_bounds__(kVThreads, 1)
   auto b_kv_full = [&](int st) { return bar(st); };
   auto b_kv_empty = [&](int st) { return bar(kNSt + st); };
   auto b_s_full = [&](int mt) { return bar(2 * kNSt + mt); };
-  auto b_s_free = [&](int mt) { return bar(2 * kNSt + 2 + mt); };
-  auto b_p_full = [&](int mt) { return bar(2 * kNSt + 4 + mt); };
-  auto b_o_done = [&](int mt) { return bar(2 * kNSt + 6 + mt); };
-  const uint32_t b_teardown = bar(2 * kNSt + 8);
+  auto b_p_full = [&](int mt) { return bar(2 * kNSt + 2 + mt); };
+  auto b_o_done = [&](int mt) { return bar(2 * kNSt + 4 + mt); };
+  const uint32_t b_teardown = bar(2 * kNSt + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
-
   auto nw_active = [&](int mt) {
     const int v = min(128, rows_here - mt * 128);
     return v > 0 ? (v + 31) >> 5 : 0;
@@ -130,7 +131,6 @@ __global__ void __launch_bounds__(kVThreads, 1)
     }
     for (int mt = 0; mt < 2; ++mt) {
       tc::mbar_init(b_s_full(mt), 1);
-      tc::mbar_init(b_s_free(mt), max(1, nw_active(mt)));
       tc::mbar_init(b_p_full(mt), max(1, nw_active(mt)));
       tc::mbar_init(b_o_done(mt), 1);
     }
@@ -139,28 +139,38 @@ __global__ void __launch_bounds__(kVThreads, 1)
     tc::fence_barrier_init();
   }
   if (warp == 1) tc::tmem_alloc(sb + L::kTmemSlot, L::kTmemCols);
-
-  // Q rows of this group -> shared memory (K-major, 128-byte swizzle); padding rows 0.
-  for (int c = threadIdx.x; c < n_mt * 128 * (D / 8); c += kVThreads) {
-    const int rr = c / (D / 8), ch = c - rr * (D / 8);
-    const int mt = rr >> 7, r = rr & 127;
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (rr < rows_here) {
-      const int grow = row0 + rr;
-      const int i = grow / p.g, hl = grow - i * p.g;
-      const uint4* src = reinterpret_cast<const uint4*>(
-          p.q + (((int64_t)b * p.n_q + i) * p.Hq + kvh * p.g + hl) * D);
-      val = __ldg(src + ch);
-    }
-    const int cb = ch >> 3, cc = ch & 7;
-    *reinterpret_cast<uint4*>(smem + L::kQ + mt * L::kQTile + cb * (128 * 128) + r * 128 +
-                              ((cc ^ (r & 7)) << 4)) = val;
-  }
-  tc::fence_proxy_async();
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlot);
+
+  // Q rows of this group -> TMEM (two bf16 per column; row r of M-tile 0 in lane r, of
+  // M-tile 1 in lane (r + 64) % 128); padding rows are zero.
+  if (warp >= 4) {
+    const int mt = (warp - 4) >> 2, q4 = warp & 3;
+    const int grow = row0 + mt * 128 + ((32 * q4 + lane + (mt ? 64 : 0)) & 127);
+    const bool ok = mt < n_mt && grow < p.R && grow < row0 + rows_here;
+    const uint4* src = nullptr;
+    if (ok) {
+      const int i = grow / p.g, hl = grow - i * p.g;
+      src = reinterpret_cast<const uint4*>(p.q + (((int64_t)b * p.n_q + i) * p.Hq + kvh * p.g + hl) * D);
+    }
+    const uint32_t q_t = tmem + ((uint32_t)(32 * q4) << 16) + L::kColQ + mt * (D / 2);
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      uint32_t w[32];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint4 v = ok ? __ldg(src + 8 * c + u) : make_uint4(0u, 0u, 0u, 0u);
+        w[4 * u] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
+      }
+      tc::tmem_st32(q_t + 32 * c, w);
+    }
+    tc::tmem_wait_st();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
 
   auto raise = [&]() {
     *abort_flag = 1;
@@ -204,19 +214,17 @@ __global__ void __launch_bounds__(kVThreads, 1)
         const int st = t % kNSt;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t a = sb + L::kQ + mt * L::kQTile + (ks >> 2) * (128 * 128) + (ks & 3) * 32;
           const uint32_t bb = sb + L::kK + st * L::kKVTile + (ks >> 2) * (kBN * 128) + (ks & 3) * 32;
-          tc::umma_ss(tmem + mt * kBN, tc::sdesc_sw128(a, 16, 1024), tc::sdesc_sw128(bb, 16, 1024),
-                      id_qk, ks > 0 ? 1u : 0u);
+          tc::umma_ts(tmem + L::kColS + mt * kBN, tmem + L::kColQ + mt * (D / 2) + ks * 8,
+                      tc::sdesc_sw128(bb, 16, 1024), id_qk, ks > 0 ? 1u : 0u);
         }
       };
       auto pv = [&](int t, int mt) {
         const int st = t % kNSt;
 #pragma unroll
         for (int ks = 0; ks < kBN / 16; ++ks) {
-          const uint32_t a = sb + L::kP + mt * L::kPTile + ks * 32;
           const uint32_t bb = sb + L::kV + st * L::kKVTile + ks * 16 * 128;
-          tc::umma_ss(tmem + 128 + mt * D, tc::sdesc_sw128(a, 16, 1024),
+          tc::umma_ts(tmem + L::kColO + mt * D, tmem + L::kColS + mt * kBN + ks * 8,
                       tc::sdesc_sw128(bb, kBN * 128, 1024), id_pv, (t > 0 || ks > 0) ? 1u : 0u);
         }
       };
@@ -234,16 +242,14 @@ __global__ void __launch_bounds__(kVThreads, 1)
                                          abort_flag)))
           break;
         for (int mt = 0; mt < n_mt && ok; ++mt) {
-          if (next) {
-            if (!(ok = tc::mbar_wait(b_s_free(mt), t & 1, abort_flag))) break;
-            tc::tc_fence_after();
-            qk(t + 1, mt);
-            tc::umma_commit(b_s_full(mt));
-          }
           if (!(ok = tc::mbar_wait(b_p_full(mt), t & 1, abort_flag))) break;
           tc::tc_fence_after();
           pv(t, mt);
           tc::umma_commit(b_o_done(mt));
+          if (next) {        // S of this M-tile is free: its P is read by the P.V above
+            qk(t + 1, mt);
+            tc::umma_commit(b_s_full(mt));
+          }
         }
         if (!ok) break;
         tc::umma_commit(b_kv_empty(t % kNSt));
@@ -258,13 +264,17 @@ __global__ void __launch_bounds__(kVThreads, 1)
     // ------------------------------------------------------------ softmax
     const int mt = (warp - 4) >> 2, q4 = warp & 3;
     const int valid_mt = min(128, rows_here - mt * 128);
-    if (mt < n_mt && 32 * q4 < valid_mt) {
-      const int r = 32 * q4 + lane;
+    // M-tile 1 keeps row r in TMEM lane (r + 64) % 128: a part-filled second tile then
+    // lands on the warps of SM sub-partitions 2-3, away from the TMA producer's
+    const int rot = mt ? 64 : 0;
+    if (mt < n_mt && ((32 * q4 + rot) & 127) < valid_mt) {
+      const int r = (32 * q4 + lane + rot) & 127;
       const int grow = row0 + mt * 128 + r;
       const bool row_ok = grow < p.R;
       const int64_t limit = row_ok ? p.P + grow / p.g : (int64_t)-1;
-      const uint32_t s_t = tmem + ((uint32_t)(32 * q4) << 16) + mt * kBN;
-      const uint32_t o_t = tmem + ((uint32_t)(32 * q4) << 16) + 128 + mt * D;
+      const uint32_t lane_t = tmem + ((uint32_t)(32 * q4) << 16);
+      const uint32_t s_t = lane_t + L::kColS + mt * kBN;
+      const uint32_t o_t = lane_t + L::kColO + mt * D;
       float m_used = -INFINITY, lsum = 0.f;
       bool ok = true;
       for (int t = 0; t < n_tiles; ++t) {
@@ -275,27 +285,29 @@ __global__ void __launch_bounds__(kVThreads, 1)
         tc::tmem_ld32(s_t, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
         tc::tmem_ld32(s_t + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tc::tmem_wait_ld();
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(b_s_free(mt));
         // visible columns j in [lo, hi] of this tile for this row (int32, clamped)
         const int64_t key0 = (tile0 + t) * kBN;
         const int lo = (int)max((int64_t)0, min((int64_t)kBN, a0 - key0));
         const int hi = (int)max((int64_t)-1, min((int64_t)(kBN - 1), min(a1 - 1, limit) - key0));
         // Row max on the raw scores (the scale is positive, so it commutes with max);
         // a tile every row of the warp sees whole skips the per-column mask.
-        float mraw = -INFINITY;
+        // (eight independent partial maxima: a short dependency chain)
+        float mx8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
         if (__all_sync(0xffffffffu, lo == 0 && hi == kBN - 1)) {
 #pragma unroll
-          for (int j = 0; j < 64; ++j) mraw = fmaxf(mraw, __uint_as_float(sr[j]));
+          for (int j = 0; j < 64; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(sr[j]));
         } else {
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
             const float v = (j >= lo && j <= hi) ? __uint_as_float(sr[j]) : -INFINITY;
             sr[j] = __float_as_uint(v);
-            mraw = fmaxf(mraw, v);
+            mx8[j & 7] = fmaxf(mx8[j & 7], v);
           }
         }
+        const float mraw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float mx = mraw * p.qk_scale2;
         const float m_new = fmaxf(m_used, mx);
         const bool resc = m_new > m_used + kRescaleLog2;
@@ -318,30 +330,23 @@ __global__ void __launch_bounds__(kVThreads, 1)
         }
         if (resc) m_used = m_new;
         const float m_safe = m_used == -INFINITY ? 0.f : m_used;
-        // the single P tile of this M-tile is free once the previous P.V has retired
-        if (t >= 1) {
-          ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt), (t - 1) & 1, abort_flag));
-          if (!ok) break;
-        }
-        uint8_t* prow = smem + L::kP + mt * L::kPTile + r * 128;
-        float rs = 0.f;
+        // P (bf16, keys packed two per column) over the first 32 columns of this S
+        // row sum in eight independent partial sums, added in a fixed order
+        uint32_t pw[32];
+        float rs8[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float e[8];
+        for (int u = 0; u < 8; ++u) rs8[u] = 0.f;
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            e[u] = ex2(fmaf(__uint_as_float(sr[8 * c + u]), p.qk_scale2, -m_safe));
-            rs += e[u];
-          }
-          uint4 pk;
-          pk.x = pack_bf16x2(e[0], e[1]);
-          pk.y = pack_bf16x2(e[2], e[3]);
-          pk.z = pack_bf16x2(e[4], e[5]);
-          pk.w = pack_bf16x2(e[6], e[7]);
-          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = pk;
+        for (int c = 0; c < 32; ++c) {
+          const float e0 = ex2(fmaf(__uint_as_float(sr[2 * c]), p.qk_scale2, -m_safe));
+          const float e1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), p.qk_scale2, -m_safe));
+          rs8[(2 * c) & 7] += e0;
+          rs8[(2 * c + 1) & 7] += e1;
+          pw[c] = pack_bf16x2(e0, e1);
         }
-        lsum += rs;
-        tc::fence_proxy_async();
+        tc::tmem_st32(s_t, pw);
+        lsum += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        tc::tmem_wait_st();
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(b_p_full(mt));
