@@ -15,17 +15,18 @@
 // Per CTA (384 threads):
 //   warp 0      TMA producer: K and V tiles [64 keys x D] (128-byte swizzle) into a
 //               6-stage ring, one mbarrier per stage with the transaction byte count.
-//   warp 1      TMEM allocator and UMMA issuer (one thread), both products with the A
-//               operand in TMEM: S = Q K^T (Q in TMEM, K from shared memory), then
-//               O += P V (P in TMEM, V from shared memory as an N-major B).
+//   warp 1      TMEM allocator; one thread of warp 1 (M-tile 0) and one of warp 2
+//   warp 2      (M-tile 1) issue the UMMAs: the tile's next S = Q K^T as soon as its
+//               softmax has copied the current S out of TMEM, then O += P V once its
+//               P is in.  Q of M-tile 0 is read from TMEM, Q of M-tile 1 from shared
+//               memory; P from TMEM, K and V from shared memory (V as an N-major B).
 //   warps 4-7   softmax of M-tile 0, warps 8-11 of M-tile 1: one thread per query row
-//               (TMEM lane); they first store the rows' Q into TMEM.  Scores in the log2
+//               (TMEM lane); M-tile 1 keeps row r in lane (r + 64) % 128, so a part-
+//               filled second tile lands on sub-partitions 2-3.  Scores in the log2
 //               domain, running max kept unless it grows by more than 2^8 (then O in
-//               TMEM is rescaled after the previous P.V), P written back as bf16 over
-//               the first 32 columns of the row's S (the next Q K^T into that S is issued
-//               after this P.V, and UMMAs from one thread run in order).
-// Shared memory then carries only K and V; TMEM columns: O0 [0,D), O1 [D,2D),
-// S0 [2D,2D+64), S1 [2D+64,2D+128), Q0 and Q1 (D/2 columns each) after them.
+//               TMEM is rescaled after the previous P.V), P written as bf16 into the
+//               M-tile's P columns once the previous P.V has read them.
+// TMEM columns: O0 [0,D), O1 [D,2D), S0, S1 (64 each), P0, P1 (32 each), Q0 (D/2).
 // Every mbarrier wait is bounded in time; on expiry the CTA raises the library's device
 // error word, releases TMEM and exits.
 // The split partials (max, sum, unnormalised O) are merged by a second kernel in
@@ -59,21 +60,24 @@ struct VerifyParams {
 
 template <int D>
 struct VLayout {
+  static constexpr int kQTile = 128 * D * 2;        // Q of M-tile 1 (128-byte swizzle)
   static constexpr int kKVTile = kBN * D * 2;
-  static constexpr int kK = 0;
+  static constexpr int kQ1 = 0;
+  static constexpr int kK = kQ1 + kQTile;
   static constexpr int kV = kK + kNSt * kKVTile;
   static constexpr int kBar = kV + kNSt * kKVTile;
-  static constexpr int kNBar = 2 * kNSt + 2 + 2 + 2 + 1;
+  static constexpr int kNBar = 2 * kNSt + 2 + 2 + 2 + 2 + 1;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kTotal = kAbort + 4;
   static constexpr int kAlloc = kTotal + 1024;
   static constexpr uint32_t kColO = 0;
   static constexpr uint32_t kColS = 2 * D;
-  static constexpr uint32_t kColQ = 2 * D + 2 * kBN;
+  static constexpr uint32_t kColP = 2 * D + 2 * kBN;
+  static constexpr uint32_t kColQ0 = kColP + 2 * (kBN / 2);
   static constexpr uint32_t kTmemCols = 512;
-  static_assert(kColQ + D <= kTmemCols, "TMEM columns");
-  static_assert(kKVTile % 1024 == 0, "align");
+  static_assert(kColQ0 + D / 2 <= kTmemCols, "TMEM columns");
+  static_assert(kQTile % 1024 == 0 && kKVTile % 1024 == 0, "align");
 };
 
 template <int D>
@@ -115,9 +119,10 @@ __global__ void __launch_bounds__(kVThreads, 1)
   auto b_kv_full = [&](int st) { return bar(st); };
   auto b_kv_empty = [&](int st) { return bar(kNSt + st); };
   auto b_s_full = [&](int mt) { return bar(2 * kNSt + mt); };
-  auto b_p_full = [&](int mt) { return bar(2 * kNSt + 2 + mt); };
-  auto b_o_done = [&](int mt) { return bar(2 * kNSt + 4 + mt); };
-  const uint32_t b_teardown = bar(2 * kNSt + 6);
+  auto b_s_free = [&](int mt) { return bar(2 * kNSt + 2 + mt); };
+  auto b_p_full = [&](int mt) { return bar(2 * kNSt + 4 + mt); };
+  auto b_o_done = [&](int mt) { return bar(2 * kNSt + 6 + mt); };
+  const uint32_t b_teardown = bar(2 * kNSt + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
   auto nw_active = [&](int mt) {
     const int v = min(128, rows_here - mt * 128);
@@ -127,14 +132,15 @@ __global__ void __launch_bounds__(kVThreads, 1)
   if (threadIdx.x == 0) {
     for (int st = 0; st < kNSt; ++st) {
       tc::mbar_init(b_kv_full(st), 1);
-      tc::mbar_init(b_kv_empty(st), 1);
+      tc::mbar_init(b_kv_empty(st), n_mt);      // released by each M-tile's issuer
     }
     for (int mt = 0; mt < 2; ++mt) {
       tc::mbar_init(b_s_full(mt), 1);
+      tc::mbar_init(b_s_free(mt), max(1, nw_active(mt)));
       tc::mbar_init(b_p_full(mt), max(1, nw_active(mt)));
       tc::mbar_init(b_o_done(mt), 1);
     }
-    tc::mbar_init(b_teardown, 1);
+    tc::mbar_init(b_teardown, n_mt);
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -144,29 +150,42 @@ __global__ void __launch_bounds__(kVThreads, 1)
   tc::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlot);
 
-  // Q rows of this group -> TMEM (two bf16 per column; row r of M-tile 0 in lane r, of
-  // M-tile 1 in lane (r + 64) % 128); padding rows are zero.
+  // Q rows of this group: M-tile 0 into TMEM (row r in lane r, two bf16 per column), M-tile
+  // 1 into shared memory (K-major, 128-byte swizzle, row r at row (r + 64) % 128);
+  // padding rows are zero.
   if (warp >= 4) {
     const int mt = (warp - 4) >> 2, q4 = warp & 3;
-    const int grow = row0 + mt * 128 + ((32 * q4 + lane + (mt ? 64 : 0)) & 127);
-    const bool ok = mt < n_mt && grow < p.R && grow < row0 + rows_here;
+    const int rl = 32 * q4 + lane;                       // TMEM lane / UMMA row
+    const int grow = row0 + mt * 128 + ((rl + (mt ? 64 : 0)) & 127);
+    const bool ok = mt < n_mt && grow < row0 + rows_here;
     const uint4* src = nullptr;
     if (ok) {
       const int i = grow / p.g, hl = grow - i * p.g;
       src = reinterpret_cast<const uint4*>(p.q + (((int64_t)b * p.n_q + i) * p.Hq + kvh * p.g + hl) * D);
     }
-    const uint32_t q_t = tmem + ((uint32_t)(32 * q4) << 16) + L::kColQ + mt * (D / 2);
+    if (mt == 0) {
+      const uint32_t q_t = tmem + ((uint32_t)(32 * q4) << 16) + L::kColQ0;
 #pragma unroll
-    for (int c = 0; c < D / 64; ++c) {
-      uint32_t w[32];
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t w[32];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint4 v = ok ? __ldg(src + 8 * c + u) : make_uint4(0u, 0u, 0u, 0u);
-        w[4 * u] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
+        for (int u = 0; u < 8; ++u) {
+          const uint4 v = ok ? __ldg(src + 8 * c + u) : make_uint4(0u, 0u, 0u, 0u);
+          w[4 * u] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
+        }
+        tc::tmem_st32(q_t + 32 * c, w);
       }
-      tc::tmem_st32(q_t + 32 * c, w);
+      tc::tmem_wait_st();
+    } else {
+#pragma unroll
+      for (int ch = 0; ch < D / 8; ++ch) {
+        const uint4 v = ok ? __ldg(src + ch) : make_uint4(0u, 0u, 0u, 0u);
+        const int cb = ch >> 3, cc = ch & 7;
+        *reinterpret_cast<uint4*>(smem + L::kQ1 + cb * (128 * 128) + rl * 128 +
+                                  ((cc ^ (rl & 7)) << 4)) = v;
+      }
+      tc::fence_proxy_async();
     }
-    tc::tmem_wait_st();
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -205,54 +224,60 @@ __global__ void __launch_bounds__(kVThreads, 1)
       for (int t = max(0, issued - kNSt); t < issued; ++t)
         tc::mbar_wait(b_kv_full(t % kNSt), (t / kNSt) & 1, nullptr, 1000000000ull);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ UMMA issuer
-    if (lane == 0) {
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ UMMA issuers
+    // One thread per M-tile (warp 1: M-tile 0, warp 2: M-tile 1), so neither tile's
+    // products wait behind the other tile's softmax.
+    const int mt = warp - 1;
+    if (lane == 0 && mt < n_mt) {
       const uint32_t id_qk = tc::idesc_bf16_f32(128, kBN, false);
       const uint32_t id_pv = tc::idesc_bf16_f32(128, D, true);
-      auto qk = [&](int t, int mt) {
+      auto qk = [&](int t) {
         const int st = t % kNSt;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t bb = sb + L::kK + st * L::kKVTile + (ks >> 2) * (kBN * 128) + (ks & 3) * 32;
-          tc::umma_ts(tmem + L::kColS + mt * kBN, tmem + L::kColQ + mt * (D / 2) + ks * 8,
-                      tc::sdesc_sw128(bb, 16, 1024), id_qk, ks > 0 ? 1u : 0u);
+          const uint64_t bdesc = tc::sdesc_sw128(bb, 16, 1024);
+          if (mt == 0) {
+            tc::umma_ts(tmem + L::kColS, tmem + L::kColQ0 + ks * 8, bdesc, id_qk, ks > 0 ? 1u : 0u);
+          } else {
+            const uint32_t a = sb + L::kQ1 + (ks >> 2) * (128 * 128) + (ks & 3) * 32;
+            tc::umma_ss(tmem + L::kColS + kBN, tc::sdesc_sw128(a, 16, 1024), bdesc, id_qk,
+                        ks > 0 ? 1u : 0u);
+          }
         }
       };
-      auto pv = [&](int t, int mt) {
+      auto pv = [&](int t) {
         const int st = t % kNSt;
 #pragma unroll
         for (int ks = 0; ks < kBN / 16; ++ks) {
           const uint32_t bb = sb + L::kV + st * L::kKVTile + ks * 16 * 128;
-          tc::umma_ts(tmem + L::kColO + mt * D, tmem + L::kColS + mt * kBN + ks * 8,
+          tc::umma_ts(tmem + L::kColO + mt * D, tmem + L::kColP + mt * (kBN / 2) + ks * 8,
                       tc::sdesc_sw128(bb, kBN * 128, 1024), id_pv, (t > 0 || ks > 0) ? 1u : 0u);
         }
       };
       bool ok = tc::mbar_wait(b_kv_full(0), 0, abort_flag);
       if (ok) {
         tc::tc_fence_after();
-        for (int mt = 0; mt < n_mt; ++mt) {
-          qk(0, mt);
-          tc::umma_commit(b_s_full(mt));
-        }
+        qk(0);
+        tc::umma_commit(b_s_full(mt));
       }
       for (int t = 0; ok && t < n_tiles; ++t) {
-        const bool next = t + 1 < n_tiles;
-        if (next && !(ok = tc::mbar_wait(b_kv_full((t + 1) % kNSt), ((t + 1) / kNSt) & 1,
-                                         abort_flag)))
-          break;
-        for (int mt = 0; mt < n_mt && ok; ++mt) {
-          if (!(ok = tc::mbar_wait(b_p_full(mt), t & 1, abort_flag))) break;
+        if (t + 1 < n_tiles) {
+          // the next Q K^T as soon as the softmax has copied this S out of TMEM
+          if (!(ok = tc::mbar_wait(b_kv_full((t + 1) % kNSt), ((t + 1) / kNSt) & 1,
+                                   abort_flag)))
+            break;
+          if (!(ok = tc::mbar_wait(b_s_free(mt), t & 1, abort_flag))) break;
           tc::tc_fence_after();
-          pv(t, mt);
-          tc::umma_commit(b_o_done(mt));
-          if (next) {        // S of this M-tile is free: its P is read by the P.V above
-            qk(t + 1, mt);
-            tc::umma_commit(b_s_full(mt));
-          }
+          qk(t + 1);
+          tc::umma_commit(b_s_full(mt));
         }
-        if (!ok) break;
-        tc::umma_commit(b_kv_empty(t % kNSt));
+        if (!(ok = tc::mbar_wait(b_p_full(mt), t & 1, abort_flag))) break;
+        tc::tc_fence_after();
+        pv(t);
+        tc::umma_commit(b_o_done(mt));
+        tc::umma_commit(b_kv_empty(t % kNSt));   // one arrival per M-tile
       }
       if (!ok) raise();
       // every UMMA issued must retire before TMEM is released
@@ -264,16 +289,15 @@ __global__ void __launch_bounds__(kVThreads, 1)
     // ------------------------------------------------------------ softmax
     const int mt = (warp - 4) >> 2, q4 = warp & 3;
     const int valid_mt = min(128, rows_here - mt * 128);
-    // M-tile 1 keeps row r in TMEM lane (r + 64) % 128: a part-filled second tile then
-    // lands on the warps of SM sub-partitions 2-3, away from the TMA producer's
     const int rot = mt ? 64 : 0;
     if (mt < n_mt && ((32 * q4 + rot) & 127) < valid_mt) {
       const int r = (32 * q4 + lane + rot) & 127;
       const int grow = row0 + mt * 128 + r;
-      const bool row_ok = grow < p.R;
-      const int64_t limit = row_ok ? p.P + grow / p.g : (int64_t)-1;
+      const bool row_ok = r < valid_mt;
+      const int64_t limit = p.P + grow / p.g;
       const uint32_t lane_t = tmem + ((uint32_t)(32 * q4) << 16);
       const uint32_t s_t = lane_t + L::kColS + mt * kBN;
+      const uint32_t p_t = lane_t + L::kColP + mt * (kBN / 2);
       const uint32_t o_t = lane_t + L::kColO + mt * D;
       float m_used = -INFINITY, lsum = 0.f;
       bool ok = true;
@@ -285,10 +309,17 @@ __global__ void __launch_bounds__(kVThreads, 1)
         tc::tmem_ld32(s_t, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
         tc::tmem_ld32(s_t + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tc::tmem_wait_ld();
-        // visible columns j in [lo, hi] of this tile for this row (int32, clamped)
+        // S is in registers: the next Q K^T may overwrite it
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(b_s_free(mt));
+        // visible columns j in [lo, hi] of this tile for this row (int32, clamped); a
+        // padding row counts as seeing the whole tile (its values are never used)
         const int64_t key0 = (tile0 + t) * kBN;
-        const int lo = (int)max((int64_t)0, min((int64_t)kBN, a0 - key0));
-        const int hi = (int)max((int64_t)-1, min((int64_t)(kBN - 1), min(a1 - 1, limit) - key0));
+        const int lo = row_ok ? (int)max((int64_t)0, min((int64_t)kBN, a0 - key0)) : 0;
+        const int hi = row_ok
+            ? (int)max((int64_t)-1, min((int64_t)(kBN - 1), min(a1 - 1, limit) - key0))
+            : kBN - 1;
         // Row max on the raw scores (the scale is positive, so it commutes with max);
         // a tile every row of the warp sees whole skips the per-column mask.
         // (eight independent partial maxima: a short dependency chain)
@@ -311,10 +342,13 @@ __global__ void __launch_bounds__(kVThreads, 1)
         const float mx = mraw * p.qk_scale2;
         const float m_new = fmaxf(m_used, mx);
         const bool resc = m_new > m_used + kRescaleLog2;
-        if (t > 0 && __any_sync(0xffffffffu, resc)) {
+        // the previous P.V must be done before O is rescaled or P overwritten
+        if (t > 0) {
           ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt), (t - 1) & 1, abort_flag));
           if (!ok) break;
           tc::tc_fence_after();
+        }
+        if (t > 0 && __any_sync(0xffffffffu, resc)) {
           const float alpha = resc ? ex2(m_used - m_new) : 1.f;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -330,8 +364,8 @@ __global__ void __launch_bounds__(kVThreads, 1)
         }
         if (resc) m_used = m_new;
         const float m_safe = m_used == -INFINITY ? 0.f : m_used;
-        // P (bf16, keys packed two per column) over the first 32 columns of this S
-        // row sum in eight independent partial sums, added in a fixed order
+        // P (bf16, keys packed two per column); row sum in eight partial sums added in a
+        // fixed order
         uint32_t pw[32];
         float rs8[8];
 #pragma unroll
@@ -344,7 +378,7 @@ __global__ void __launch_bounds__(kVThreads, 1)
           rs8[(2 * c + 1) & 7] += e1;
           pw[c] = pack_bf16x2(e0, e1);
         }
-        tc::tmem_st32(s_t, pw);
+        tc::tmem_st32(p_t, pw);
         lsum += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
         tc::tmem_wait_st();
         tc::tc_fence_before();
