@@ -342,30 +342,12 @@ __global__ void __launch_bounds__(kVThreads, 1)
         const float mx = mraw * p.qk_scale2;
         const float m_new = fmaxf(m_used, mx);
         const bool resc = m_new > m_used + kRescaleLog2;
-        // the previous P.V must be done before O is rescaled or P overwritten
-        if (t > 0) {
-          ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt), (t - 1) & 1, abort_flag));
-          if (!ok) break;
-          tc::tc_fence_after();
-        }
-        if (t > 0 && __any_sync(0xffffffffu, resc)) {
-          const float alpha = resc ? ex2(m_used - m_new) : 1.f;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tc::tmem_ld32(o_t + 32 * c, o);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tc::tmem_st32(o_t + 32 * c, o);
-          }
-          tc::tmem_wait_st();
-          lsum *= alpha;
-        }
+        const float alpha = resc ? ex2(m_used - m_new) : 1.f;
         if (resc) m_used = m_new;
         const float m_safe = m_used == -INFINITY ? 0.f : m_used;
-        // P (bf16, keys packed two per column); row sum in eight partial sums added in a
-        // fixed order
+        // P (bf16, keys packed two per column) in registers first -- it does not depend on
+        // O -- so the exponentials overlap the previous P.V; row sum in eight partial sums
+        // added in a fixed order
         uint32_t pw[32];
         float rs8[8];
 #pragma unroll
@@ -378,6 +360,25 @@ __global__ void __launch_bounds__(kVThreads, 1)
           rs8[(2 * c + 1) & 7] += e1;
           pw[c] = pack_bf16x2(e0, e1);
         }
+        // the previous P.V must be done before O is rescaled or P overwritten
+        if (t > 0) {
+          ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt), (t - 1) & 1, abort_flag));
+          if (!ok) break;
+          tc::tc_fence_after();
+        }
+        if (t > 0 && __any_sync(0xffffffffu, resc)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tc::tmem_ld32(o_t + 32 * c, o);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tc::tmem_st32(o_t + 32 * c, o);
+          }
+          tc::tmem_wait_st();
+        }
+        lsum *= alpha;
         tc::tmem_st32(p_t, pw);
         lsum += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
         tc::tmem_wait_st();
