@@ -52,6 +52,8 @@ template <int THREADS, int CL, int U>
 __global__ void __launch_bounds__(THREADS) argmax_rows_kernel(const float* __restrict__ logits,
                                                               int V, int32_t* __restrict__ target,
                                                               RowEpilogue ep) {
+  pdl_wait();
+  pdl_trigger();
   namespace cg = cooperative_groups;
   const int64_t row = blockIdx.x / CL;
   const int crank = (int)(blockIdx.x % CL);
@@ -79,10 +81,15 @@ __global__ void __launch_bounds__(THREADS) argmax_rows_kernel(const float* __res
         const int i = base + u * THREADS;
         f[u] = i < hi4 ? __ldcs(x4 + i) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
       }
+      // A thread meets its indices in increasing order, so an equal value never
+      // replaces its best: only a group holding a NaN or a strictly larger value
+      // needs the per-element pass (fmaxf ignores NaN; out-of-range lanes are -inf).
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int i = base + u * THREADS;
-        if (i < hi4) {
+        const float m4 = fmaxf(fmaxf(f[u].x, f[u].y), fmaxf(f[u].z, f[u].w));
+        const bool nan4 = isnan(f[u].x) | isnan(f[u].y) | isnan(f[u].z) | isnan(f[u].w);
+        if (nan4 | (m4 > best.val)) {
           take(f[u].x, 4 * i);
           take(f[u].y, 4 * i + 1);
           take(f[u].z, 4 * i + 2);
@@ -173,6 +180,8 @@ __global__ void accept_kernel(int n_q, const int32_t* __restrict__ drafts,
                               int32_t* __restrict__ target, int32_t* __restrict__ accept_len,
                               int32_t* __restrict__ commit, int32_t* __restrict__ n_commit,
                               int32_t* __restrict__ err_flag) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x;
   const int lane = threadIdx.x;
   int32_t* tg = target + (int64_t)b * n_q;
@@ -210,24 +219,8 @@ constexpr int kArgUnroll = 8;
 template <int CL>
 vc_status launch_argmax(const float* logits, int V, int rows, int32_t* target,
                         const RowEpilogue& ep, cudaStream_t stream) {
-  if constexpr (CL == 1) {
-    argmax_rows_kernel<kArgThreads, 1, kArgUnroll><<<rows, kArgThreads, 0, stream>>>(
-        logits, V, target, ep);
-  } else {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(rows * CL);
-    cfg.blockDim = dim3(kArgThreads);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CL;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    VC_CUDA(cudaLaunchKernelEx(&cfg, argmax_rows_kernel<kArgThreads, CL, kArgUnroll>, logits,
-                               V, target, ep));
-  }
+  VC_CUDA(launch_pdl(argmax_rows_kernel<kArgThreads, CL, kArgUnroll>, dim3(rows * CL),
+                     dim3(kArgThreads), 0, stream, CL, logits, V, target, ep));
   VC_CUDA(cudaGetLastError());
   return VC_OK;
 }
@@ -255,8 +248,8 @@ vc_status launch_accept(const float* logits, const int32_t* drafts, int B, int n
     default: st = launch_argmax<8>(logits, V, rows, target, ep, stream); break;
   }
   if (st != VC_OK || n_q == 1) return st;
-  accept_kernel<<<B, 32, 0, stream>>>(n_q, drafts, target, accept_len, commit, n_commit,
-                                      err_flag);
+  VC_CUDA(launch_pdl(accept_kernel, dim3(B), dim3(32), 0, stream, 1, n_q, drafts, target,
+                     accept_len, commit, n_commit, err_flag));
   VC_CUDA(cudaGetLastError());
   return VC_OK;
 }

@@ -74,6 +74,8 @@ struct DraftSmem {
 
 template <int D, int NST>
 __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexedParams p) {
+  pdl_wait();
+  pdl_trigger();
   using SM = DraftSmem<D>;
   constexpr int CH = D / 8;                 // 16-byte chunks per row
   constexpr int NT = D / 8;                 // n-tiles of the output
@@ -424,6 +426,8 @@ __device__ __forceinline__ void split_f16(float a, float b, uint32_t& hi, uint32
 
 template <int D, int NST>
 __global__ void __launch_bounds__(128, 2) draft_int4_kernel(const DraftInt4Params p) {
+  pdl_wait();
+  pdl_trigger();
   using SM = Int4Smem<D>;
   constexpr int NT = D / 8;
   constexpr int NW = D / 32;                 // K words per (token, c); channel groups of V
@@ -680,6 +684,8 @@ template <int D, typename OutT>
 __global__ void __launch_bounds__(kCombWarps * 32) draft_combine_kernel(
     PartialSet a, PartialSet b, int nsets, int g, int Hkv, int Hq, OutT* __restrict__ out,
     float* __restrict__ lse) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int DPL = D / 32;                 // output channels per lane
   __shared__ float s_o[kCombWarps][D];
   __shared__ float s_m[kCombWarps], s_l[kCombWarps];
@@ -820,11 +826,11 @@ vc_status launch_combine(const PartialSet& a, const PartialSet& b, int nsets, in
   const int blocks = pairs * g;
   constexpr int T = kCombWarps * 32;
   if (flags & VC_OUT_F32)
-    draft_combine_kernel<D, float><<<blocks, T, 0, stream>>>(a, b, nsets, g, Hkv, Hq,
-                                                             static_cast<float*>(out), lse);
+    VC_CUDA(launch_pdl(draft_combine_kernel<D, float>, dim3(blocks), dim3(T), 0, stream, 1, a, b,
+                       nsets, g, Hkv, Hq, static_cast<float*>(out), lse));
   else
-    draft_combine_kernel<D, __nv_bfloat16><<<blocks, T, 0, stream>>>(
-        a, b, nsets, g, Hkv, Hq, static_cast<__nv_bfloat16*>(out), lse);
+    VC_CUDA(launch_pdl(draft_combine_kernel<D, __nv_bfloat16>, dim3(blocks), dim3(T), 0, stream,
+                       1, a, b, nsets, g, Hkv, Hq, static_cast<__nv_bfloat16*>(out), lse));
   VC_CUDA(cudaGetLastError());
   return VC_OK;
 }
@@ -865,7 +871,8 @@ vc_status run_indexed(const DraftIndexedParams& p, cudaStream_t stream) {
   const size_t sm = draft_indexed_smem<D>();
   VC_CUDA(cudaFuncSetAttribute(draft_indexed_kernel<D, kNStage>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-  draft_indexed_kernel<D, kNStage><<<p.W / kDraftWarps, 128, sm, stream>>>(p);
+  VC_CUDA(launch_pdl(draft_indexed_kernel<D, kNStage>, dim3(p.W / kDraftWarps), dim3(128), sm,
+                     stream, 1, p));
   VC_CUDA(cudaGetLastError());
   return VC_OK;
 }
@@ -875,7 +882,8 @@ vc_status run_int4(const DraftInt4Params& p, cudaStream_t stream) {
   const size_t sm = draft_int4_smem<D>();
   VC_CUDA(cudaFuncSetAttribute(draft_int4_kernel<D, kNStageInt4>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-  draft_int4_kernel<D, kNStageInt4><<<p.W / kDraftWarps, 128, sm, stream>>>(p);
+  VC_CUDA(launch_pdl(draft_int4_kernel<D, kNStageInt4>, dim3(p.W / kDraftWarps), dim3(128), sm,
+                     stream, 1, p));
   VC_CUDA(cudaGetLastError());
   return VC_OK;
 }

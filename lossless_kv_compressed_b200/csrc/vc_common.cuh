@@ -91,4 +91,41 @@ __device__ __forceinline__ float warp_max_xor(float v, int mask_bits) {
   return v;
 }
 
+// Programmatic dependent launch.  Every hot-path kernel starts with pdl_wait(): it returns
+// once the kernel launched before it on the stream has completed and its writes are
+// visible (at once when there is no such dependency), so nothing a kernel reads or
+// writes can overlap its predecessor.  pdl_trigger() then lets the next kernel be
+// launched and its blocks placed while this one still runs; they wait in their own
+// pdl_wait().  Only the launch latency between kernels is hidden.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch with programmatic stream serialization (and a 1-D cluster when cluster > 1).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, int cluster, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = (unsigned)cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 }  // namespace vc

@@ -84,6 +84,8 @@ template <int D>
 __global__ void __launch_bounds__(kVThreads, 1)
     verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const VerifyParams p) {
+  pdl_wait();
+  pdl_trigger();
   using L = VLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -437,6 +439,8 @@ __global__ void __launch_bounds__(kVCombWarps * 32) verify_combine_kernel(
     const float* __restrict__ ws_o, const float* __restrict__ ws_ml, int n_split, int R, int g,
     int n_q, int Hq, int Hkv, int flags, float* m_state, float* l_state, float* acc_state,
     OutT* __restrict__ out, int rows) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int DPL = D / 32;
   constexpr int CH = 8;
   const int lane = threadIdx.x & 31;
@@ -576,18 +580,20 @@ static vc_status run_verify(const Plan& pl, const VerifyParams& vp, const CUtens
   VC_CUDA(cudaFuncSetAttribute(verify_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                L::kAlloc));
   dim3 grid(pl.n_split, pl.n_rg, pl.pairs);
-  verify_kernel<D><<<grid, kVThreads, L::kAlloc, stream>>>(mk, mv, vp);
+  VC_CUDA(launch_pdl(verify_kernel<D>, grid, dim3(kVThreads), L::kAlloc, stream, 1, mk, mv, vp));
   VC_CUDA(cudaGetLastError());
   const int rows = pl.pairs * pl.R;
   const int cblocks = (rows + kVCombWarps - 1) / kVCombWarps;
   if (flags & VC_OUT_F32)
-    verify_combine_kernel<D, float><<<cblocks, kVCombWarps * 32, 0, stream>>>(
-        vp.ws_o, vp.ws_ml, pl.n_split, pl.R, pl.g, vp.n_q, vp.Hq, vp.Hkv, flags, m, l, acc,
-        static_cast<float*>(out), rows);
+    VC_CUDA(launch_pdl(verify_combine_kernel<D, float>, dim3(cblocks), dim3(kVCombWarps * 32), 0,
+                       stream, 1, (const float*)vp.ws_o, (const float*)vp.ws_ml, pl.n_split, pl.R,
+                       pl.g, vp.n_q, vp.Hq, vp.Hkv, flags, m, l, acc, static_cast<float*>(out),
+                       rows));
   else
-    verify_combine_kernel<D, __nv_bfloat16><<<cblocks, kVCombWarps * 32, 0, stream>>>(
-        vp.ws_o, vp.ws_ml, pl.n_split, pl.R, pl.g, vp.n_q, vp.Hq, vp.Hkv, flags, m, l, acc,
-        static_cast<__nv_bfloat16*>(out), rows);
+    VC_CUDA(launch_pdl(verify_combine_kernel<D, __nv_bfloat16>, dim3(cblocks),
+                       dim3(kVCombWarps * 32), 0, stream, 1, (const float*)vp.ws_o,
+                       (const float*)vp.ws_ml, pl.n_split, pl.R, pl.g, vp.n_q, vp.Hq, vp.Hkv,
+                       flags, m, l, acc, static_cast<__nv_bfloat16*>(out), rows));
   VC_CUDA(cudaGetLastError());
   return VC_OK;
 }
