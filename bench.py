@@ -591,6 +591,161 @@ def run_config5(args) -> int:
     return 0
 
 
+def run_table(args) -> int:
+    """Per-kernel rates at every workload's shapes (one JSON line per row): draft calls
+    (bytes / time, % of HBM), verify calls (useful flops / time, % of the tensor peak and of
+    the attainable min(tensor, I x HBM)), acceptance calls, and the oracle on bounded
+    samples (all host threads and one thread).  Device inputs are seeded random tensors
+    of each workload's shapes (the rates do not depend on the values); each call is timed
+    with CUDA events, median of 20 after 5 warm-ups, the L2 flushed before each."""
+    import torch
+    import lossless_kv_compressed_b200 as vc
+    from synth.configs import get_config
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(2024)
+    peaks = measured_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn, reps=20, warm=5):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e-3)
+        return statistics.median(ts)
+
+    bf = lambda *shape: torch.randn(*shape, device=dev, generator=g).to(torch.bfloat16)
+    emit = lambda d: print(json.dumps(d), flush=True)
+
+    def draft_row(cfg_n, cache, q, nbytes, note):
+        ws = torch.empty(vc.draft_workspace_size(cache), dtype=torch.uint8, device=dev)
+        out = torch.empty_like(q)
+        t = timed(lambda: vc.draft_attn(q, cache, out=out, ws=ws))
+        emit({"table": "draft", "workload": cfg_n, "us": t * 1e6, "bytes": nbytes,
+              "GB/s": nbytes / t / 1e9, "frac_hbm": nbytes / t / 1e9 / peaks["hbm_gbs"],
+              "note": note})
+
+    def verify_row(cfg_n, B, Hq, Hkv, D, P, n_q, k_all, v_all, note):
+        q = bf(B, n_q, Hq, D)
+        out = torch.empty_like(q)
+        ws = torch.empty(vc.verify_workspace_size(B, n_q, Hq, Hkv, D, 0, P + n_q),
+                         dtype=torch.uint8, device=dev)
+        t = timed(lambda: vc.verify_attn(q, k_all, v_all, P, out=out, ws=ws))
+        flops = 4 * D * (Hq // Hkv) * sum(P + i + 1 for i in range(n_q)) * B * Hkv
+        nbytes = B * Hkv * (P + n_q) * D * 4 + 2 * B * n_q * Hq * D * 2
+        attain = min(peaks["bf16_tflops"], flops / nbytes * peaks["hbm_gbs"] / 1e3)
+        tf = flops / t / 1e12
+        emit({"table": "verify", "workload": cfg_n, "us": t * 1e6, "GFLOP": flops / 1e9,
+              "bytes": nbytes, "TFLOP/s": tf, "frac_tensor": tf / peaks["bf16_tflops"],
+              "frac_attainable": tf / attain, "GB/s": nbytes / t / 1e9, "note": note})
+
+    # ---- workload 1: B1, 8/2 heads, D 64, 256 slots of 1024 + 8 tail rows; verify k = 8
+    c = get_config(1)
+    T = c.L_cap
+    k1, v1 = bf(c.B, c.Hkv, T, c.D), bf(c.B, c.Hkv, T, c.D)
+    idx = torch.stack([torch.sort(torch.randperm(c.P, device=dev, generator=g)[:c.S])[0]
+                       for _ in range(c.B * c.Hkv)]).view(c.B, c.Hkv, c.S).int()
+    deg = torch.randint(1, 9, (c.B, c.Hkv, c.S), device=dev, generator=g, dtype=torch.int32)
+    cache = vc.IndexedCache(k=k1, v=v1, S=c.S, Hq=c.Hq, idx=idx, deg=deg,
+                            k_tail=bf(c.B, c.Hkv, c.k, c.D), v_tail=bf(c.B, c.Hkv, c.k, c.D),
+                            n_tail=c.k)
+    draft_row(1, cache, bf(c.B, c.Hq, c.D), draft_bytes(c, c.k), "L2-resident: report us")
+    verify_row(1, c.B, c.Hq, c.Hkv, c.D, c.P, c.k + 1, k1, v1, "latency-bound")
+    # ---- workload 2
+    c = get_config(2)
+    k2, v2 = bf(c.B, c.Hkv, c.L_cap, c.D), bf(c.B, c.Hkv, c.L_cap, c.D)
+    idx = torch.stack([torch.sort(torch.randperm(c.P, device=dev, generator=g)[:c.S])[0]
+                       for _ in range(c.B * c.Hkv)]).view(c.B, c.Hkv, c.S).int()
+    deg = torch.randint(1, 17, (c.B, c.Hkv, c.S), device=dev, generator=g, dtype=torch.int32)
+    cache = vc.IndexedCache(k=k2, v=v2, S=c.S, Hq=c.Hq, idx=idx, deg=deg,
+                            k_tail=bf(c.B, c.Hkv, c.k, c.D), v_tail=bf(c.B, c.Hkv, c.k, c.D),
+                            n_tail=c.k)
+    draft_row(2, cache, bf(c.B, c.Hq, c.D), draft_bytes(c, c.k), "indexed, 32 tail rows")
+    verify_row(2, c.B, c.Hq, c.Hkv, c.D, c.P, c.k + 1, k2, v2, "k = 32")
+    del k2, v2, cache
+    # ---- workload 3: int4 cache of 130944 tokens + 128 bf16 tail rows; verify over bf16
+    c = get_config(3)
+    nb = (c.P - c.tail_bf16) // 32
+    pairs = (c.B, c.Hkv, nb)
+    ri = lambda *shape: torch.randint(-2 ** 31, 2 ** 31 - 1, shape, device=dev, generator=g,
+                                      dtype=torch.int64).to(torch.int32)
+    f16 = lambda lo, hi, *shape: (torch.rand(*shape, device=dev, generator=g) * (hi - lo) +
+                                   lo).half()
+    cache = vc.Int4Cache(kq=ri(*pairs, 32, 4, c.D // 32), k_scale=f16(0.01, 0.1, *pairs, c.D),
+                         k_zero=f16(-1, 1, *pairs, c.D), vq=ri(*pairs, c.D, 4),
+                         v_scale=f16(0.01, 0.1, *pairs, c.D // 32, 32),
+                         v_zero=f16(-1, 1, *pairs, c.D // 32, 32), S=nb * 32, Hq=c.Hq,
+                         k_tail=bf(c.B, c.Hkv, c.tail_bf16, c.D),
+                         v_tail=bf(c.B, c.Hkv, c.tail_bf16, c.D), n_tail=c.tail_bf16)
+    nbytes = c.B * c.Hkv * (nb * 32 * (c.D + c.D * 2 * 2 * 2 // 32) +
+                            c.tail_bf16 * c.D * 4) + 2 * c.B * c.Hq * c.D * 2
+    draft_row(3, cache, bf(c.B, c.Hq, c.D), nbytes,
+              "int4: 160 B per token at D 128 (random packed words and scales)")
+    del cache
+    k3, v3 = bf(c.B, c.Hkv, c.L_cap, c.D), bf(c.B, c.Hkv, c.L_cap, c.D)
+    verify_row(3, c.B, c.Hq, c.Hkv, c.D, c.P, c.k + 1, k3, v3, "k = 32, 128K context")
+    del k3, v3
+    # ---- workload 4: compact 65536-slot caches for 3 requests; verify over a device-resident
+    #      1M-token context (the staged form is bench.py --config 4)
+    c = get_config(4)
+    nd = c.n_draft_requests
+    kc, vcc = bf(nd, c.Hkv, c.S, c.D), bf(nd, c.Hkv, c.S, c.D)
+    deg = torch.randint(1, 17, (nd, c.Hkv, c.S), device=dev, generator=g, dtype=torch.int32)
+    cache = vc.IndexedCache(k=kc, v=vcc, S=c.S, Hq=c.Hq, deg=deg)
+    nbytes = nd * c.Hkv * c.S * (c.D * 4 + 4) + 2 * nd * c.Hq * c.D * 2
+    draft_row(4, cache, bf(nd, c.Hq, c.D), nbytes, "compact caches (no index)")
+    del kc, vcc, cache
+    k4, v4 = bf(1, c.Hkv, c.P + c.k + 1, c.D), bf(1, c.Hkv, c.P + c.k + 1, c.D)
+    verify_row(4, 1, c.Hq, c.Hkv, c.D, c.P, c.k + 1, k4, v4,
+               "k = 40, 1M-token context resident in HBM (one call)")
+    del k4, v4
+    # ---- acceptance
+    for name, (B, n_q, V) in {"1": (1, 9, 1024), "5": (1, 33, 8192), "2 verify": (8, 33, 128256),
+                              "2 draft step": (8, 1, 128256)}.items():
+        lg = torch.randn(B, n_q, V, device=dev, generator=g)
+        dr = torch.randint(0, V, (B, n_q - 1), device=dev, generator=g, dtype=torch.int32)
+        tgt = torch.empty(B, n_q, dtype=torch.int32, device=dev)
+        err = torch.empty(B, dtype=torch.int32, device=dev)
+        if n_q > 1:
+            al = torch.empty(B, dtype=torch.int32, device=dev)
+            cm = torch.empty(B, n_q, dtype=torch.int32, device=dev)
+            nc = torch.empty(B, dtype=torch.int32, device=dev)
+            fn = lambda: vc.accept(lg, dr, target=tgt, accept_len=al, commit=cm, n_commit=nc,
+                                   err_flag=err)
+        else:
+            fn = lambda: vc.accept(lg, None, target=tgt, err_flag=err)
+        t = timed(fn)
+        emit({"table": "accept", "workload": name, "rows": B * n_q, "vocab": V,
+              "us": t * 1e6, "GB/s": lg.numel() * 4 / t / 1e9})
+    # ---- the oracle on bounded samples, all host threads and one thread
+    if not args.no_cpu_baseline:
+        from threadpoolctl import threadpool_limits
+        from synth import gen
+        case1 = gen.attn_case(1)
+        case2 = gen.attn_case(2)
+        for threads in (None, 1):
+            with threadpool_limits(limits=threads):
+                for name, case in (("1", case1), ("2", case2)):
+                    ts = []
+                    for _ in range(3):
+                        nb_, dt = oracle_pair_sample(case, 0, 0)
+                        ts.append(dt)
+                    dt = statistics.median(ts)
+                    emit({"table": "oracle", "workload": name,
+                          "threads": "all" if threads is None else 1,
+                          "sample": "one (batch, kv head) pair: its k draft calls and verify rows",
+                          "s": dt, "GB/s": nb_ / dt / 1e9})
+    return 0
+
+
 def run_profile_case(kind: str) -> int:
     """A short run of one call of the workload-2 round for an ncu capture: one copy of
     the inputs (about 1.2 GB on the device), five calls of the chosen entry point."""
@@ -636,6 +791,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="vc", choices=["vc", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--table", action="store_true",
+                    help="per-kernel rates at every workload's shapes, one JSON line per row")
     ap.add_argument("--profile-case", choices=["draft", "verify", "accept"], default=None,
                     help="run five calls of one entry point on the workload-2 inputs (one "
                          "copy) for an ncu capture, and print no bench line")
@@ -647,6 +804,8 @@ def main():
         args.warmup = 3
     if args.profile_case:
         return run_profile_case(args.profile_case)
+    if args.table:
+        return run_table(args)
     if args.config == 4 and args.impl == "vc":
         return run_config4(args)
     if args.config == 5 and args.impl == "vc":
