@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
 // subtracted) and the scales move to the other operand, so nothing proportional to a
 // dequantised value is ever rounded to fp16:
 //   q . k_hat = sum_d (q_d s_d) n_d + sum_d q_d z_d              (K: per channel)
-//   sum_t p_t v_hat_t = sum_t (p_t s_t)(n_t - 7.5) + sum_t p_t (z_t + 7.5 s_t)
+//   sum_t p_t v_hat_t = sum_t (p_t s_t / 2)(2 n_t - 15) + sum_t p_t (z_t + 7.5 s_t)
 //                                                                 (V: per token, group;
 //   centred so that neither sum is much larger than the result)
 // q_d s_d and p_t s_t are split into fp16 high and low parts placed in A rows 0-7 and
@@ -408,10 +408,14 @@ __device__ __forceinline__ uint32_t nib_pair(uint32_t w, int j) {
   asm("sub.f16x2 %0, %1, %2;" : "=r"(n) : "r"(x), "r"(0x64006400u));
   return n;
 }
-// Same, centred on the middle of the 4-bit range: (n0 - 7.5, n1 - 7.5), still exact.
-__device__ __forceinline__ uint32_t nib_pair_c(uint32_t w, int j) {
+// Same, centred on the middle of the 4-bit range and doubled: (2 n0 - 15, 2 n1 - 15),
+// exact.  2n + 1 goes into the mantissa of fp16 1024 (the nibble shifted up one bit,
+// the low bit set) and 1040 is subtracted, so one subtraction does both steps.
+__device__ __forceinline__ uint32_t nib_pair_c2(uint32_t w, int j) {
+  const uint32_t sh = j == 0 ? (w << 1) : (w >> (4 * j - 1));
+  const uint32_t x = (sh & 0x001E001Eu) | 0x64016401u;     // 1024 + 2n + 1
   uint32_t c;
-  asm("sub.f16x2 %0, %1, %2;" : "=r"(c) : "r"(nib_pair(w, j)), "r"(0x47804780u));
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(c) : "r"(x), "r"(0x64106410u));   // - 1040
   return c;
 }
 __device__ __forceinline__ float2 h2f(uint32_t h) {
@@ -441,10 +445,15 @@ __global__ void __launch_bounds__(128, 2) draft_int4_kernel(const DraftInt4Param
   const uint32_t wbuf_s = smem_u32(smem + warp * NST * SM::kStageB);
   uint8_t* wbuf = smem + warp * NST * SM::kStageB;
 
+  // Block x0 + i lies in pair (x0 + i) / nblk: carried forward, not divided per block.
+  const int nblk = p.nblk;
+  const int64_t pair_first = x0 / nblk;
+  const int rem_first = (int)(x0 - pair_first * nblk);
+  int64_t is_pair = pair_first;
+  int is_rem = rem_first;
   auto issue = [&](int it, int st) {
-    const int64_t x = x0 + it;
-    const int64_t pair = x / p.nblk;
-    const int64_t blk = pair * p.nblk_cap + (x - pair * p.nblk);
+    const int64_t blk = is_pair * p.nblk_cap + is_rem;
+    if (++is_rem == nblk) { is_rem = 0; ++is_pair; }
     const uint32_t dst = wbuf_s + st * SM::kStageB;
 #pragma unroll
     for (int i = 0; i < (CH + 31) / 32; ++i) {
@@ -480,8 +489,7 @@ __global__ void __launch_bounds__(128, 2) draft_int4_kernel(const DraftInt4Param
       dst[ks][1] = ok ? __ldg(qp + (16 * ks + 8 + 2 * qc) / 2) : 0u;
     }
   };
-  const int64_t pair_first = x0 / p.nblk;
-  const int64_t pair_last = (x0 + n - 1) / p.nblk;
+  const int64_t pair_last = (x0 + n - 1) / nblk;
   load_q(pair_first, qa);
   if (pair_last > pair_first) load_q(pair_first + 1, qn);
 
@@ -526,20 +534,22 @@ __global__ void __launch_bounds__(128, 2) draft_int4_kernel(const DraftInt4Param
     if (st < n) issue(st, st);
     cp_async_commit();
   }
+  int c_rem = rem_first;
   for (int it = 0; it < n; ++it) {
     if (it + NST - 1 < n) issue(it + NST - 1, (it + NST - 1) % NST);
     cp_async_commit();
     cp_async_wait<NST - 1>();
     __syncwarp();
-    const int64_t pair = (x0 + it) / p.nblk;
-    if (pair != cur) {
+    if (c_rem == nblk) {                             // segment boundary
+      c_rem = 0;
       flush(cur);
       reset();
-      cur = pair;
+      ++cur;
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) { qa[ks][0] = qn[ks][0]; qa[ks][1] = qn[ks][1]; }
-      if (pair < pair_last) load_q(pair + 1, qn);
+      if (cur < pair_last) load_q(cur + 1, qn);
     }
+    ++c_rem;
     const uint8_t* sbase = wbuf + (it % NST) * SM::kStageB;
     const uint32_t* kw = reinterpret_cast<const uint32_t*>(sbase);
     const uint32_t* vw = reinterpret_cast<const uint32_t*>(sbase + SM::kKW);
@@ -638,20 +648,23 @@ __global__ void __launch_bounds__(128, 2) draft_int4_kernel(const DraftInt4Param
         mma_f16(zacc, ph[2 * kt], pl[2 * kt], ph[2 * kt + 1], pl[2 * kt + 1], z0, z1);
       }
     }
-    // ---- O += (p s) N per channel group, B = exact nibbles of V
+    // ---- O += (p s / 2) (2N - 15) per channel group, B = exact doubled centred nibbles
+    float sh[4][2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) { sh[j][0] = 0.5f * s[j][0]; sh[j][1] = 0.5f * s[j][1]; }
 #pragma unroll
     for (int G = 0; G < NW; ++G) {
       uint32_t pah[4], pal[4];                      // [kt * 2 + half]
 #pragma unroll
       for (int j = 0; j < 4; ++j) {                 // token pair 2qc + 8j: n-tile j
         const float2 sv = h2f(vsc[(G * 32 + 2 * qc + 8 * j) / 2]);
-        split_f16(s[j][0] * sv.x, s[j][1] * sv.y, pah[j], pal[j]);
+        split_f16(sh[j][0] * sv.x, sh[j][1] * sv.y, pah[j], pal[j]);
       }
 #pragma unroll
       for (int nn = 4 * G; nn < 4 * G + 4; ++nn) {
         const uint32_t wv = vw[(nn * 8 + qr) * 4 + qc];
-        mma_f16(o[nn], pah[0], pal[0], pah[1], pal[1], nib_pair_c(wv, 0), nib_pair_c(wv, 1));
-        mma_f16(o[nn], pah[2], pal[2], pah[3], pal[3], nib_pair_c(wv, 2), nib_pair_c(wv, 3));
+        mma_f16(o[nn], pah[0], pal[0], pah[1], pal[1], nib_pair_c2(wv, 0), nib_pair_c2(wv, 1));
+        mma_f16(o[nn], pah[2], pal[2], pah[3], pal[3], nib_pair_c2(wv, 2), nib_pair_c2(wv, 3));
       }
     }
     __syncwarp();
