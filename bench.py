@@ -540,12 +540,10 @@ def run_config4(args) -> int:
 # ------------------------------------------------------------------ workload 5
 def run_config5(args) -> int:
     """The loop end to end on the tiny decoder: accepted tokens/s of the VeriCache loop
-    and of full-KV greedy decoding on the same GPU, the acceptance-length histogram,
-    and the GPU's greedy stream against the fp64 oracle's on the first tokens."""
+    and of full-KV greedy decoding on the same GPU, and the acceptance-length histogram.
+    (The GPU stream against the fp64 oracle's is a GPU test, not a bench figure.)"""
     import torch
-    import oracle
     from lossless_kv_compressed_b200.loop import GpuTinyLM, greedy_loop, vericache_loop
-    from oracle import tinylm
     from synth import gen
     from synth.configs import get_config
     cfg = get_config(5)
@@ -568,10 +566,6 @@ def run_config5(args) -> int:
                                                      cfg.budget, cfg.n_sinks, cfg.n_recent,
                                                      cfg.score_window))
     hist = np.bincount(np.asarray(alens), minlength=cfg.k + 1).tolist()
-    n_cmp = 16
-    ref = tinylm.greedy_loop(tinylm.TinyLM({k: oracle.bf16_to_f64(v) for k, v in w.items()}, cfg),
-                             prompt, n_cmp)
-    div = next((i for i in range(n_cmp) if ref[i] != greedy[i]), None)
     line = {
         "metric": METRIC, "value": cfg.gen_tokens / tv, "unit": "accepted tokens/s",
         "n_gpus": 1, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
@@ -585,7 +579,7 @@ def run_config5(args) -> int:
         "greedy_tokens_per_s": cfg.gen_tokens / tg,
         "rounds": len(alens), "mean_accept_len": float(np.mean(alens)),
         "accept_len_histogram": hist,
-        "oracle_fp64_agreement": {"tokens_compared": n_cmp, "first_divergence": div},
+        "oracle_fp64": "tests/test_gpu_loop.py::test_workload5_greedy_follows_oracle_to_a_near_tie",
     }
     print(json.dumps(line), flush=True)
     return 0
