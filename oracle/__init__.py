@@ -11,8 +11,9 @@ It is written from two web summaries:
   Arabic translation gist.science/ar/paper/2605.17613): the draft-then-verify
   loop, greedy acceptance with the bonus token, and the staging of the full KV.
 * "Riassunto Tecnico: CentroidKV" (gist.science/it/paper/2506.11418): the per-slot
-  degree n_t entering the softmax as a logarithmic term, and the preservation of
-  attention sinks and recent tokens.
+  degree n_t entering the softmax as a logarithmic term, the preservation of
+  attention sinks and recent tokens, and the Chunked Soft Matching compressor
+  (``oracle.csm``).
 
 The pages print no formula.  Each function states the plain definition it
 implements and the reading taken where the pages are silent.  Everything is
@@ -34,3 +35,4 @@ from .accept import argmax_row, accept  # noqa: F401
 from .quant import (  # noqa: F401
     quantize_k_groups, quantize_v_groups, dequant_k_groups, dequant_v_groups,
 )
+from . import csm  # noqa: F401,E402
