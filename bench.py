@@ -701,6 +701,22 @@ def run_table(args) -> int:
     verify_row(4, 1, c.Hq, c.Hkv, c.D, c.P, c.k + 1, k4, v4,
                "k = 40, 1M-token context resident in HBM (one call)")
     del k4, v4
+    # ---- Chunked Soft Matching, one round over workload 2's full caches (chunk 256,
+    #      r = 0.5): reads K, V and degrees, writes the compact cache
+    c = get_config(2)
+    kc, vcc = bf(c.B, c.Hkv, c.P, c.D), bf(c.B, c.Hkv, c.P, c.D)
+    deg = torch.randint(1, 17, (c.B, c.Hkv, c.P), device=dev, generator=g, dtype=torch.int32)
+    n_out = vc.csm_out_len(c.P, 4, 512, 256, 0.5)
+    ko = torch.empty(c.B, c.Hkv, n_out, c.D, dtype=torch.bfloat16, device=dev)
+    vo, do = torch.empty_like(ko), torch.empty(c.B, c.Hkv, n_out, dtype=torch.int32, device=dev)
+    t = timed(lambda: vc.csm_compress(kc, vcc, 4, 512, 256, 0.5, deg=deg, k_out=ko, v_out=vo,
+                                      deg_out=do))
+    pairs = c.B * c.Hkv
+    nbytes = pairs * (c.P * (c.D * 4 + 4) + n_out * (c.D * 4 + 4))
+    emit({"table": "csm", "workload": 2, "us": t * 1e6, "rows_in": c.P, "rows_out": n_out,
+          "bytes": nbytes, "GB/s": nbytes / t / 1e9,
+          "frac_hbm": nbytes / t / 1e9 / peaks["hbm_gbs"], "note": "chunk 256, r 0.5"})
+    del kc, vcc, ko, vo
     # ---- acceptance
     for name, (B, n_q, V) in {"1": (1, 9, 1024), "5": (1, 33, 8192), "2 verify": (8, 33, 128256),
                               "2 draft step": (8, 1, 128256)}.items():

@@ -225,6 +225,38 @@ vc_status vc_stage_full_kv(void* dst_dev, const void* src_host, size_t bytes,
  * VC_ERR_TIMEOUT after timeout_s seconds, or VC_ERR_CUDA. */
 vc_status vc_event_wait(cudaEvent_t ev, double timeout_s);
 
+/* ----------------------------------------------------------------------------
+ * One round of Chunked Soft Matching: CentroidKV's one-pass clustering of a KV cache
+ * ([CKV] "Riassunto Tecnico: CentroidKV", section "Metodologia", items 2-4).  For each
+ * (batch, kv head) pair, rows [0, n_sinks) and [T - n_recent, T) are kept as they are;
+ * the rows between are cut into consecutive chunks of `chunk` rows (the last may be
+ * shorter).  In a chunk, A = rows at even offsets, B = rows at odd offsets; each A row is
+ * matched to its most similar B row by cosine of the key rows (lowest B row on ties; an
+ * all-zero row has cosine 0 with everything); the m = floor(r * |A|) A rows with the
+ * highest similarity (lower row on ties) merge into their matches.  A B row and the A
+ * rows merged into it become one centroid: K and V = degree-weighted means (fp32 sums,
+ * the B row first, then its A rows in ascending order, rounded to bf16 once), degree =
+ * the sum.  A one-row chunk (no B row) merges nothing.  Output order: sinks, each chunk's surviving rows in their order (a centroid in
+ * its B row's place), recent rows.  The result is a compact cache (idx = NULL, deg =
+ * deg_out) for vc_draft_attn.  A decreasing r over successive rounds (r_j = r_init -
+ * j * delta_r) is the caller's schedule.  Similarities use bf16 products with fp32
+ * accumulation; a near-tie may resolve either way.
+ *
+ *   k, v      bf16 [pairs, T_cap, D] (device), the cache rows [0, T) of each pair
+ *   deg       int32 [pairs, T_cap] degrees >= 1, or NULL (all 1)
+ *   k_out, v_out  bf16 [pairs, T_cap_out, D]; deg_out int32 [pairs, T_cap_out]
+ *             (must not overlap the inputs); rows [0, vc_csm_out_len(...)) are written
+ *   dest      int32 [pairs, T_cap] or NULL: output row of every input row (the
+ *             centroid's row for a merged row)
+ *   D in {64, 128}; 2 <= chunk <= 256; 0 <= r <= 1; n_sinks + n_recent <= T <= T_cap;
+ *   T < 2^31; pairs <= 65535; pointers 16-byte aligned.
+ * ---------------------------------------------------------------------------- */
+int64_t vc_csm_out_len(int64_t T, int n_sinks, int n_recent, int chunk, double r);
+vc_status vc_csm_compress(const void* k, const void* v, const int32_t* deg, int pairs, int D,
+                          int64_t T, int64_t T_cap, int n_sinks, int n_recent, int chunk,
+                          double r, void* k_out, void* v_out, int32_t* deg_out,
+                          int64_t T_cap_out, int32_t* dest, cudaStream_t stream);
+
 /* The library's device error word on the current device (synchronous read; clear != 0
  * resets it).  Bit 0: a bounded wait inside a verify-attention CTA expired (the call's
  * output is then invalid; the CTA released its resources and exited). */

@@ -22,6 +22,7 @@ EXPORTS = (
     "vc_draft_workspace_size", "vc_draft_attn", "vc_draft_attn_noalloc",
     "vc_verify_workspace_size", "vc_verify_attn",
     "vc_accept", "vc_stage_full_kv", "vc_event_wait", "vc_device_error",
+    "vc_csm_out_len", "vc_csm_compress",
 )
 # Model glue of the end-to-end loop (include/vericache_glue.h).
 GLUE_EXPORTS = (
@@ -93,6 +94,13 @@ def lib() -> ctypes.CDLL:
         L.vc_event_wait.argtypes = [_p, ctypes.c_double]
         L.vc_device_error.restype = ctypes.c_int
         L.vc_device_error.argtypes = [ctypes.POINTER(_i32), ctypes.c_int]
+        L.vc_csm_out_len.restype = _i64
+        L.vc_csm_out_len.argtypes = [_i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_double]
+        L.vc_csm_compress.restype = ctypes.c_int
+        L.vc_csm_compress.argtypes = ([_p, _p, _p, ctypes.c_int, ctypes.c_int, _i64, _i64,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                       _p, _p, _p, _i64, _p, _p])
         for name in GLUE_EXPORTS:
             getattr(L, name).restype = ctypes.c_int
         L.vc_glue_embed.argtypes = [_p, _p, ctypes.c_int, ctypes.c_int, _p, _p]

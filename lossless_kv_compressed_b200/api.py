@@ -273,3 +273,40 @@ def device_error(clear: bool = True) -> int:
     v = ctypes.c_int32(0)
     check(lib().vc_device_error(ctypes.byref(v), int(clear)), "vc_device_error")
     return int(v.value)
+
+
+def csm_out_len(T: int, n_sinks: int, n_recent: int, chunk: int, r: float) -> int:
+    """Rows left by one Chunked Soft Matching round over T rows (-1 if invalid)."""
+    return int(lib().vc_csm_out_len(T, n_sinks, n_recent, chunk, r))
+
+
+def csm_compress(k: torch.Tensor, v: torch.Tensor, n_sinks: int, n_recent: int, chunk: int,
+                 r: float, deg: Optional[torch.Tensor] = None, T: Optional[int] = None,
+                 k_out=None, v_out=None, deg_out=None, dest=None, stream=None):
+    """One Chunked Soft Matching round (CentroidKV) over rows [0, T) of every pair.
+
+    k, v: [B, Hkv, T_cap, D] bf16; deg: [B, Hkv, T_cap] int32 or None (all 1).
+    Returns (k_out, v_out, deg_out, n_out): a compact cache of n_out rows per pair."""
+    _need(k, torch.bfloat16, "k")
+    _need(v, torch.bfloat16, "v")
+    B, Hkv, T_cap, D = k.shape
+    T = T_cap if T is None else T
+    n_out = csm_out_len(T, n_sinks, n_recent, chunk, r)
+    if n_out < 0:
+        raise ValueError("csm_compress: invalid sizes or ratio")
+    if k_out is None:
+        k_out = torch.empty((B, Hkv, max(n_out, 1), D), dtype=k.dtype, device=k.device)
+    if v_out is None:
+        v_out = torch.empty_like(k_out)
+    if deg_out is None:
+        deg_out = torch.empty(k_out.shape[:3], dtype=torch.int32, device=k.device)
+    if deg is not None:
+        _need(deg, torch.int32, "deg")
+    if dest is not None:
+        _need(dest, torch.int32, "dest")
+    check(lib().vc_csm_compress(k.data_ptr(), v.data_ptr(), _ptr(deg), B * Hkv, D, T, T_cap,
+                                n_sinks, n_recent, chunk, float(r), k_out.data_ptr(),
+                                v_out.data_ptr(), deg_out.data_ptr(), k_out.shape[2], _ptr(dest),
+                                _stream(stream)), "vc_csm_compress")
+    return k_out, v_out, deg_out, n_out
+

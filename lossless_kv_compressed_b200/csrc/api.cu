@@ -190,4 +190,32 @@ vc_status vc_event_wait(cudaEvent_t ev, double timeout_s) { return event_wait(ev
 
 vc_status vc_device_error(int32_t* value, int clear) { return read_device_error(value, clear); }
 
+int64_t vc_csm_out_len(int64_t T, int n_sinks, int n_recent, int chunk, double r) {
+  if (T < 0 || n_sinks < 0 || n_recent < 0 || (int64_t)n_sinks + n_recent > T || chunk < 2 ||
+      chunk > 256 || !(r >= 0.0 && r <= 1.0))
+    return -1;
+  return csm_out_len(T, n_sinks, n_recent, chunk, r);
+}
+
+vc_status vc_csm_compress(const void* k, const void* v, const int32_t* deg, int pairs, int D,
+                          int64_t T, int64_t T_cap, int n_sinks, int n_recent, int chunk,
+                          double r, void* k_out, void* v_out, int32_t* deg_out,
+                          int64_t T_cap_out, int32_t* dest, cudaStream_t stream) {
+  if (pairs <= 0 || pairs > 65535) return fail(VC_ERR_INVALID, "csm: pairs");
+  if (D != 64 && D != 128) return fail(VC_ERR_UNSUPPORTED, "csm: D must be 64 or 128");
+  if (chunk < 2 || chunk > 256) return fail(VC_ERR_UNSUPPORTED, "csm: chunk must be in [2, 256]");
+  if (!(r >= 0.0 && r <= 1.0)) return fail(VC_ERR_INVALID, "csm: r must be in [0, 1]");
+  if (n_sinks < 0 || n_recent < 0 || (int64_t)n_sinks + n_recent > T || T > T_cap ||
+      T >= ((int64_t)1 << 31))
+    return fail(VC_ERR_INVALID, "csm: need n_sinks + n_recent <= T <= T_cap, T < 2^31");
+  if (!k || !v || !k_out || !v_out || !deg_out)
+    return fail(VC_ERR_INVALID, "csm: k, v, k_out, v_out, deg_out must be set");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_out) || !aligned16(v_out))
+    return fail(VC_ERR_INVALID, "csm: k / v / k_out / v_out misaligned");
+  const int64_t n_out = csm_out_len(T, n_sinks, n_recent, chunk, r);
+  if (n_out > T_cap_out) return fail(VC_ERR_INVALID, "csm: T_cap_out < output rows");
+  return launch_csm(k, v, deg, pairs, D, T, T_cap, n_sinks, n_recent, chunk, r, k_out, v_out,
+                    deg_out, T_cap_out, dest, stream);
+}
+
 }  // extern "C"

@@ -1,0 +1,360 @@
+// One round of Chunked Soft Matching (CSM), the one-pass KV-cache clustering of the
+// CentroidKV summary ("Riassunto Tecnico: CentroidKV", section "Metodologia": item 2,
+// sinks and recent tokens kept out of the partition; item 3, chunks, alternating A/B
+// partition, bipartite matching, only the most similar fraction r merged; item 4,
+// degree-weighted centroids whose degree n_t later enters the draft softmax as ln n_t).
+//
+// Readings (the page gives no formula): A = rows at even offsets of a chunk, B = odd
+// offsets; similarity = cosine of the key rows (0 for an all-zero row); each A row's
+// match is its most similar B row (lowest on ties); the m = floor(r |A|) A rows with the
+// highest similarity (lower row on ties) merge into their matches; a centroid is the
+// degree-weighted mean of K and V with the summed degree and takes its B row's place;
+// the output keeps sinks, then the survivors of each chunk in order, then recent rows.
+//
+// Design: one CTA per (chunk, pair) -- a chunk is <= 256 rows, so everything after the
+// loads stays in shared memory.  The chunk's key rows land once in a swizzled tile
+// (cp.async); the |A| x |B| dot products run on mma.sync (bf16 in, fp32 accumulate,
+// each warp one 16-row A tile against all B rows) and every A row keeps its best
+// dot / |b| with a quad reduction; the top-m selection is a rank count over the
+// chunk's <= 128 candidates; the centroids sum in a fixed order (the B row, then its
+// merged A rows in ascending order) in fp32 and round to bf16 once.  One extra CTA per
+// pair copies the sinks and recent rows.  The rows a chunk keeps and their output
+// places depend only on that chunk, so every CTA writes its own output rows.
+#include <climits>
+#include <cmath>
+
+#include "vc_common.cuh"
+#include "vc_internal.h"
+
+namespace vc {
+
+constexpr int kCsmThreads = 256;
+constexpr int kCsmMaxChunk = 256;
+
+struct CsmParams {
+  const __nv_bfloat16* k;    // [pairs, T_cap, D]
+  const __nv_bfloat16* v;
+  const int32_t* deg;        // [pairs, T_cap] or null (all 1)
+  __nv_bfloat16* k_out;      // [pairs, T_cap_out, D]
+  __nv_bfloat16* v_out;
+  int32_t* deg_out;          // [pairs, T_cap_out]
+  int32_t* dest;             // [pairs, T_cap] or null: output row of each input row
+  int64_t T_cap, T_cap_out;
+  int T, n_sinks, n_recent, chunk, n_chunks;
+  int m_full, m_last;        // merges per full chunk / the last chunk
+  int out_len;
+};
+
+template <int D>
+struct CsmSmem {
+  static constexpr int kRowB = D * 2;
+  static constexpr int kK = 0;                                     // [256][D] bf16
+  static constexpr int kInvN = kK + kCsmMaxChunk * kRowB;          // float [256]
+  static constexpr int kBestB = kInvN + kCsmMaxChunk * 4;          // int [128]
+  static constexpr int kBestS = kBestB + 128 * 4;                  // float [128]
+  static constexpr int kMerged = kBestS + 128 * 4;                 // int [128]
+  static constexpr int kScan = kMerged + 128 * 4;                  // int [256]
+  static constexpr int kTotal = kScan + kCsmMaxChunk * 4;
+};
+
+template <int D>
+__device__ __forceinline__ uint32_t csm_row_addr(uint32_t base, int r, int c) {
+  return base + r * CsmSmem<D>::kRowB + ((c ^ (r & 7)) << 4);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
+  pdl_wait();
+  pdl_trigger();
+  using SM = CsmSmem<D>;
+  constexpr int CH = D / 8;                       // 16-byte chunks per row
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t pair = blockIdx.y;
+  const __nv_bfloat16* kin = p.k + pair * p.T_cap * D;
+  const __nv_bfloat16* vin = p.v + pair * p.T_cap * D;
+  const int32_t* din = p.deg ? p.deg + pair * p.T_cap : nullptr;
+  __nv_bfloat16* kout = p.k_out + pair * p.T_cap_out * D;
+  __nv_bfloat16* vout = p.v_out + pair * p.T_cap_out * D;
+  int32_t* dout = p.deg_out + pair * p.T_cap_out;
+  int32_t* dst = p.dest ? p.dest + pair * p.T_cap : nullptr;
+  auto deg_of = [&](int row) { return din ? din[row] : 1; };
+
+  if ((int)blockIdx.x == p.n_chunks) {
+    // ---- sinks and recent rows: copied unchanged
+    const int n_copy = p.n_sinks + p.n_recent;
+    for (int e = warp; e < n_copy; e += kCsmThreads / 32) {
+      const int row = e < p.n_sinks ? e : p.T - p.n_recent + (e - p.n_sinks);
+      const int orow = e < p.n_sinks ? e : p.out_len - p.n_recent + (e - p.n_sinks);
+      for (int c = lane; c < CH; c += 32) {
+        reinterpret_cast<uint4*>(kout + (int64_t)orow * D)[c] =
+            reinterpret_cast<const uint4*>(kin + (int64_t)row * D)[c];
+        reinterpret_cast<uint4*>(vout + (int64_t)orow * D)[c] =
+            reinterpret_cast<const uint4*>(vin + (int64_t)row * D)[c];
+      }
+      if (lane == 0) {
+        dout[orow] = deg_of(row);
+        if (dst) dst[row] = orow;
+      }
+    }
+    return;
+  }
+
+  const int c_idx = blockIdx.x;
+  const int r0 = p.n_sinks + c_idx * p.chunk;
+  const int len = min(p.chunk, p.T - p.n_recent - r0);
+  const int nA = (len + 1) >> 1, nB = len >> 1;
+  const int m = nB > 0 ? (c_idx == p.n_chunks - 1 ? p.m_last : p.m_full) : 0;
+  const int base = p.n_sinks + c_idx * (p.chunk - p.m_full);
+  const uint32_t ks = smem_u32(smem + SM::kK);
+  float* invn = reinterpret_cast<float*>(smem + SM::kInvN);
+  int* best_b = reinterpret_cast<int*>(smem + SM::kBestB);
+  float* best_s = reinterpret_cast<float*>(smem + SM::kBestS);
+  int* merged = reinterpret_cast<int*>(smem + SM::kMerged);
+  int* scan = reinterpret_cast<int*>(smem + SM::kScan);
+
+  // ---- key rows of the chunk -> shared memory (rows past the chunk zeroed)
+  for (int e = tid; e < kCsmMaxChunk * CH; e += kCsmThreads) {
+    const int r = e / CH, c = e - r * CH;
+    const bool ok = r < len;
+    cp_async16(csm_row_addr<D>(ks, r, c), kin + (int64_t)(r0 + (ok ? r : 0)) * D + c * 8,
+               ok ? 16u : 0u);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // ---- 1 / |k| of every row (0 for an all-zero row: its cosines are 0)
+  {
+    const int r = tid;
+    float ss = 0.f;
+    if (r < len) {
+      const uint8_t* row = smem + SM::kK + r * SM::kRowB;
+#pragma unroll 4
+      for (int c = 0; c < CH; ++c) {
+        const uint4 w = *reinterpret_cast<const uint4*>(row + ((c ^ (r & 7)) << 4));
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float a = bf16_lo(ww[u]), b = bf16_hi(ww[u]);
+          ss = fmaf(a, a, ss);
+          ss = fmaf(b, b, ss);
+        }
+      }
+    }
+    invn[r] = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+  }
+  __syncthreads();
+
+  // ---- best B match of every A row: warp w takes A rows 16w .. 16w+15 (chunk rows
+  //      2i), all B rows (chunk rows 2j+1), dot products on mma.sync
+  if (16 * warp < nA) {
+    const int qr = lane >> 2, qc = lane & 3;
+    // A fragments for all k-steps: rows i = 16w + (lane & 15), chunk 2ks + (lane >> 4)
+    uint32_t af[D / 16][4];
+    {
+      const int i = 16 * warp + (lane & 15);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+        ldsm_x4(csm_row_addr<D>(ks, 2 * i, 2 * kk + (lane >> 4)), af[kk][0], af[kk][1],
+                af[kk][2], af[kk][3]);
+    }
+    float bv[2] = {-INFINITY, -INFINITY};
+    int bj[2] = {INT_MAX, INT_MAX};
+    for (int nt = 0; nt < (nB + 7) / 8; ++nt) {
+      float s[4] = {0.f, 0.f, 0.f, 0.f};
+      const int j = 8 * nt + (lane & 7);              // B row of this lane's ldmatrix row
+#pragma unroll
+      for (int kk = 0; kk < D / 32; ++kk) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(csm_row_addr<D>(ks, 2 * j + 1, 4 * kk + (lane >> 3)), b0, b1, b2, b3);
+        mma_bf16(s, af[2 * kk][0], af[2 * kk][1], af[2 * kk][2], af[2 * kk][3], b0, b1);
+        mma_bf16(s, af[2 * kk + 1][0], af[2 * kk + 1][1], af[2 * kk + 1][2],
+                 af[2 * kk + 1][3], b2, b3);
+      }
+      // accumulator: rows qr, qr + 8; columns (B rows) 8nt + 2qc, +1
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int jj = 8 * nt + 2 * qc + (e & 1);
+        const int h = e >> 1;
+        if (jj < nB) {
+          const float val = s[e] * invn[2 * jj + 1];
+          if (val > bv[h] || (val == bv[h] && jj < bj[h])) { bv[h] = val; bj[h] = jj; }
+        }
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int o = 1; o < 4; o <<= 1) {
+        const float v2 = __shfl_xor_sync(0xffffffffu, bv[h], o);
+        const int j2 = __shfl_xor_sync(0xffffffffu, bj[h], o);
+        if (v2 > bv[h] || (v2 == bv[h] && j2 < bj[h])) { bv[h] = v2; bj[h] = j2; }
+      }
+      const int i = 16 * warp + qr + 8 * h;
+      if (qc == 0 && i < nA) {
+        best_b[i] = bj[h] == INT_MAX ? 0 : bj[h];
+        best_s[i] = bv[h] == -INFINITY ? 0.f : bv[h] * invn[2 * i];
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- the m most similar A rows merge (higher cosine first, lower row on ties)
+  if (tid < 128) {
+    int mg = 0;
+    if (tid < nA && m > 0) {
+      const float st = best_s[tid];
+      int rank = 0;
+      for (int u = 0; u < nA; ++u) {
+        const float su = best_s[u];
+        rank += (su > st || (su == st && u < tid)) ? 1 : 0;
+      }
+      mg = rank < m ? 1 : 0;
+    }
+    merged[tid] = mg;
+  }
+  __syncthreads();
+
+  // ---- output places: exclusive prefix count of the kept rows of the chunk
+  const bool keep = tid < len && !((tid & 1) == 0 && merged[tid >> 1]);
+  scan[tid] = keep ? 1 : 0;
+  __syncthreads();
+  for (int off = 1; off < kCsmMaxChunk; off <<= 1) {
+    const int add = tid >= off ? scan[tid - off] : 0;
+    __syncthreads();
+    scan[tid] += add;
+    __syncthreads();
+  }
+  // scan[t] is now the inclusive count: kept row t goes to base + scan[t] - 1
+  if (dst && tid < len) {
+    const int own = tid & 1 ? tid : (merged[tid >> 1] ? 2 * best_b[tid >> 1] + 1 : tid);
+    dst[r0 + tid] = base + scan[own] - 1;
+  }
+
+  // ---- write the kept rows: unmerged A rows as they are, B rows as centroids
+  constexpr int DPL = D / 32;                     // channels per lane
+  for (int t = warp; t < len; t += kCsmThreads / 32) {
+    if ((t & 1) == 0 && merged[t >> 1]) continue;  // warp-uniform
+    const int orow = base + scan[t] - 1;
+    const int row = r0 + t;
+    float ak[DPL], av[DPL];
+    int ntot = deg_of(row);
+    const float nb = (float)ntot;
+    auto load_k = [&](int r, float (&x)[DPL]) {     // channels lane*DPL .. from shared
+      const int d0 = lane * DPL;
+      const uint8_t* src = smem + SM::kK + r * SM::kRowB + (((d0 >> 3) ^ (r & 7)) << 4) +
+                           (d0 & 7) * 2;
+      if constexpr (DPL == 4) {
+        const uint2 w = *reinterpret_cast<const uint2*>(src);
+        x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+      } else {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(src);
+        x[0] = bf16_lo(w); x[1] = bf16_hi(w);
+      }
+    };
+    auto load_v = [&](int r, float (&x)[DPL]) {     // from global
+      const __nv_bfloat16* src = vin + (int64_t)(r0 + r) * D + lane * DPL;
+      if constexpr (DPL == 4) {
+        const uint2 w = *reinterpret_cast<const uint2*>(src);
+        x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+      } else {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(src);
+        x[0] = bf16_lo(w); x[1] = bf16_hi(w);
+      }
+    };
+    load_k(t, ak);
+    load_v(t, av);
+    if (t & 1) {
+      // a B row: add the A rows merged into it, in ascending order
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) { ak[e] *= nb; av[e] *= nb; }
+      const int j = t >> 1;
+      for (int i0 = 0; i0 < nA; i0 += 32) {
+        const int i = i0 + lane;
+        const bool in = i < nA && merged[i] && best_b[i] == j;
+        unsigned bal = __ballot_sync(0xffffffffu, in);
+        while (bal) {
+          const int a = i0 + __ffs(bal) - 1;
+          bal &= bal - 1;
+          const int na = deg_of(r0 + 2 * a);
+          float xk[DPL], xv[DPL];
+          load_k(2 * a, xk);
+          load_v(2 * a, xv);
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) {
+            ak[e] = fmaf((float)na, xk[e], ak[e]);
+            av[e] = fmaf((float)na, xv[e], av[e]);
+          }
+          ntot += na;
+        }
+      }
+      const float inv = (float)ntot;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) { ak[e] = ak[e] / inv; av[e] = av[e] / inv; }
+    }
+    __nv_bfloat16* ko = kout + (int64_t)orow * D + lane * DPL;
+    __nv_bfloat16* vo = vout + (int64_t)orow * D + lane * DPL;
+    if constexpr (DPL == 4) {
+      *reinterpret_cast<uint2*>(ko) = make_uint2(pack_bf16x2(ak[0], ak[1]), pack_bf16x2(ak[2], ak[3]));
+      *reinterpret_cast<uint2*>(vo) = make_uint2(pack_bf16x2(av[0], av[1]), pack_bf16x2(av[2], av[3]));
+    } else {
+      *reinterpret_cast<uint32_t*>(ko) = pack_bf16x2(ak[0], ak[1]);
+      *reinterpret_cast<uint32_t*>(vo) = pack_bf16x2(av[0], av[1]);
+    }
+    if (lane == 0) dout[orow] = ntot;
+  }
+}
+
+int64_t csm_out_len(int64_t T, int n_sinks, int n_recent, int chunk, double r) {
+  const int64_t mid = T - n_sinks - n_recent;
+  int64_t n = n_sinks + n_recent;
+  for (int64_t c0 = 0; c0 < mid; c0 += chunk) {
+    const int64_t len = mid - c0 < chunk ? mid - c0 : chunk;
+    // a one-row chunk has no B row: nothing merges
+    n += len - (len >= 2 ? (int64_t)std::floor(r * (double)((len + 1) / 2)) : 0);
+  }
+  return n;
+}
+
+vc_status launch_csm(const void* k, const void* v, const int32_t* deg, int pairs, int D,
+                     int64_t T, int64_t T_cap, int n_sinks, int n_recent, int chunk, double r,
+                     void* k_out, void* v_out, int32_t* deg_out, int64_t T_cap_out,
+                     int32_t* dest, cudaStream_t stream) {
+  CsmParams p;
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.deg = deg;
+  p.k_out = static_cast<__nv_bfloat16*>(k_out);
+  p.v_out = static_cast<__nv_bfloat16*>(v_out);
+  p.deg_out = deg_out;
+  p.dest = dest;
+  p.T_cap = T_cap;
+  p.T_cap_out = T_cap_out;
+  p.T = (int)T;
+  p.n_sinks = n_sinks;
+  p.n_recent = n_recent;
+  p.chunk = chunk;
+  const int64_t mid = T - n_sinks - n_recent;
+  p.n_chunks = (int)((mid + chunk - 1) / chunk);
+  const int64_t last = mid - (int64_t)(p.n_chunks - 1) * chunk;
+  p.m_full = (int)std::floor(r * (double)((chunk + 1) / 2));
+  p.m_last = p.n_chunks > 0 && last >= 2 ? (int)std::floor(r * (double)((last + 1) / 2)) : 0;
+  p.out_len = (int)csm_out_len(T, n_sinks, n_recent, chunk, r);
+  const dim3 grid(p.n_chunks + 1, pairs);
+  if (D == 128) {
+    VC_CUDA(cudaFuncSetAttribute(csm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 CsmSmem<128>::kTotal));
+    VC_CUDA(launch_pdl(csm_kernel<128>, grid, dim3(kCsmThreads), CsmSmem<128>::kTotal, stream,
+                       1, p));
+  } else {
+    VC_CUDA(cudaFuncSetAttribute(csm_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 CsmSmem<64>::kTotal));
+    VC_CUDA(launch_pdl(csm_kernel<64>, grid, dim3(kCsmThreads), CsmSmem<64>::kTotal, stream, 1,
+                       p));
+  }
+  VC_CUDA(cudaGetLastError());
+  return VC_OK;
+}
+
+}  // namespace vc

@@ -38,6 +38,12 @@ vc_status launch_verify(const void* q, int B, int n_q, int Hq, int Hkv, int D, c
 
 vc_status read_device_error(int32_t* value, int clear);
 
+int64_t csm_out_len(int64_t T, int n_sinks, int n_recent, int chunk, double r);
+vc_status launch_csm(const void* k, const void* v, const int32_t* deg, int pairs, int D,
+                     int64_t T, int64_t T_cap, int n_sinks, int n_recent, int chunk, double r,
+                     void* k_out, void* v_out, int32_t* deg_out, int64_t T_cap_out,
+                     int32_t* dest, cudaStream_t stream);
+
 vc_status launch_accept(const float* logits, const int32_t* drafts, int B, int n_q, int V,
                         int32_t* target, int32_t* accept_len, int32_t* commit,
                         int32_t* n_commit, int32_t* err_flag, cudaStream_t stream);

@@ -39,7 +39,8 @@ def out_len(T: int, n_sinks: int, n_recent: int, chunk: int, r: float) -> int:
     n = n_sinks + n_recent
     for c0 in range(0, mid, chunk):
         ln = min(chunk, mid - c0)
-        n += ln - math.floor(r * ((ln + 1) // 2))
+        # a one-row chunk has no B row: nothing merges
+        n += ln - (math.floor(r * ((ln + 1) // 2)) if ln >= 2 else 0)
     return n
 
 
