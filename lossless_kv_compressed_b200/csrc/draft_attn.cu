@@ -20,8 +20,11 @@
 //   Scores live in the log2 domain: s2 = s * scale * log2(e) + log2(n_t); the online
 //   softmax uses ex2.  A warp writes one partial (max, sum, unnormalised o) per pair
 //   it touches; a second kernel merges the partials of each head in a fixed order.
-//   (Measured and rejected: L2 bulk prefetch of rows beyond the ring, 37% slower;
-//   launching the merge as a programmatic dependent, 4% slower.)
+//   Both kernels start with pdl_wait() and are launched as programmatic dependents, so
+//   the merge's launch overlaps the split kernel's tail (vc_common.cuh).
+//   (Measured and rejected: an L2 bulk prefetch of rows beyond the ring, 37% slower;
+//   per-lane cp.async.bulk row copies on an mbarrier ring, 20% slower; 3 CTAs per SM
+//   with a 2-stage ring, no gain.)
 #include <climits>
 
 #include "vc_common.cuh"
