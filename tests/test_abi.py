@@ -95,3 +95,29 @@ def test_accept_and_stage_reject_bad_arguments():
     assert L.vc_accept(1 << 20, None, 1, 9, 1024, 1 << 20, 1 << 20, 1 << 20, 1 << 20, None, None) == 1
     assert L.vc_stage_full_kv(1 << 20, 1 << 20, 100, 0, None, None, 0) == 1
     assert L.vc_stage_full_kv(None, 1 << 20, 100, 10, None, None, 0) == 1
+
+
+@pytest.mark.parametrize("T,ns,nr,chunk,r", [(40, 4, 6, 8, 0.5), (90, 2, 3, 2, 1.0),
+                                            (32768, 4, 512, 256, 0.5), (517, 8, 9, 256, 0.3),
+                                            (31, 0, 0, 10, 1.0), (10, 5, 5, 4, 0.7),
+                                            (1000, 0, 0, 7, 0.999), (64, 4, 4, 16, 0.0)])
+def test_csm_out_len_matches_the_oracle(T, ns, nr, chunk, r):
+    from oracle import csm
+    assert vc.lib().vc_csm_out_len(T, ns, nr, chunk, r) == csm.out_len(T, ns, nr, chunk, r)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(D=96), 2), (dict(chunk=1), 2), (dict(chunk=512), 2), (dict(r=1.5), 1),
+    (dict(r=-0.1), 1), (dict(n_sinks=60, n_recent=60), 1), (dict(T=300), 1),
+    (dict(T_cap_out=10), 1), (dict(pairs=0), 1), (dict(k=3), 1)])
+def test_csm_rejects_bad_arguments(kw, status):
+    a = dict(k=256, v=256, deg=0, pairs=2, D=128, T=100, T_cap=200, n_sinks=4, n_recent=4,
+             chunk=16, r=0.5, k_out=256, v_out=256, deg_out=256, T_cap_out=200, dest=0)
+    a.update(kw)
+    L = vc.lib()
+    st = L.vc_csm_compress(a["k"], a["v"], a["deg"] or None, a["pairs"], a["D"], a["T"],
+                           a["T_cap"], a["n_sinks"], a["n_recent"], a["chunk"], a["r"],
+                           a["k_out"], a["v_out"], a["deg_out"], a["T_cap_out"],
+                           a["dest"] or None, None)
+    assert st == status, _lib.status_name(st)
+    assert vc.lib().vc_last_error()
