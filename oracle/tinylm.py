@@ -21,7 +21,7 @@ Loops:
   CentroidKV", item 2: sinks and recent tokens are kept; eviction by attention
   score as in its "Problematica" section).
 
-Readings for what the pages leave open (listed again in the design doc):
+Readings for what the pages leave open:
 the verify pass feeds the pending token plus the k drafts (k + 1 rows); on a
 disagreement the full-KV prediction at that row is committed as the correction;
 after a round the full cache keeps the a + 1 verified block entries, the draft
