@@ -435,7 +435,7 @@ def e2e_measure(rnd, steps: int, warmup: int, device) -> dict:
             "ms_per_step": tot / steps * 1e3}
 
 
-# ------------------------------------------------------------------ workload 4
+# ------------------------------------------------------------------ 1M-token staged verify
 def run_config4(args) -> int:
     """Long-context staging: one request's 1M-token full cache (4 GiB, chunk-major in
     pinned host memory) streams through a 3-slot HBM ring for its k = 40 verify while
@@ -537,7 +537,7 @@ def run_config4(args) -> int:
     return 0
 
 
-# ------------------------------------------------------------------ workload 5
+# ------------------------------------------------------------------ tiny-decoder loop
 def run_config5(args) -> int:
     """The loop end to end on the tiny decoder: accepted tokens/s of the VeriCache loop
     and of full-KV greedy decoding on the same GPU, and the acceptance-length histogram.
@@ -579,7 +579,7 @@ def run_config5(args) -> int:
         "greedy_tokens_per_s": cfg.gen_tokens / tg,
         "rounds": len(alens), "mean_accept_len": float(np.mean(alens)),
         "accept_len_histogram": hist,
-        "oracle_fp64": "tests/test_gpu_loop.py::test_workload5_greedy_follows_oracle_to_a_near_tie",
+        "oracle_fp64": "tests/test_gpu_loop.py::test_tinylm_loop_greedy_follows_oracle_to_a_near_tie",
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -641,7 +641,7 @@ def run_table(args) -> int:
               "bytes": nbytes, "TFLOP/s": tf, "frac_tensor": tf / peaks["bf16_tflops"],
               "frac_attainable": tf / attain, "GB/s": nbytes / t / 1e9, "note": note})
 
-    # ---- workload 1: B1, 8/2 heads, D 64, 256 slots of 1024 + 8 tail rows; verify k = 8
+    # ---- tiny: B1, 8/2 heads, D 64, 256 slots of 1024 + 8 tail rows; verify k = 8
     c = get_config(1)
     T = c.L_cap
     k1, v1 = bf(c.B, c.Hkv, T, c.D), bf(c.B, c.Hkv, T, c.D)
@@ -653,7 +653,7 @@ def run_table(args) -> int:
                             n_tail=c.k)
     draft_row(1, cache, bf(c.B, c.Hq, c.D), draft_bytes(c, c.k), "L2-resident: report us")
     verify_row(1, c.B, c.Hq, c.Hkv, c.D, c.P, c.k + 1, k1, v1, "latency-bound")
-    # ---- workload 2
+    # ---- 32K context: B8, 32/8 heads, D 128, 8192 slots + 32 tail rows; verify k = 32
     c = get_config(2)
     k2, v2 = bf(c.B, c.Hkv, c.L_cap, c.D), bf(c.B, c.Hkv, c.L_cap, c.D)
     idx = torch.stack([torch.sort(torch.randperm(c.P, device=dev, generator=g)[:c.S])[0]
@@ -665,7 +665,7 @@ def run_table(args) -> int:
     draft_row(2, cache, bf(c.B, c.Hq, c.D), draft_bytes(c, c.k), "indexed, 32 tail rows")
     verify_row(2, c.B, c.Hq, c.Hkv, c.D, c.P, c.k + 1, k2, v2, "k = 32")
     del k2, v2, cache
-    # ---- workload 3: int4 cache of 130944 tokens + 128 bf16 tail rows; verify over bf16
+    # ---- 128K int4: 130944 quantised tokens + 128 bf16 tail rows; verify over bf16
     c = get_config(3)
     nb = (c.P - c.tail_bf16) // 32
     pairs = (c.B, c.Hkv, nb)
@@ -687,7 +687,7 @@ def run_table(args) -> int:
     k3, v3 = bf(c.B, c.Hkv, c.L_cap, c.D), bf(c.B, c.Hkv, c.L_cap, c.D)
     verify_row(3, c.B, c.Hq, c.Hkv, c.D, c.P, c.k + 1, k3, v3, "k = 32, 128K context")
     del k3, v3
-    # ---- workload 4: compact 65536-slot caches for 3 requests; verify over a device-resident
+    # ---- 1M tokens: compact 65536-slot caches for 3 requests; verify over a device-resident
     #      1M-token context (the staged form is bench.py --config 4)
     c = get_config(4)
     nd = c.n_draft_requests
@@ -701,7 +701,7 @@ def run_table(args) -> int:
     verify_row(4, 1, c.Hq, c.Hkv, c.D, c.P, c.k + 1, k4, v4,
                "k = 40, 1M-token context resident in HBM (one call)")
     del k4, v4
-    # ---- Chunked Soft Matching, one round over workload 2's full caches (chunk 256,
+    # ---- Chunked Soft Matching, one round over the 32K-context full caches (chunk 256,
     #      r = 0.5): reads K, V and degrees, writes the compact cache
     c = get_config(2)
     kc, vcc = bf(c.B, c.Hkv, c.P, c.D), bf(c.B, c.Hkv, c.P, c.D)
@@ -757,7 +757,7 @@ def run_table(args) -> int:
 
 
 def run_profile_case(kind: str) -> int:
-    """A short run of one call of the workload-2 round for an ncu capture: one copy of
+    """A short run of one call of the 32K-context round for an ncu capture: one copy of
     the inputs (about 1.2 GB on the device), five calls of the chosen entry point."""
     import torch
     import lossless_kv_compressed_b200 as vc
@@ -804,7 +804,7 @@ def main():
     ap.add_argument("--table", action="store_true",
                     help="per-kernel rates at every workload's shapes, one JSON line per row")
     ap.add_argument("--profile-case", choices=["draft", "verify", "accept"], default=None,
-                    help="run five calls of one entry point on the workload-2 inputs (one "
+                    help="run five calls of one entry point on the 32K-context inputs (one "
                          "copy) for an ncu capture, and print no bench line")
     ap.add_argument("--config", type=int, default=2, choices=[2, 4, 5],
                     help="2: the round of the 32K-context layer (default line); "

@@ -33,9 +33,9 @@ class AttnConfig:
     vocab: int = 0         # vocabulary of the acceptance logits
     rho: float = 0.9       # AR(1) coefficient along the sequence (0 = i.i.d.)
     outlier_frac: float = 0.0  # int4 workload: fraction of (kv head, channel) pairs scaled x10
-    n_draft_requests: int = 0  # workload 4: other requests drafting meanwhile
-    draft_context: int = 0     # workload 4: their context length
-    chunk_tokens: int = 0      # workload 4: KV_full streamed in chunks of this many tokens
+    n_draft_requests: int = 0  # staged verify: other requests drafting meanwhile
+    draft_context: int = 0     # staged verify: their context length
+    chunk_tokens: int = 0      # staged verify: KV_full streamed in chunks of this many tokens
 
     @property
     def g(self) -> int:
@@ -53,7 +53,7 @@ class AttnConfig:
 
 @dataclass(frozen=True)
 class LoopConfig:
-    """Workload 5: the end-to-end loop on a tiny random-init decoder."""
+    """The end-to-end loop on a tiny random-init decoder."""
 
     num: int = 5
     name: str = "tinylm-loop"

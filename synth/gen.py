@@ -223,7 +223,7 @@ def ar1_chunks(rng: Generator, lead: tuple, L: int, D: int, rho: float, chunk: i
 
 
 def staged_case(cfg=None, chunk: int | None = None, P: int | None = None):
-    """Workload-4 inputs: the full cache of one request as chunk-major bf16 bits
+    """1M-token staged inputs: the full cache of one request as chunk-major bf16 bits
     (generator of [2 (K|V), Hkv, chunk, D] pieces), its verify queries and block K/V,
     and the compact compressed caches of the drafting requests."""
     cfg = cfg or get_config(4)

@@ -35,7 +35,7 @@ def _check(logits, drafts):
     return g
 
 
-def test_workload1():
+def test_tiny_1k_context_inputs():
     case = gen.attn_case(1)
     g = _check(case["logits"], case["drafts"])
     assert g["accept_len"].tolist() == [5] and g["n_commit"].tolist() == [6]

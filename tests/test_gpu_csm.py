@@ -137,7 +137,7 @@ def test_clear_margins_give_the_oracle_decisions():
     assert np.array_equal(dest[0, 0], want)
 
 
-def test_workload2_size_sampled_pairs():
+def test_32k_context_size_sampled_pairs():
     """B 8 x 8 kv heads x 32768 rows, D 128, chunk 256, r = 0.5, degrees 1..16: structure
     and decisions checked on sampled pairs."""
     kb, vb, deg = _inputs(8, 8, 32768, 128, seed=2, deg_max=16, ar=0.9)

@@ -48,7 +48,7 @@ def _run(case, S, n_tail, use_idx=True, use_deg=True, check_lse=True):
     return res
 
 
-def test_workload1_full():
+def test_tiny_1k_context_full():
     case = gen.attn_case(1)
     for n_tail in (0, 1, 9):
         _run(case, case["cfg"].S, n_tail)
@@ -94,8 +94,8 @@ def case2():
     return gen.attn_case(2)
 
 
-def test_workload2_full_size(case2):
-    """Full workload-2 sizes (B 8, 32/8 heads, D 128, 8192 slots of a 32K context,
+def test_32k_context_full_size(case2):
+    """Full 32K-context sizes (B 8, 32/8 heads, D 128, 8192 slots of a 32K context,
     degrees 1..16) with the longest draft tail of a round (k = 32)."""
     _run(case2, case2["cfg"].S, case2["cfg"].k)
 

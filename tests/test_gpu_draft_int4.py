@@ -107,8 +107,8 @@ def test_tail_only_and_no_tail():
     _run(case, 256, 0)
 
 
-def test_workload3_full_size_sampled_pairs():
-    """Full workload-3 sizes: batch 4, 32/8 heads, D 128, 130944 quantised tokens
+def test_128k_int4_full_size_sampled_pairs():
+    """Full 128K int4 sizes: batch 4, 32/8 heads, D 128, 130944 quantised tokens
     (4092 groups, 1% outlier channels x10) plus the 128-token bf16 tail."""
     cfg = gen.get_config(3)
     case = gen.attn_case(3)

@@ -133,9 +133,10 @@ def test_no_compression_accepts_every_draft():
     assert toks == greedy_loop(_model(cfg, w), prompt, cfg.gen_tokens)
 
 
-def test_workload5_full_size():
-    """Workload 5: 4 layers, d 512, 8/2 heads of 64, SwiGLU 1408, vocab 8192, N(0, 0.02)
-    weights; 8192-token prompt, 512 generated, k = 32, 2048-slot budget."""
+def test_tinylm_loop_full_size():
+    """The tiny-decoder loop at full size: 4 layers, d 512, 8/2 heads of 64, SwiGLU
+    1408, vocab 8192, N(0, 0.02) weights; 8192-token prompt, 512 generated, k = 32,
+    2048-slot budget."""
     cfg = get_config(5)
     w = gen.tinylm_weights(cfg)
     prompt = gen.tinylm_prompt(cfg)
@@ -146,9 +147,10 @@ def test_workload5_full_size():
     assert sum(a + 1 for a in alens) >= cfg.gen_tokens - 1
 
 
-def test_workload5_greedy_follows_oracle_to_a_near_tie():
-    """Workload 5: the GPU decoder's logits stay within the bf16-activation error of the
-    fp64 oracle's on the GPU's own greedy stream (the oracle is fed the same tokens), and
+def test_tinylm_loop_greedy_follows_oracle_to_a_near_tie():
+    """The tiny-decoder loop model: the GPU decoder's logits stay within the
+    bf16-activation error of the fp64 oracle's on the GPU's own greedy stream (the
+    oracle is fed the same tokens), and
     wherever the two argmaxes differ, the oracle's margin between its pick and the GPU's
     is inside that error -- a near-tie, where either token is a correct rounding.  (The
     random N(0, 0.02) logits are near-flat: top-2 gaps of 1e-4 occur within 16 tokens.)"""
@@ -166,7 +168,8 @@ def test_workload5_greedy_follows_oracle_to_a_near_tie():
         assert err < 3e-2, f"step {step}: logit error {err:.3e}"
         tg, to = int(np.argmax(g)), int(np.argmax(o))
         if tg != to:
-            assert o[to] - o[tg] <= 2 * err, f"step {step}: margin {o[to] - o[tg]:.3e} > 2 x {err:.3e}"
+            margin = o[to] - o[tg]
+            assert margin <= 2 * err, f"step {step}: margin {margin:.3e} > 2 x {err:.3e}"
         ids = torch.tensor([tg], dtype=torch.int32, device="cuda")
         g = m.forward(ids, 1, p, "full").double().cpu().numpy()[0]
         o = tinylm._decode_full(om, tg, p, Ks, Vs)

@@ -42,10 +42,10 @@ def _oracle(case, q_bits, P):
                               f(case["v_bits"][:, :, :P + n_q]), P)
 
 
-def test_workload1():
+def test_tiny_1k_context():
     case = gen.attn_case(1)
     q_bits, out = _verify(case)
-    assert_close_attn(host_f64(out), _oracle(case, q_bits, case["cfg"].P), "verify wl1")
+    assert_close_attn(host_f64(out), _oracle(case, q_bits, case["cfg"].P), "verify tiny 1K context")
 
 
 @pytest.mark.parametrize("D,Hq,Hkv", [(128, 32, 8), (64, 8, 2), (128, 8, 8), (64, 16, 2)])
@@ -140,8 +140,8 @@ def case2():
     return gen.attn_case(2)
 
 
-def test_workload2_sampled_rows(case2):
-    """Full workload-2 size (B 8, 32/8 heads, D 128, P 32768, k 32) in the bench's
+def test_32k_context_sampled_rows(case2):
+    """Full 32K-context size (B 8, 32/8 heads, D 128, P 32768, k 32) in the bench's
     launch configuration; the oracle recomputes sampled block positions one by one."""
     cfg = case2["cfg"]
     q_bits, out = _verify(case2)
@@ -152,4 +152,4 @@ def test_workload2_sampled_rows(case2):
         P_i = cfg.P + i
         want = oracle.verify_attn(f(q_bits[b:b + 1, i:i + 1]), f(case2["k_bits"][b:b + 1, :, :P_i + 1]),
                                   f(case2["v_bits"][b:b + 1, :, :P_i + 1]), P_i)
-        assert_close_attn(got[b:b + 1, i:i + 1], want, f"wl2 b={b} i={i}")
+        assert_close_attn(got[b:b + 1, i:i + 1], want, f"32K context b={b} i={i}")

@@ -80,8 +80,8 @@ def test_drafts_none_gives_argmax_only():
     assert r["target"][:, 0].tolist() == np.argmax(logits[:, 0], axis=1).tolist()
 
 
-def test_workload1_construction_accepts_five():
-    """Workload 1 lifts the draft logit on rows 0-4 and breaks row 5."""
+def test_tiny_inputs_construction_accepts_five():
+    """The tiny 1K-context inputs lift the draft logit on rows 0-4 and break row 5."""
     case = gen.attn_case(1)
     r = oracle.accept(case["logits"], case["drafts"])
     assert r["accept_len"].tolist() == [5]

@@ -253,7 +253,7 @@ def test_verify_chunked_equals_unchunked(chunk):
 
 
 def test_verify_on_workload1_inputs_matches_sdpa():
-    """The oracle on the seeded workload-1 inputs (bf16 widened exactly)."""
+    """The oracle on the seeded tiny 1K-context inputs (bf16 widened exactly)."""
     case = gen.attn_case(1)
     cfg = case["cfg"]
     q = oracle.bf16_to_f64(case["q_verify_bits"])
