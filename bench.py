@@ -220,6 +220,18 @@ def oracle_pair_sample(case, b: int, j: int):
     return nbytes, time.perf_counter() - t0
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (first entry of /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(case, budget_s: float = 20.0) -> dict:
     """The oracle, as it stands, on a bounded sample of the same workload."""
     cfg = case["cfg"]
@@ -236,6 +248,7 @@ def cpu_baseline(case, budget_s: float = 20.0) -> dict:
             break
     cores = max(1, round((time.process_time() - c0) / max(time.perf_counter() - w0, 1e-9)))
     return {"value": tot_b / tot_t / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "cpu": cpu_model(), "host_cores": os.cpu_count(),
             "sample": f"{n} of {len(pairs)} (batch, kv head) pairs of one round: all {cfg.k} "
                       f"draft calls and the {cfg.k + 1} verify positions of each pair, fp64 "
                       f"NumPy on {os.cpu_count()} host cores ({tot_t:.1f} s)"}
@@ -269,6 +282,7 @@ def run_reference(args, world, rank, case=None):
                        "head_dim": cfg.D, "context": cfg.P, "slots": cfg.S, "draft_len": cfg.k,
                        "step": "one (batch, kv head) pair's share of a round"},
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "cpu": cpu_model(), "host_cores": os.cpu_count(),
                              "sample": "each step: one (batch, kv head) pair's k draft calls "
                                        "and verify rows, fp64 NumPy"},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
