@@ -5,7 +5,10 @@
 //
 // Kernel 1: float4 streaming argmax of each logits row (ties -> lowest index; NaN
 //           larger than any number, first NaN wins).  Each thread keeps 8 float4 loads
-//           in flight; when the rows are few (a draft step's B rows) each row is split
+//           in flight, and a group of 4 values takes the per-element comparison only
+//           when it holds a NaN or a value above the thread's best so far (a thread
+//           meets its indices in increasing order, so equal values never replace the
+//           best).  When the rows are few (a draft step's B rows) each row is split
 //           over a cluster of up to 8 CTAs merged through distributed shared memory, so
 //           the grid still covers the SMs.  The row's NaN bit is parked in bit 31 of its
 //           target entry -- except for one-position rows (n_q == 1), whose outputs this
