@@ -79,3 +79,22 @@ def test_argmax_only():
     rng = np.random.default_rng(4)
     logits = rng.standard_normal((8, 1, 128256)).astype(np.float32)
     _check(logits, None)
+
+
+@pytest.mark.parametrize("V", [5000, 33, 128256])
+def test_one_position_rows_ties_nan_and_minus_inf(V):
+    """One-position rows (a draft step) finish in the argmax launch itself: ties to the
+    lowest index, the first NaN wins and flags the row, an all -inf row gives 0; in
+    acceptance mode accept_len 0, commit [target], n_commit 1."""
+    rng = np.random.default_rng(V)
+    logits = rng.integers(-2, 2, size=(5, 1, V)).astype(np.float32)
+    logits[1, 0, V - 2] = np.nan
+    logits[1, 0, V // 3] = np.nan
+    logits[2, 0, :] = -np.inf
+    logits[3, 0, V - 1] = 7.0
+    g = _check(logits, None)
+    assert g["err"].tolist() == [0, 1, 0, 0, 0]
+    assert g["target"][1, 0] == V // 3 and g["target"][2, 0] == 0 and g["target"][3, 0] == V - 1
+    g = _check(logits, np.zeros((5, 0), np.int32))
+    assert g["accept_len"].tolist() == [0] * 5 and g["n_commit"].tolist() == [1] * 5
+    assert np.array_equal(g["commit"][:, 0], g["target"][:, 0])
