@@ -929,8 +929,10 @@ def main():
             "gpu_launches": rnd.launches_per_step * args.steps,
             "kernels": {
                 "vc_draft_attn": {"us": d_time * 1e6, "GB/s": achieved,
-                                  "frac_hbm": achieved / peaks["hbm_gbs"]},
+                                  "frac_hbm": achieved / peaks["hbm_gbs"],
+                                  "queries_per_s": cfg.B / d_time},
                 "vc_verify_attn": {"us": verify_s * 1e6,
+                                   "queries_per_s": cfg.B * (cfg.k + 1) / verify_s,
                                    "TFLOP/s": verify_flops(cfg) / verify_s / 1e12,
                                    "frac_tensor": verify_flops(cfg) / verify_s / 1e12
                                    / peaks["bf16_tflops"],
@@ -939,6 +941,7 @@ def main():
                                    / peaks["hbm_gbs"]},
             },
             "round_bytes": rb,
+            "rounds_per_s": world * args.steps / t_max,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
