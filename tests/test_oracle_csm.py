@@ -129,3 +129,19 @@ def test_centroid_of_identical_rows_keeps_the_attention():
     comp, _ = oracle.draft_attn(q, Ko[None, None], Vo[None, None], len(no), None,
                                 no[None, None].astype(np.int64))
     assert np.allclose(full, comp, rtol=0, atol=1e-12)
+
+
+def test_hand_worked_cases():
+    """tests/golden/csm_cases.json: a six-row chunk in 2-D worked by hand (cosines,
+    matches, ranking, centroids) at r = 0.5 and r = 1."""
+    import json
+    import os
+    d = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "csm_cases.json")))
+    K, V, n = (np.asarray(d[k], dtype=np.float64) for k in ("K", "V", "n"))
+    for c in d["cases"]:
+        Ko, Vo, no, dest = csm.compress(K, V, n.astype(np.int64), d["n_sinks"], d["n_recent"],
+                                        d["chunk"], c["r"])
+        assert dest.tolist() == c["dest"], c["note"]
+        assert no.tolist() == c["n_out"], c["note"]
+        assert np.allclose(Ko, c["K_out"], rtol=0, atol=1e-15), c["note"]
+        assert np.allclose(Vo, c["V_out"], rtol=0, atol=1e-15), c["note"]
