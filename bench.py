@@ -546,6 +546,10 @@ def run_config4(args) -> int:
         "draft": {"alone_us": draft_alone_s * 1e6, "alone_GBs": d_bytes / draft_alone_s / 1e9,
                   "steps_during_round": n_drafts,
                   "overlapped_GBs": n_drafts * d_bytes / draft_span_s / 1e9},
+        # context only: the verified request's committed tokens/s if each round accepted
+        # the 25-40 tokens the VeriCache summary reports for trained models
+        "modelled_accepted_tokens_per_s_at_25_40": [25 / (round_ms * 1e-3),
+                                                    40 / (round_ms * 1e-3)],
     }
     print(json.dumps(line), flush=True)
     return 0
