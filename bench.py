@@ -198,8 +198,9 @@ def job_throughput(units_per_rank_step: float, steps: int, world: int,
 # ------------------------------------------------------------------ oracle baseline
 def oracle_pair_sample(case, b: int, j: int):
     """The oracle's share of one round for one (batch, kv head) pair: the k draft calls
-    and the verify rows of that pair, plus acceptance of that batch row.  Returns
-    (algorithmic bytes, seconds)."""
+    and the verify rows of that pair (acceptance is not included: it is per batch row,
+    not per pair, and negligible next to attention).  Returns (algorithmic bytes,
+    seconds)."""
     import oracle
     cfg = case["cfg"]
     f = oracle.bf16_to_f64
@@ -232,6 +233,19 @@ def cpu_model() -> str:
     return "unknown"
 
 
+def oracle_threads() -> int:
+    """Threads the oracle's NumPy runs on: the BLAS pool size (the same figure for the
+    GPU arm's baseline and the reference arm)."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n and max(n) > 0:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
 def cpu_baseline(case, budget_s: float = 20.0) -> dict:
     """The oracle, as it stands, on a bounded sample of the same workload."""
     cfg = case["cfg"]
@@ -246,8 +260,9 @@ def cpu_baseline(case, budget_s: float = 20.0) -> dict:
         n += 1
         if tot_t > budget_s:
             break
-    cores = max(1, round((time.process_time() - c0) / max(time.perf_counter() - w0, 1e-9)))
-    return {"value": tot_b / tot_t / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+    util = (time.process_time() - c0) / max(time.perf_counter() - w0, 1e-9)
+    return {"value": tot_b / tot_t / 1e9, "unit": "GB/s", "cores": oracle_threads(),
+            "cpu_utilisation": round(util, 2), "kind": "oracle",
             "cpu": cpu_model(), "host_cores": os.cpu_count(),
             "sample": f"{n} of {len(pairs)} (batch, kv head) pairs of one round: all {cfg.k} "
                       f"draft calls and the {cfg.k + 1} verify positions of each pair, fp64 "
@@ -272,7 +287,7 @@ def run_reference(args, world, rank, case=None):
         nb, dt = oracle_pair_sample(case, *pairs[(args.warmup + s) % len(pairs)])
         tot_b += nb
         tot_t += dt
-    cores = max(1, round((time.process_time() - c0) / max(time.perf_counter() - w0, 1e-9)))
+    util = (time.process_time() - c0) / max(time.perf_counter() - w0, 1e-9)
     value = tot_b / tot_t / 1e9
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
@@ -281,7 +296,8 @@ def run_reference(args, world, rank, case=None):
             "config": {"workload": cfg.name, "batch": cfg.B, "heads": f"{cfg.Hq}/{cfg.Hkv}",
                        "head_dim": cfg.D, "context": cfg.P, "slots": cfg.S, "draft_len": cfg.k,
                        "step": "one (batch, kv head) pair's share of a round"},
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle_threads(),
+                             "cpu_utilisation": round(util, 2), "kind": "oracle",
                              "cpu": cpu_model(), "host_cores": os.cpu_count(),
                              "sample": "each step: one (batch, kv head) pair's k draft calls "
                                        "and verify rows, fp64 NumPy"},
@@ -476,16 +492,11 @@ def run_config4(args) -> int:
     st = StagedVerify(host, cfg.P, bk, bv, n_slots=3)
     out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
     # drafting requests: 3 x 8 kv heads x 65536 compact slots, degrees 1..16
-    r = gen.children(cfg.seed + 200, 4)
     S = cfg.S
-    kc = b16(gen.f32_to_bf16_bits(gen.ar1(r[0], (cfg.n_draft_requests, cfg.Hkv), S, cfg.D,
-                                          cfg.rho))).to(dev)
-    vcc = b16(gen.f32_to_bf16_bits(gen.ar1(r[1], (cfg.n_draft_requests, cfg.Hkv), S, cfg.D,
-                                           cfg.rho))).to(dev)
-    deg = torch.from_numpy(gen.slot_degrees(r[2], (cfg.n_draft_requests, cfg.Hkv), S,
-                                            cfg.n_sinks, cfg.n_recent, cfg.deg_max)).to(dev)
-    dq = b16(gen.f32_to_bf16_bits(gen.normal(r[3], (cfg.n_draft_requests, cfg.Hq,
-                                                    cfg.D)))).to(dev)
+    dc = gen.staged_draft_case(cfg)
+    kc, vcc = b16(dc["kc_bits"]).to(dev), b16(dc["vc_bits"]).to(dev)
+    deg = torch.from_numpy(dc["deg"]).to(dev)
+    dq = b16(dc["q_bits"]).to(dev)
     dcache = vc.IndexedCache(k=kc, v=vcc, S=S, Hq=cfg.Hq, deg=deg)
     dws = torch.empty(vc.draft_workspace_size(dcache), dtype=torch.uint8, device=dev)
     dout = torch.empty_like(dq)

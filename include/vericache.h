@@ -149,7 +149,8 @@ vc_status vc_draft_attn(const void* q, const vc_comp_cache* cache, float scale, 
  *     with VC_ERR_UNSUPPORTED before anything is launched.
  *   - The first call on each device does a one-time set-up (it looks up the array's
  *     device address with that device current); make that first call before any stream
- *     capture begins.
+ *     capture begins.  The address is kept per CUDA context, so the set-up runs again
+ *     on the first call after a cudaDeviceReset or under another context.
  *   - All calls on a device share the one array and it keeps the last call's contents
  *     (nothing in it needs to start at zero).  Calls that overlap on the GPU -- on
  *     different streams, or from different threads -- race on it: serialise them. */
@@ -261,6 +262,18 @@ vc_status vc_csm_compress(const void* k, const void* v, const int32_t* deg, int 
  * resets it).  Bit 0: a bounded wait inside a verify-attention CTA expired (the call's
  * output is then invalid; the CTA released its resources and exited). */
 vc_status vc_device_error(int32_t* value, int clear);
+
+/* Failure detection (no counterpart in the pages).  Sets the time limit of every
+ * pipeline wait inside the verify-attention kernel for the launches that follow (a
+ * process-wide setting; default 2 s; seconds == 0 restores it; at most 60 s) and
+ * returns the previous limit in *previous (may be NULL).  A wait that runs out raises
+ * bit 0 of the device error word and the CTA exits cleanly, leaving the context usable;
+ * a very short limit makes that happen on purpose, which is how the error path is tested
+ * without any device fault.
+ * Staging has a host-side injection point for the same purpose: with the environment
+ * variable VC_FAULT_INJECT=stage_fail, vc_stage_full_kv returns VC_ERR_CUDA before
+ * enqueueing anything. */
+vc_status vc_set_wait_limit(double seconds, double* previous);
 
 #ifdef __cplusplus
 }

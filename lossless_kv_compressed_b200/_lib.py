@@ -21,8 +21,8 @@ EXPORTS = (
     "vc_status_string", "vc_last_error", "vc_abi_version",
     "vc_draft_workspace_size", "vc_draft_attn", "vc_draft_attn_noalloc",
     "vc_verify_workspace_size", "vc_verify_attn",
-    "vc_accept", "vc_stage_full_kv", "vc_event_wait", "vc_device_error",
-    "vc_csm_out_len", "vc_csm_compress",
+    "vc_accept", "vc_stage_full_kv", "vc_event_wait",
+    "vc_csm_out_len", "vc_csm_compress", "vc_device_error", "vc_set_wait_limit",
 )
 # Model glue of the end-to-end loop (include/vericache_glue.h).
 GLUE_EXPORTS = (
@@ -94,6 +94,8 @@ def lib() -> ctypes.CDLL:
         L.vc_event_wait.argtypes = [_p, ctypes.c_double]
         L.vc_device_error.restype = ctypes.c_int
         L.vc_device_error.argtypes = [ctypes.POINTER(_i32), ctypes.c_int]
+        L.vc_set_wait_limit.restype = ctypes.c_int
+        L.vc_set_wait_limit.argtypes = [ctypes.c_double, ctypes.POINTER(ctypes.c_double)]
         L.vc_csm_out_len.restype = _i64
         L.vc_csm_out_len.argtypes = [_i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_double]

@@ -275,6 +275,14 @@ def device_error(clear: bool = True) -> int:
     return int(v.value)
 
 
+def set_wait_limit(seconds: float) -> float:
+    """Time limit of the verify kernel's pipeline waits for the launches that follow
+    (0 restores the 2 s default); returns the previous limit in seconds."""
+    prev = ctypes.c_double(0.0)
+    check(lib().vc_set_wait_limit(float(seconds), ctypes.byref(prev)), "vc_set_wait_limit")
+    return float(prev.value)
+
+
 def csm_out_len(T: int, n_sinks: int, n_recent: int, chunk: int, r: float) -> int:
     """Rows left by one Chunked Soft Matching round over T rows (-1 if invalid)."""
     return int(lib().vc_csm_out_len(T, n_sinks, n_recent, chunk, r))

@@ -190,6 +190,15 @@ vc_status vc_event_wait(cudaEvent_t ev, double timeout_s) { return event_wait(ev
 
 vc_status vc_device_error(int32_t* value, int clear) { return read_device_error(value, clear); }
 
+vc_status vc_set_wait_limit(double seconds, double* previous) {
+  if (!(seconds >= 0.0 && seconds <= 60.0))
+    return fail(VC_ERR_INVALID, "wait limit must be in [0, 60] s (0 restores 2 s)");
+  const uint64_t ns = seconds == 0.0 ? kDefaultWaitNs : (uint64_t)(seconds * 1e9);
+  const uint64_t old = set_verify_wait_ns(ns < 1 ? 1 : ns);
+  if (previous) *previous = (double)old * 1e-9;
+  return VC_OK;
+}
+
 int64_t vc_csm_out_len(int64_t T, int n_sinks, int n_recent, int chunk, double r) {
   if (T < 0 || n_sinks < 0 || n_recent < 0 || (int64_t)n_sinks + n_recent > T || chunk < 2 ||
       chunk > 256 || !(r >= 0.0 && r <= 1.0))

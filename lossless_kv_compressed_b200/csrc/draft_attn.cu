@@ -1009,6 +1009,9 @@ vc_status launch_draft_int4(const void* q, const vc_comp_cache* c, float scale, 
 // attention with its split-K partials in the array below, which lives in the library's
 // own device image: every GPU that loads the library holds these bytes until the
 // process exits, and no call allocates anything.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 #include <vector>
 
@@ -1016,8 +1019,41 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = 8u << 20;   // 8 MiB per device
 static __device__ __align__(256) unsigned char g_draft_noalloc_scratch[kNoAllocScratchBytes];
 
+// Device address of the array, per CUDA context: a context is named by its unique id
+// (cuCtxGetId), which is never reused within the process, so a context created after a
+// cudaDeviceReset, or a non-primary context, gets its own look-up.
+struct NoAllocEntry {
+  int dev;
+  unsigned long long ctx_id;
+  void* ptr;
+};
 std::mutex g_noalloc_mu;
-std::vector<void*> g_noalloc_ptr;   // device address of the array, per device ordinal
+std::vector<NoAllocEntry> g_noalloc;
+
+// Id of the context current on this thread; 0 when none is current yet (the runtime
+// binds the device's primary context at its first call that needs one).
+bool current_ctx_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+  });
+  if (!get_cur || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS) return false;
+  *id = 0;
+  if (ctx && get_id(ctx, id) != CUDA_SUCCESS) return false;
+  return true;
+}
 }  // namespace
 
 extern "C" vc_status vc_draft_attn_noalloc(const void* q, const vc_comp_cache* cache,
@@ -1032,25 +1068,30 @@ extern "C" vc_status vc_draft_attn_noalloc(const void* q, const vc_comp_cache* c
                     "draft_noalloc: this cache needs %zu bytes of scratch, the fixed scratch "
                     "holds %zu (use vc_draft_attn with a caller workspace)",
                     need, kNoAllocScratchBytes);
-  // One-time set-up per device, with that device current: in host code the array's
-  // name is only a stand-in, so its device address is looked up once and kept.
+  // Set-up once per device and context, with that device current: in host code the
+  // array's name is only a stand-in, so its device address is looked up and kept.
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess)
     return vc::fail(VC_ERR_CUDA, "draft_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+  unsigned long long ctx = 0;
+  if (!current_ctx_id(&ctx))
+    return vc::fail(VC_ERR_CUDA, "draft_noalloc: cannot identify the current context");
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if ((int)g_noalloc_ptr.size() <= dev) g_noalloc_ptr.resize(dev + 1, nullptr);
-    if (!g_noalloc_ptr[dev]) {
-      void* p = nullptr;
-      e = cudaGetSymbolAddress(&p, g_draft_noalloc_scratch);
-      if (e != cudaSuccess || !p)
+    for (const NoAllocEntry& en : g_noalloc)
+      if (ctx != 0 && en.dev == dev && en.ctx_id == ctx) scratch = en.ptr;
+    if (!scratch) {
+      e = cudaGetSymbolAddress(&scratch, g_draft_noalloc_scratch);
+      if (e != cudaSuccess || !scratch)
         return vc::fail(VC_ERR_CUDA, "draft_noalloc: cudaGetSymbolAddress: %s",
                         cudaGetErrorString(e));
-      g_noalloc_ptr[dev] = p;
+      // the look-up bound the device's context if none was current: name it now
+      if (ctx == 0 && !current_ctx_id(&ctx))
+        return vc::fail(VC_ERR_CUDA, "draft_noalloc: cannot identify the current context");
+      if (ctx != 0) g_noalloc.push_back({dev, ctx, scratch});
     }
-    scratch = g_noalloc_ptr[dev];
   }
   // Nothing in the partials has to start at zero: every entry a call reads was written
   // earlier in the same call, so the previous call's leftovers are harmless.

@@ -9,14 +9,26 @@
 // call per chunk, no SM involved) on a caller-given side stream; an event after each
 // chunk lets the verify stream start on chunk i while chunk i+1 is in flight.
 #include <chrono>
+#include <cstdlib>
+#include <cstring>
 #include <thread>
 
 #include "vc_internal.h"
 
 namespace vc {
 
+// Host-side fault injection for failure-detection tests: with VC_FAULT_INJECT set to
+// "stage_fail" in the environment, every staging call fails as a failed copy would,
+// before anything is enqueued (no device work, no device fault).
+static bool inject_stage_failure() {
+  const char* e = std::getenv("VC_FAULT_INJECT");
+  return e != nullptr && std::strcmp(e, "stage_fail") == 0;
+}
+
 vc_status stage_full_kv(void* dst, const void* src, size_t bytes, size_t chunk,
                         cudaStream_t stream, cudaEvent_t* done, int n_events) {
+  if (inject_stage_failure())
+    return fail(VC_ERR_CUDA, "stage: injected copy failure (VC_FAULT_INJECT=stage_fail)");
   if (!dst || !src) return fail(VC_ERR_INVALID, "stage: null pointer");
   if (chunk == 0) return fail(VC_ERR_INVALID, "stage: chunk_bytes == 0");
   const size_t n_chunks = bytes == 0 ? 0 : (bytes + chunk - 1) / chunk;

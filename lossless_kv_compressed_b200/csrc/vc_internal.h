@@ -37,6 +37,8 @@ vc_status launch_verify(const void* q, int B, int n_q, int Hq, int Hkv, int D, c
                         void* out, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 vc_status read_device_error(int32_t* value, int clear);
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;   // 2 s
+uint64_t set_verify_wait_ns(uint64_t ns);            // returns the previous limit
 
 int64_t csm_out_len(int64_t T, int n_sinks, int n_recent, int chunk, double r);
 vc_status launch_csm(const void* k, const void* v, const int32_t* deg, int pairs, int D,

@@ -27,12 +27,16 @@
 //               TMEM is rescaled after the previous P.V), P written as bf16 into the
 //               M-tile's P columns once the previous P.V has read them.
 // TMEM columns: O0 [0,D), O1 [D,2D), S0, S1 (64 each), P0, P1 (32 each), Q0 (D/2).
-// Every mbarrier wait is bounded in time; on expiry the CTA raises the library's device
-// error word, releases TMEM and exits.
+// Every mbarrier wait is bounded in time (pipeline waits by a launch parameter, 2 s
+// unless vc_set_wait_limit changed it; teardown waits by 1 s); on expiry the CTA raises
+// the library's device error word, lets its copies and products in flight land,
+// releases TMEM and exits.
 // The split partials (max, sum, unnormalised O) are merged by a second kernel in
 // split order, optionally together with a carried state for chunked (streamed) keys.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+
+#include <atomic>
 
 #include "tc05.cuh"
 #include "vc_common.cuh"
@@ -56,6 +60,7 @@ struct VerifyParams {
   float qk_scale2;          // scale * log2(e)
   float* ws_o;              // [pairs, n_split, R, D]
   float* ws_ml;             // [pairs, n_split, R, 2]
+  uint64_t wait_ns;         // limit of every pipeline wait (teardown waits keep their own)
 };
 
 template <int D>
@@ -206,7 +211,7 @@ __global__ void __launch_bounds__(kVThreads, 1)
       int issued = 0;
       for (int t = 0; t < n_tiles; ++t) {
         const int st = t % kNSt;
-        if (t >= kNSt && !tc::mbar_wait(b_kv_empty(st), ((t / kNSt) - 1) & 1, abort_flag)) {
+        if (t >= kNSt && !tc::mbar_wait(b_kv_empty(st), ((t / kNSt) - 1) & 1, abort_flag, p.wait_ns)) {
           raise();
           break;
         }
@@ -258,7 +263,7 @@ __global__ void __launch_bounds__(kVThreads, 1)
                       tc::sdesc_sw128(bb, kBN * 128, 1024), id_pv, (t > 0 || ks > 0) ? 1u : 0u);
         }
       };
-      bool ok = tc::mbar_wait(b_kv_full(0), 0, abort_flag);
+      bool ok = tc::mbar_wait(b_kv_full(0), 0, abort_flag, p.wait_ns);
       if (ok) {
         tc::tc_fence_after();
         qk(0);
@@ -268,14 +273,14 @@ __global__ void __launch_bounds__(kVThreads, 1)
         if (t + 1 < n_tiles) {
           // the next Q K^T as soon as the softmax has copied this S out of TMEM
           if (!(ok = tc::mbar_wait(b_kv_full((t + 1) % kNSt), ((t + 1) / kNSt) & 1,
-                                   abort_flag)))
+                                   abort_flag, p.wait_ns)))
             break;
-          if (!(ok = tc::mbar_wait(b_s_free(mt), t & 1, abort_flag))) break;
+          if (!(ok = tc::mbar_wait(b_s_free(mt), t & 1, abort_flag, p.wait_ns))) break;
           tc::tc_fence_after();
           qk(t + 1);
           tc::umma_commit(b_s_full(mt));
         }
-        if (!(ok = tc::mbar_wait(b_p_full(mt), t & 1, abort_flag))) break;
+        if (!(ok = tc::mbar_wait(b_p_full(mt), t & 1, abort_flag, p.wait_ns))) break;
         tc::tc_fence_after();
         pv(t);
         tc::umma_commit(b_o_done(mt));
@@ -304,7 +309,7 @@ __global__ void __launch_bounds__(kVThreads, 1)
       float m_used = -INFINITY, lsum = 0.f;
       bool ok = true;
       for (int t = 0; t < n_tiles; ++t) {
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(b_s_full(mt), t & 1, abort_flag));
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(b_s_full(mt), t & 1, abort_flag, p.wait_ns));
         if (!ok) break;
         tc::tc_fence_after();
         uint32_t sr[64];
@@ -364,7 +369,7 @@ __global__ void __launch_bounds__(kVThreads, 1)
         }
         // the previous P.V must be done before O is rescaled or P overwritten
         if (t > 0) {
-          ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt), (t - 1) & 1, abort_flag));
+          ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt), (t - 1) & 1, abort_flag, p.wait_ns));
           if (!ok) break;
           tc::tc_fence_after();
         }
@@ -390,7 +395,7 @@ __global__ void __launch_bounds__(kVThreads, 1)
       }
       if (ok) {
         const int tl = n_tiles - 1;
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt), tl & 1, abort_flag));
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt), tl & 1, abort_flag, p.wait_ns));
       }
       if (!ok) {
         raise();
@@ -598,6 +603,11 @@ static vc_status run_verify(const Plan& pl, const VerifyParams& vp, const CUtens
   return VC_OK;
 }
 
+// Limit of the verify kernel's pipeline waits, for the launches that follow.
+static std::atomic<uint64_t> g_verify_wait_ns{kDefaultWaitNs};
+
+uint64_t set_verify_wait_ns(uint64_t ns) { return g_verify_wait_ns.exchange(ns); }
+
 vc_status launch_verify(const void* q, int B, int n_q, int Hq, int Hkv, int D, const void* k,
                         const void* v, int64_t L_cap, int64_t kv_start, int64_t kv_len,
                         int64_t P, float* m, float* l, float* acc, int flags, float scale,
@@ -624,6 +634,7 @@ vc_status launch_verify(const void* q, int B, int n_q, int Hq, int Hkv, int D, c
   vp.qk_scale2 = scale * kLog2e;
   vp.ws_o = static_cast<float*>(ws);
   vp.ws_ml = vp.ws_o + (size_t)pl.pairs * pl.n_split * pl.R * D;
+  vp.wait_ns = g_verify_wait_ns.load();
   if (D == 128) return run_verify<128>(pl, vp, mk, mv, flags, m, l, acc, out, stream);
   return run_verify<64>(pl, vp, mk, mv, flags, m, l, acc, out, stream);
 }

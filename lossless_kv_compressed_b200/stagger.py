@@ -54,14 +54,29 @@ class StagedVerify:
         self.t_staged = torch.cuda.Event(enable_timing=True)
         self.t_done = torch.cuda.Event(enable_timing=True)
         self.chunk_bytes = self.ring[0].numel() * self.ring.element_size()
+        self._launched = False
 
     def _rows(self, c: int) -> int:
         return min(self.chunk, self.P - c * self.chunk)
 
     def launch(self, q: torch.Tensor, out: torch.Tensor, state=None, ws=None):
         """Enqueue the whole staged verify of q [1, n_q, Hq, D] and return at once;
-        ``self.t_done`` completes when ``out`` is written."""
+        ``self.t_done`` completes when ``out`` is written (``wait()`` orders a stream
+        after it).
+
+        Ordering: both side streams first wait for the caller's current stream, so q,
+        the block's keys and anything else written there before this call are visible;
+        the first chunks of this launch reuse ring slots and events of the previous
+        launch, so its copies also wait for that launch's last verify (``t_done``)."""
         B, n_q, Hq, D = q.shape
+        current = torch.cuda.current_stream(self.device)
+        self.s_copy.wait_stream(current)
+        self.s_verify.wait_stream(current)
+        if self._launched:
+            # ring slots 0..n_slots-1 and the per-chunk events are about to be reused
+            self.s_copy.wait_event(self.t_done)
+            self.s_verify.wait_event(self.t_done)
+        self._launched = True
         if state is None:
             state = (torch.empty((B, n_q, Hq), dtype=torch.float32, device=self.device),
                      torch.empty((B, n_q, Hq), dtype=torch.float32, device=self.device),
@@ -101,6 +116,12 @@ class StagedVerify:
                     stream=self.s_verify)
         self.t_done.record(self.s_verify)
         return out
+
+    def wait(self, stream=None) -> None:
+        """Make ``stream`` (default: the current one) wait until the last launch's
+        output is written, without blocking the host."""
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        s.wait_event(self.t_done)
 
 
 def run_alongside(staged: StagedVerify, q, out, draft_step: Callable[[torch.cuda.Stream], None],

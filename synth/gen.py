@@ -238,3 +238,24 @@ def staged_case(cfg=None, chunk: int | None = None, P: int | None = None):
     out["block_v_bits"] = f32_to_bf16_bits(normal(r[3], (1, cfg.Hkv, n_q, cfg.D)))
     out["q_verify_bits"] = f32_to_bf16_bits(normal(r[4], (1, n_q, cfg.Hq, cfg.D)))
     return out
+
+
+def staged_draft_case(cfg=None, n_tail: int = 0) -> dict:
+    """Inputs of the requests that draft while the long-context request verifies: per
+    request and kv head a compact compressed cache of S rows (AR(1) along the rows, as
+    the full caches), degrees U{1..deg_max} on the kept middle rows, one query per
+    query head, and ``n_tail`` i.i.d. N(0, 1) tail rows (the drafts appended so far).
+    Returns bits: kc_bits, vc_bits [R, Hkv, S, D], deg [R, Hkv, S], q_bits [R, Hq, D],
+    tail_k_bits, tail_v_bits [R, Hkv, max(n_tail, 1), D]."""
+    cfg = cfg or get_config(4)
+    R, S = cfg.n_draft_requests, cfg.S
+    r = children(cfg.seed + 200, 6)
+    out = {"cfg": cfg, "n_tail": n_tail}
+    out["kc_bits"] = f32_to_bf16_bits(ar1(r[0], (R, cfg.Hkv), S, cfg.D, cfg.rho))
+    out["vc_bits"] = f32_to_bf16_bits(ar1(r[1], (R, cfg.Hkv), S, cfg.D, cfg.rho))
+    out["deg"] = slot_degrees(r[2], (R, cfg.Hkv), S, cfg.n_sinks, cfg.n_recent, cfg.deg_max)
+    out["q_bits"] = f32_to_bf16_bits(normal(r[3], (R, cfg.Hq, cfg.D)))
+    nt = max(n_tail, 1)
+    out["tail_k_bits"] = f32_to_bf16_bits(normal(r[4], (R, cfg.Hkv, nt, cfg.D)))
+    out["tail_v_bits"] = f32_to_bf16_bits(normal(r[5], (R, cfg.Hkv, nt, cfg.D)))
+    return out

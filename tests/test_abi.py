@@ -121,3 +121,29 @@ def test_csm_rejects_bad_arguments(kw, status):
                            a["dest"] or None, None)
     assert st == status, _lib.status_name(st)
     assert vc.lib().vc_last_error()
+
+
+def test_stage_fault_injection_fails_before_any_cuda_call(monkeypatch):
+    """VC_FAULT_INJECT=stage_fail: the staging call reports a copy failure before it
+    enqueues anything (here on a host with no GPU, where any CUDA call would fail
+    differently), and works normally once the variable is cleared."""
+    L = vc.lib()
+    monkeypatch.setenv("VC_FAULT_INJECT", "stage_fail")
+    assert L.vc_stage_full_kv(1 << 20, 1 << 20, 100, 10, None, None, 0) == _lib.VC_ERR_CUDA
+    assert b"injected" in L.vc_last_error()
+    monkeypatch.setenv("VC_FAULT_INJECT", "something_else")
+    assert L.vc_stage_full_kv(None, 1 << 20, 100, 10, None, None, 0) == _lib.VC_ERR_INVALID
+    monkeypatch.delenv("VC_FAULT_INJECT")
+    assert L.vc_stage_full_kv(None, 1 << 20, 100, 10, None, None, 0) == _lib.VC_ERR_INVALID
+
+
+def test_wait_limit_setting():
+    prev = ctypes.c_double(-1.0)
+    L = vc.lib()
+    assert L.vc_set_wait_limit(-1.0, None) == _lib.VC_ERR_INVALID
+    assert L.vc_set_wait_limit(61.0, None) == _lib.VC_ERR_INVALID
+    assert L.vc_set_wait_limit(float("nan"), None) == _lib.VC_ERR_INVALID
+    assert L.vc_set_wait_limit(0.5, ctypes.byref(prev)) == _lib.VC_OK
+    assert prev.value == pytest.approx(2.0)
+    assert vc.set_wait_limit(0.0) == pytest.approx(0.5)     # 0 restores the default
+    assert vc.set_wait_limit(0.0) == pytest.approx(2.0)

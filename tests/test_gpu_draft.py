@@ -109,3 +109,33 @@ def test_deterministic_across_calls(case2):
     b = vc.draft_attn(q, cache)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+def test_long_context_drafters_65536_compact_slots():
+    """The drafting requests of the 1M-token staggered workload at their own shapes:
+    3 requests x 64/8 heads (g = 8), D 128, 65536 compact slots each (idx = NULL),
+    degrees 1..16, plus a 17-row bf16 tail; every head of every request against the
+    oracle (one request at a time, to bound host memory)."""
+    from synth.configs import get_config
+    cfg = get_config(4)
+    n_tail = 17
+    dc = gen.staged_draft_case(cfg, n_tail=n_tail)
+    cache = vc.IndexedCache(
+        k=dev_bf16(dc["kc_bits"]), v=dev_bf16(dc["vc_bits"]), S=cfg.S, Hq=cfg.Hq,
+        deg=dev_i32(dc["deg"]), k_tail=dev_bf16(dc["tail_k_bits"]),
+        v_tail=dev_bf16(dc["tail_v_bits"]), n_tail=n_tail,
+        err_flag=torch.zeros(1, dtype=torch.int32, device="cuda"))
+    q = dev_bf16(dc["q_bits"])
+    lse = torch.empty((cfg.n_draft_requests, cfg.Hq), dtype=torch.float32, device="cuda")
+    out = both_outputs(lambda dt: vc.draft_attn(q, cache, lse=lse, out=torch.empty(
+        q.shape, dtype=dt, device="cuda")))
+    assert int(cache.err_flag.item()) == 0
+    got, got_lse = host_f64(out), host_f64(lse)
+    f = oracle.bf16_to_f64
+    for r in range(cfg.n_draft_requests):
+        s = slice(r, r + 1)
+        o_ref, lse_ref = oracle.draft_attn(f(dc["q_bits"][s]), f(dc["kc_bits"][s]),
+                                           f(dc["vc_bits"][s]), cfg.S, None, dc["deg"][s],
+                                           f(dc["tail_k_bits"][s]), f(dc["tail_v_bits"][s]))
+        assert_close_attn(got[s], o_ref, f"65536-slot drafter {r}")
+        np.testing.assert_allclose(got_lse[s], lse_ref, atol=2e-3, rtol=0)

@@ -153,3 +153,34 @@ def test_32k_context_sampled_rows(case2):
         want = oracle.verify_attn(f(q_bits[b:b + 1, i:i + 1]), f(case2["k_bits"][b:b + 1, :, :P_i + 1]),
                                   f(case2["v_bits"][b:b + 1, :, :P_i + 1]), P_i)
         assert_close_attn(got[b:b + 1, i:i + 1], want, f"32K context b={b} i={i}")
+
+
+def test_device_resident_1m_context_sampled_rows():
+    """The long-context workload's verify with the whole full cache resident in HBM:
+    P = 1,048,576 keys plus the 41-row block, 64/8 heads, D 128 (2.1 GB per K or V
+    tensor, so byte offsets run past 2^31).  The inputs are generated and uploaded in
+    64K-token chunks; the oracle follows the chunks for rows 0, 20 and 40 on kv heads
+    0 and 7."""
+    from synth.configs import get_config
+    from tests.long_context import walk_chunks
+    cfg = get_config(4)
+    P, n_q = cfg.P, cfg.k + 1
+    case = gen.staged_case(cfg, chunk=cfg.chunk_tokens, P=P)
+    K = torch.empty((1, cfg.Hkv, P + n_q, cfg.D), dtype=torch.bfloat16, device="cuda")
+    V = torch.empty_like(K)
+
+    def upload(kb, vb, s0):
+        n = kb.shape[1]
+        K[0, :, s0:s0 + n] = dev_bf16(kb)
+        V[0, :, s0:s0 + n] = dev_bf16(vb)
+
+    want = walk_chunks(case, (0, 20, 40), (0, 7), upload)
+    K[0, :, P:] = dev_bf16(case["block_k_bits"][0])
+    V[0, :, P:] = dev_bf16(case["block_v_bits"][0])
+    q = dev_bf16(case["q_verify_bits"])
+    out = vc.verify_attn(q, K, V, P, out=torch.empty(q.shape, dtype=torch.float32, device="cuda"))
+    torch.cuda.synchronize()
+    got = host_f64(out)
+    g = cfg.g
+    for (i, j), w in want.items():
+        assert_close_attn(got[0, i, j * g:(j + 1) * g], w, f"1M context row {i} kv head {j}")

@@ -3,9 +3,10 @@ scratch memory (for example a plugin whose host runtime owns all device memory, 
 path that must not call cudaMalloc).  It keeps its split-K partials in a fixed 8 MiB
 array inside the library, so the caller passes only inputs and outputs.
 
-The test calls it through the C ABI twice in a row on different problems (the second
-call runs over whatever the first left in the shared array) and compares each result
-with the ordinary vc_draft_attn, which uses a caller-allocated workspace.  It also
+The test calls it through the C ABI three times in a row on different problems (each
+call runs over whatever the one before left in the shared array; the third is a 4-bit
+cache with a bf16 tail, whose partials fill the array as two sets) and compares each
+result with the ordinary vc_draft_attn, which uses a caller-allocated workspace.  It also
 checks that a problem too big for the fixed array is refused before anything runs.
 """
 import ctypes
@@ -17,7 +18,7 @@ import torch
 import lossless_kv_compressed_b200 as vc
 from lossless_kv_compressed_b200._lib import CompCache, lib
 from synth import gen
-from tests.gpu_util import assert_close_attn, dev_bf16, dev_i32, host_f64
+from tests.gpu_util import assert_close_attn, dev_bf16, dev_f16, dev_i32, dev_u32, host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -46,14 +47,32 @@ def _with_workspace(q, cache):
     return vc.draft_attn(q, cache, out=torch.empty(q.shape, dtype=torch.float32, device="cuda"))
 
 
-def test_two_calls_in_a_row_match_the_workspace_entry_point():
+def _int4_problem(n_tail):
+    """A small 4-bit cache (1024 quantised tokens per pair) with a bf16 tail: its partials
+    fill the fixed array as two sets, the quantised blocks' then the tail's."""
+    from tests.test_gpu_draft_int4 import _quantised
+    case = gen.attn_case(3, B=2, P=1024 + 64, k=4, vocab=0)
+    cfg, T_q = case["cfg"], 1024
+    qz = _quantised(case, T_q)
+    cache = vc.Int4Cache(
+        kq=dev_u32(qz["kq"]), k_scale=dev_f16(qz["sk"]), k_zero=dev_f16(qz["zk"]),
+        vq=dev_u32(qz["vq"]), v_scale=dev_f16(qz["vs"]), v_zero=dev_f16(qz["vz"]), S=T_q,
+        Hq=cfg.Hq, k_tail=dev_bf16(case["k_bits"][:, :, T_q:T_q + n_tail]),
+        v_tail=dev_bf16(case["v_bits"][:, :, T_q:T_q + n_tail]), n_tail=n_tail)
+    return dev_bf16(case["q_draft_bits"]), cache
+
+
+def test_calls_in_a_row_match_the_workspace_entry_point():
     first = _problem(gen.attn_case(2, B=4, P=8192, S=3000, n_recent=128), 17)
     second = _problem(gen.attn_case(1), 5)
-    got = [_noalloc(*first), _noalloc(*second)]
+    third = _int4_problem(19)
+    problems = (first, second, third)
+    assert all(vc.draft_workspace_size(c) <= (8 << 20) for _, c in problems)
+    got = [_noalloc(*p) for p in problems]
     torch.cuda.synchronize()
-    want = [_with_workspace(*first), _with_workspace(*second)]
+    want = [_with_workspace(*p) for p in problems]
     torch.cuda.synchronize()
-    for g, w, name in zip(got, want, ("first call", "second call")):
+    for g, w, name in zip(got, want, ("first call", "second call", "third call (int4)")):
         assert_close_attn(host_f64(g), host_f64(w), name)
 
 
