@@ -258,6 +258,59 @@ vc_status vc_csm_compress(const void* k, const void* v, const int32_t* deg, int 
                           double r, void* k_out, void* v_out, int32_t* deg_out,
                           int64_t T_cap_out, int32_t* dest, cudaStream_t stream);
 
+/* ----------------------------------------------------------------------------
+ * Int4 compressor: quantise whole 32-token blocks of bf16 K/V rows into the
+ * VC_CACHE_INT4 layout above ([VC] "Supporto Architetturale": quantisation plugs into
+ * the uniform compression interface; [CKV] "Problematica": quantisation among the known
+ * KV-cache reductions).  Groups as in the layout: keys per channel over the block's 32
+ * tokens, values per token over 32 consecutive channels;
+ *     z = fp16(min), s = fp16((max - min) / 15) (1 if that is 0),
+ *     n = clamp(rint((x - z) / s), 0, 15), round half to even, in fp64.
+ * This is how tokens leaving a bf16 window join the quantised part of the cache: call it
+ * on each 32 rows that leave, with blk0 = the next free block.
+ *   k, v      bf16 [pairs, src_cap, D]; rows src_t0 .. src_t0 + 32 n_blocks - 1 of every
+ *             pair are read
+ *   kq, k_scale, k_zero, vq, v_scale, v_zero: the int4 arrays with capacity blk_cap
+ *             blocks per pair (T_cap = 32 blk_cap); blocks blk0 .. blk0 + n_blocks - 1
+ *             of every pair are written, nothing else
+ *   D in {64, 128}; pairs <= 65535; pointers (and row src_t0) 16-byte aligned.
+ *   Groups with values beyond the fp16 range cannot be represented (result unspecified).
+ * ---------------------------------------------------------------------------- */
+vc_status vc_int4_quantize(const void* k, const void* v, int pairs, int D, int64_t src_cap,
+                           int64_t src_t0, int n_blocks, uint32_t* kq, void* k_scale,
+                           void* k_zero, uint32_t* vq, void* v_scale, void* v_zero,
+                           int64_t blk_cap, int64_t blk0, cudaStream_t stream);
+
+/* ----------------------------------------------------------------------------
+ * Token eviction by attention score ([CKV] "Problematica": eviction drops the tokens
+ * with the lowest attention scores; [CKV] "Metodologia" item 2 "Preservazione": sinks and
+ * recent tokens are always kept; [VC] "Supporto Architetturale": eviction compressors
+ * plug into the same interface).
+ *
+ * vc_evict_scores: for a prompt of n tokens, the attention mass each key receives from
+ * the last W prompt queries over the g query heads of its kv head:
+ *     score[b, j, t] = sum_{w < W, h in group j} softmax_{t' <= n-W+w}(q . k_t' * scale)[t]
+ *   q      bf16 [B, W, Hq, D]: the queries of positions n-W .. n-1 (as attention sees
+ *          them, i.e. after any rotary embedding)
+ *   k      bf16 [B, Hkv, L_cap, D]: keys of positions 0 .. n-1 in rows 0 .. n-1
+ *   score  fp32 [B, Hkv, score_cap], entries [0, n) written (each a fixed-order fp32 sum)
+ *   ws     device workspace of vc_evict_workspace_size(B, W, Hq) bytes
+ *   scale <= 0 selects D^-1/2.  D in {64, 128}, g <= 8, W <= 32, W <= n <= L_cap.
+ *
+ * vc_evict_select: per row r (e.g. (batch, kv head)) of score [rows, score_cap], the kept
+ * positions in ascending order: [0, n_sinks), then the budget - n_sinks - n_recent
+ * highest-scoring positions of [n_sinks, n - n_recent) (equal scores: the lower position
+ * first), then [n - n_recent, n); budget >= n keeps 0 .. n-1.  Writes idx int32
+ * [rows, S_cap], entries [0, min(budget, n)).  Exact: depends only on the scores' order.
+ * ---------------------------------------------------------------------------- */
+size_t vc_evict_workspace_size(int B, int W, int Hq);
+vc_status vc_evict_scores(const void* q, int B, int W, int Hq, int Hkv, int D, const void* k,
+                          int64_t L_cap, int64_t n, float scale, float* score,
+                          int64_t score_cap, void* ws, size_t ws_bytes, cudaStream_t stream);
+vc_status vc_evict_select(const float* score, int rows, int64_t score_cap, int64_t n,
+                          int budget, int n_sinks, int n_recent, int32_t* idx, int64_t S_cap,
+                          cudaStream_t stream);
+
 /* The library's device error word on the current device (synchronous read; clear != 0
  * resets it).  Bit 0: a bounded wait inside a verify-attention CTA expired (the call's
  * output is then invalid; the CTA released its resources and exited). */

@@ -22,7 +22,8 @@ EXPORTS = (
     "vc_draft_workspace_size", "vc_draft_attn", "vc_draft_attn_noalloc",
     "vc_verify_workspace_size", "vc_verify_attn",
     "vc_accept", "vc_stage_full_kv", "vc_event_wait",
-    "vc_csm_out_len", "vc_csm_compress", "vc_device_error", "vc_set_wait_limit",
+    "vc_csm_out_len", "vc_csm_compress", "vc_int4_quantize", "vc_evict_workspace_size",
+    "vc_evict_scores", "vc_evict_select", "vc_device_error", "vc_set_wait_limit",
 )
 # Model glue of the end-to-end loop (include/vericache_glue.h).
 GLUE_EXPORTS = (
@@ -94,6 +95,17 @@ def lib() -> ctypes.CDLL:
         L.vc_event_wait.argtypes = [_p, ctypes.c_double]
         L.vc_device_error.restype = ctypes.c_int
         L.vc_device_error.argtypes = [ctypes.POINTER(_i32), ctypes.c_int]
+        L.vc_int4_quantize.restype = ctypes.c_int
+        L.vc_int4_quantize.argtypes = ([_p, _p, ctypes.c_int, ctypes.c_int, _i64, _i64,
+                                        ctypes.c_int] + [_p] * 6 + [_i64, _i64, _p])
+        L.vc_evict_workspace_size.restype = _sz
+        L.vc_evict_workspace_size.argtypes = [ctypes.c_int] * 3
+        L.vc_evict_scores.restype = ctypes.c_int
+        L.vc_evict_scores.argtypes = ([_p] + [ctypes.c_int] * 5 + [_p, _i64, _i64, ctypes.c_float,
+                                                                   _p, _i64, _p, _sz, _p])
+        L.vc_evict_select.restype = ctypes.c_int
+        L.vc_evict_select.argtypes = [_p, ctypes.c_int, _i64, _i64, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, _p, _i64, _p]
         L.vc_set_wait_limit.restype = ctypes.c_int
         L.vc_set_wait_limit.argtypes = [ctypes.c_double, ctypes.POINTER(ctypes.c_double)]
         L.vc_csm_out_len.restype = _i64

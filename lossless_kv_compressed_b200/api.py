@@ -275,6 +275,69 @@ def device_error(clear: bool = True) -> int:
     return int(v.value)
 
 
+def int4_quantize(k: torch.Tensor, v: torch.Tensor, cache: "Int4Cache", n_blocks: int,
+                  src_t0: int = 0, blk0: int = 0, stream=None) -> None:
+    """Quantise rows [src_t0, src_t0 + 32 n_blocks) of k, v [B, Hkv, src_cap, D] (bf16)
+    into blocks [blk0, blk0 + n_blocks) of every pair of ``cache``'s int4 arrays."""
+    _need(k, torch.bfloat16, "k")
+    _need(v, torch.bfloat16, "v")
+    B, Hkv, src_cap, D = k.shape
+    blk_cap = cache.k_scale.shape[2]
+    check(lib().vc_int4_quantize(k.data_ptr(), v.data_ptr(), B * Hkv, D, src_cap, src_t0,
+                                 n_blocks, cache.kq.data_ptr(), cache.k_scale.data_ptr(),
+                                 cache.k_zero.data_ptr(), cache.vq.data_ptr(),
+                                 cache.v_scale.data_ptr(), cache.v_zero.data_ptr(), blk_cap,
+                                 blk0, _stream(stream)), "vc_int4_quantize")
+
+
+def empty_int4_cache(B: int, Hq: int, Hkv: int, D: int, T_cap: int, device="cuda") -> "Int4Cache":
+    """Uninitialised int4 arrays for T_cap tokens per pair (S = 0 live tokens)."""
+    nb = T_cap // 32
+    i32, f16 = dict(dtype=torch.int32, device=device), dict(dtype=torch.float16, device=device)
+    return Int4Cache(kq=torch.empty((B, Hkv, nb, 32, 4, D // 32), **i32),
+                     k_scale=torch.empty((B, Hkv, nb, D), **f16),
+                     k_zero=torch.empty((B, Hkv, nb, D), **f16),
+                     vq=torch.empty((B, Hkv, nb, D, 4), **i32),
+                     v_scale=torch.empty((B, Hkv, nb, D // 32, 32), **f16),
+                     v_zero=torch.empty((B, Hkv, nb, D // 32, 32), **f16), S=0, Hq=Hq)
+
+
+def evict_scores(q: torch.Tensor, k: torch.Tensor, n: int, score: Optional[torch.Tensor] = None,
+                 ws: Optional[torch.Tensor] = None, scale: float = 0.0, stream=None) -> torch.Tensor:
+    """Attention mass per key from the last W prompt queries q [B, W, Hq, D] over keys
+    [0, n) of k [B, Hkv, L_cap, D]; returns score fp32 [B, Hkv, >= n]."""
+    _need(q, torch.bfloat16, "q")
+    _need(k, torch.bfloat16, "k")
+    B, W, Hq, D = q.shape
+    Hkv, L_cap = k.shape[1], k.shape[2]
+    if score is None:
+        score = torch.empty((B, Hkv, n), dtype=torch.float32, device=q.device)
+    _need(score, torch.float32, "score")
+    if ws is None:
+        ws = torch.empty(int(lib().vc_evict_workspace_size(B, W, Hq)), dtype=torch.uint8,
+                         device=q.device)
+    check(lib().vc_evict_scores(q.data_ptr(), B, W, Hq, Hkv, D, k.data_ptr(), L_cap, n,
+                                float(scale), score.data_ptr(), score.shape[-1], ws.data_ptr(),
+                                ws.numel(), _stream(stream)), "vc_evict_scores")
+    return score
+
+
+def evict_select(score: torch.Tensor, n: int, budget: int, n_sinks: int, n_recent: int,
+                 idx: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Kept positions (ascending) per row of score [..., score_cap]: sinks, the top
+    middle scores (ties to the lower position) up to the budget, the recent window."""
+    _need(score, torch.float32, "score")
+    rows = score.numel() // score.shape[-1]
+    if idx is None:
+        idx = torch.empty(score.shape[:-1] + (min(budget, n),), dtype=torch.int32,
+                          device=score.device)
+    _need(idx, torch.int32, "idx")
+    check(lib().vc_evict_select(score.data_ptr(), rows, score.shape[-1], n, budget, n_sinks,
+                                n_recent, idx.data_ptr(), idx.shape[-1], _stream(stream)),
+          "vc_evict_select")
+    return idx
+
+
 def set_wait_limit(seconds: float) -> float:
     """Time limit of the verify kernel's pipeline waits for the launches that follow
     (0 restores the 2 s default); returns the previous limit in seconds."""

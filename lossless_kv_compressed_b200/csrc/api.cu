@@ -227,4 +227,66 @@ vc_status vc_csm_compress(const void* k, const void* v, const int32_t* deg, int 
                     deg_out, T_cap_out, dest, stream);
 }
 
+vc_status vc_int4_quantize(const void* k, const void* v, int pairs, int D, int64_t src_cap,
+                           int64_t src_t0, int n_blocks, uint32_t* kq, void* k_scale,
+                           void* k_zero, uint32_t* vq, void* v_scale, void* v_zero,
+                           int64_t blk_cap, int64_t blk0, cudaStream_t stream) {
+  if (pairs <= 0 || pairs > 65535) return fail(VC_ERR_INVALID, "quantize: pairs");
+  if (D != 64 && D != 128) return fail(VC_ERR_UNSUPPORTED, "quantize: D must be 64 or 128");
+  if (n_blocks < 0 || src_t0 < 0 || blk0 < 0 || src_t0 + 32 * (int64_t)n_blocks > src_cap ||
+      blk0 + n_blocks > blk_cap)
+    return fail(VC_ERR_INVALID, "quantize: block range outside the source or the cache");
+  if (!k || !v || !kq || !k_scale || !k_zero || !vq || !v_scale || !v_zero)
+    return fail(VC_ERR_INVALID, "quantize: NULL pointer");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(kq) || !aligned16(vq) ||
+      !aligned16(k_scale) || !aligned16(k_zero) || !aligned16(v_scale) || !aligned16(v_zero))
+    return fail(VC_ERR_INVALID, "quantize: misaligned pointer");
+  if (((src_t0 * D * 2) & 15) != 0) return fail(VC_ERR_INVALID, "quantize: src_t0 misaligned");
+  return launch_int4_quantize(k, v, pairs, D, src_cap, src_t0, n_blocks, kq, k_scale, k_zero,
+                              vq, v_scale, v_zero, blk_cap, blk0, stream);
+}
+
+size_t vc_evict_workspace_size(int B, int W, int Hq) {
+  if (B <= 0 || W <= 0 || Hq <= 0) return 0;
+  return (size_t)B * W * Hq * sizeof(float) + 256;
+}
+
+vc_status vc_evict_scores(const void* q, int B, int W, int Hq, int Hkv, int D, const void* k,
+                          int64_t L_cap, int64_t n, float scale, float* score,
+                          int64_t score_cap, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (B <= 0 || W <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv)
+    return fail(VC_ERR_INVALID, "evict_scores: sizes");
+  if (D != 64 && D != 128) return fail(VC_ERR_UNSUPPORTED, "evict_scores: D must be 64 or 128");
+  if (Hq / Hkv > 8) return fail(VC_ERR_UNSUPPORTED, "evict_scores: g > 8");
+  if (W > 32) return fail(VC_ERR_UNSUPPORTED, "evict_scores: W > 32");
+  if (n < W || n > L_cap || n > score_cap || (int64_t)B * Hkv > 65535)
+    return fail(VC_ERR_INVALID, "evict_scores: need W <= n <= L_cap, n <= score_cap");
+  if (!q || !k || !score || !ws) return fail(VC_ERR_INVALID, "evict_scores: NULL pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(ws))
+    return fail(VC_ERR_INVALID, "evict_scores: misaligned pointer");
+  if (ws_bytes < (size_t)B * W * Hq * sizeof(float))
+    return fail(VC_ERR_INVALID, "evict_scores: workspace too small");
+  if (scale <= 0.f) scale = 1.0f / sqrtf((float)D);
+  return launch_evict_scores(q, B, W, Hq, Hkv, D, k, L_cap, n, scale, score, score_cap,
+                             static_cast<float*>(ws), stream);
+}
+
+vc_status vc_evict_select(const float* score, int rows, int64_t score_cap, int64_t n,
+                          int budget, int n_sinks, int n_recent, int32_t* idx, int64_t S_cap,
+                          cudaStream_t stream) {
+  if (rows <= 0 || n <= 0 || n > score_cap || n >= ((int64_t)1 << 31))
+    return fail(VC_ERR_INVALID, "evict_select: sizes");
+  if (n_sinks < 0 || n_recent < 0 || budget < 1)
+    return fail(VC_ERR_INVALID, "evict_select: budget, n_sinks, n_recent");
+  if ((int64_t)budget < n && (int64_t)n_sinks + n_recent > budget)
+    return fail(VC_ERR_INVALID, "evict_select: sinks + recent exceed the budget");
+  if ((int64_t)budget < n && (int64_t)n_sinks + n_recent > n)
+    return fail(VC_ERR_INVALID, "evict_select: sinks + recent exceed n");
+  if (S_cap < ((int64_t)budget < n ? (int64_t)budget : n))
+    return fail(VC_ERR_INVALID, "evict_select: S_cap too small");
+  if (!score || !idx) return fail(VC_ERR_INVALID, "evict_select: NULL pointer");
+  return launch_evict_select(score, rows, score_cap, n, budget, n_sinks, n_recent, idx, S_cap,
+                             stream);
+}
+
 }  // extern "C"

@@ -30,6 +30,16 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
   return ok != 0;
 }
+// Same test with an explicit bound on how long the thread may stay suspended in the
+// instruction (the hardware wakes it earlier when the phase completes).
+__device__ __forceinline__ bool mbar_try_for(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(bar), "r"(parity), "r"(hint_ns) : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -38,17 +48,18 @@ __device__ __forceinline__ uint64_t globaltimer() {
 
 // Bounded wait: returns false after ~limit_ns of wall time or once *abort is set
 // by another role of the CTA (so one stuck role cannot hang the others).  abort may be
-// null (teardown waits that must not be cut short by the flag).
+// null (teardown waits that must not be cut short by the flag).  Each test suspends the
+// thread for at most min(limit_ns, 1 ms), so the limit and the flag are checked at least
+// that often whatever the hardware's own suspend time.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns = 2000000000ull) {
-  if (mbar_try(bar, parity)) return true;
+  const uint32_t hint = limit_ns < 1000000ull ? (uint32_t)limit_ns : 1000000u;
+  if (mbar_try_for(bar, parity, hint)) return true;
   const uint64_t t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (abort != nullptr && *abort) return false;
-      if (globaltimer() - t0 > limit_ns) return false;
-    }
+  for (;;) {
+    if (mbar_try_for(bar, parity, hint)) return true;
+    if (abort != nullptr && *abort) return false;
+    if (globaltimer() - t0 > limit_ns) return false;
   }
 }
 

@@ -46,6 +46,18 @@ vc_status launch_csm(const void* k, const void* v, const int32_t* deg, int pairs
                      void* k_out, void* v_out, int32_t* deg_out, int64_t T_cap_out,
                      int32_t* dest, cudaStream_t stream);
 
+vc_status launch_int4_quantize(const void* k, const void* v, int pairs, int D, int64_t src_cap,
+                               int64_t src_t0, int n_blocks, uint32_t* kq, void* k_scale,
+                               void* k_zero, uint32_t* vq, void* v_scale, void* v_zero,
+                               int64_t blk_cap, int64_t blk0, cudaStream_t stream);
+
+vc_status launch_evict_scores(const void* q, int B, int W, int Hq, int Hkv, int D,
+                              const void* k, int64_t L_cap, int64_t n, float scale,
+                              float* score, int64_t score_cap, float* ws, cudaStream_t stream);
+vc_status launch_evict_select(const float* score, int rows, int64_t score_cap, int64_t n,
+                              int budget, int n_sinks, int n_recent, int32_t* idx,
+                              int64_t S_cap, cudaStream_t stream);
+
 vc_status launch_accept(const float* logits, const int32_t* drafts, int B, int n_q, int V,
                         int32_t* target, int32_t* accept_len, int32_t* commit,
                         int32_t* n_commit, int32_t* err_flag, cudaStream_t stream);

@@ -13,7 +13,8 @@ embedding, RMSNorm, fused QKV / O / gate-up / down / LM-head GEMMs, RoPE with th
 store and SwiGLU; vc_draft_attn / vc_verify_attn / vc_accept for the method.  Token ids
 stay on the device between draft steps (each argmax is written straight into the next
 step's input); the host reads back only the accepted length and the commits, once per
-round.  Eviction scores after the prefill are computed with torch (set-up, not timed).
+round.  Eviction after the prefill (attention-mass scores of the last prompt queries and
+the top-budget selection) runs in the library too.
 
 Readings (same as the fp64 oracle in oracle/tinylm.py): k+1 verify rows (pending token +
 k drafts); on a disagreement the full-KV prediction is committed as the correction; the
@@ -28,7 +29,8 @@ import numpy as np
 import torch
 
 from . import _lib
-from .api import IndexedCache, accept, draft_attn, draft_workspace_size, verify_attn
+from .api import (IndexedCache, accept, draft_attn, draft_workspace_size, evict_scores,
+                  evict_select, verify_attn)
 from ._lib import check, lib
 
 
@@ -160,33 +162,16 @@ class GpuTinyLM:
         return logits[n - 1:n]
 
     def evict(self, n: int, budget: int, n_sinks: int, n_recent: int):
-        """Set-up: per layer and kv head keep sinks, the recent window and the middle
-        positions with the highest attention mass from the last prompt queries (ties to
-        the lower position); positions ascending, degree 1."""
+        """Per layer and kv head keep sinks, the recent window and the middle positions
+        with the highest attention mass from the last prompt queries (ties to the lower
+        position); positions ascending, degree 1.  Scores and selection run in the
+        library (vc_evict_scores, vc_evict_select)."""
         c = self.cfg
-        g = c.Hq // c.Hkv
         for l in range(c.n_layers):
-            q = self.qlast[l].float()                         # [W, Hq, D]
-            Wn = q.shape[0]
-            K = self.K[l][0, :, :n].float()                   # [Hkv, n, D]
-            sc = torch.einsum("whd,htd->hwt", q, K.repeat_interleave(g, 0)) / (c.D ** 0.5)
-            qpos = torch.arange(n - Wn, n, device=self.dev)
-            mask = torch.arange(n, device=self.dev)[None, :] <= qpos[:, None]
-            sc = sc.masked_fill(~mask[None], float("-inf")).softmax(-1)
-            score = sc.sum(1).view(c.Hkv, g, n).sum(1)        # [Hkv, n]
-            lo, hi = n_sinks, n - n_recent
-            take = budget - n_sinks - n_recent
-            for j in range(c.Hkv):
-                mid = score[j, lo:hi].double().cpu().numpy()
-                pos = np.arange(lo, hi)
-                order = np.lexsort((pos, -mid))[:take]
-                kept = np.concatenate([np.arange(n_sinks), np.sort(pos[order]),
-                                       np.arange(hi, n)]).astype(np.int32)
-                self.idx[l][0, j, :len(kept)] = torch.from_numpy(kept).to(self.dev)
-        self.S = budget if budget < n else n
-        if budget >= n:
-            for l in range(c.n_layers):
-                self.idx[l][0, :, :n] = self.arange[:n]
+            q = self.qlast[l].view(1, *self.qlast[l].shape)      # [1, W, Hq, D]
+            score = evict_scores(q, self.K[l], n)
+            evict_select(score, n, budget, n_sinks, n_recent, idx=self.idx[l])
+        self.S = min(budget, n)
 
 
 def greedy_loop(model: GpuTinyLM, prompt: np.ndarray, n_gen: int) -> list:
