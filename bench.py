@@ -11,7 +11,11 @@ token-evicted compressed cache of 8192 slots with degrees 1..16, draft length k 
   vc_accept         first-mismatch acceptance + bonus over [8, 33, 128256] logits
 
 Metric: attention GB/s = algorithmic bytes of the draft and verify calls per round /
-device time of the round.  Inputs are synthetic (seeded, see synth/), resident in HBM;
+device time of the round.  At N = 1 the line also carries ``workloads``: the tiny
+1024-token layer (latencies), the 128K-context int4 layer (int4 draft vs the HBM roofline,
+verify vs the tensor roofline, the oracle on a sample), the 1M-token staged verify
+(PCIe staging while three requests draft) and the tiny-decoder loop (accepted tokens/s,
+greedy tokens/s, acceptance histogram), each with its own clock record.  Inputs are synthetic (seeded, see synth/), resident in HBM;
 four copies of the layer's cache rotate across calls so no call re-reads another's
 data from the 126 MB L2, and L2 is flushed (256 MB write) between timed steps.
 
@@ -465,39 +469,224 @@ def e2e_measure(rnd, steps: int, warmup: int, device) -> dict:
             "ms_per_step": tot / steps * 1e3}
 
 
-# ------------------------------------------------------------------ 1M-token staged verify
-def run_config4(args) -> int:
+# ------------------------------------------------------------------ the other workloads
+def _events_median(fn, reps: int = 20, warm: int = 5, flush=None) -> float:
+    """Median seconds of fn() between CUDA events on the current stream, after warm-up,
+    with the L2 flushed (a 256 MB write) before each timed call when ``flush`` is given."""
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e-3)
+    return statistics.median(ts)
+
+
+def _clock_sampler(dev):
+    import torch
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    return ClockSampler(uuid)
+
+
+def _accept_case(B, n_q, V, dev, seed):
+    import torch
+    import lossless_kv_compressed_b200 as vc
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    lg = torch.randn(B, n_q, V, device=dev, generator=g)
+    dr = torch.randint(0, V, (B, max(n_q - 1, 1)), device=dev, generator=g, dtype=torch.int32)
+    i32 = dict(dtype=torch.int32, device=dev)
+    tgt, err = torch.empty(B, n_q, **i32), torch.empty(B, **i32)
+    al, cm, nc = torch.empty(B, **i32), torch.empty(B, n_q, **i32), torch.empty(B, **i32)
+    return lambda: vc.accept(lg, dr[:, :n_q - 1], target=tgt, accept_len=al, commit=cm,
+                             n_commit=nc, err_flag=err)
+
+
+def workload_tiny(dev) -> dict:
+    """The 1024-token tiny layer (batch 1, 8/2 heads of 64, 256 slots, k = 8): every call
+    is latency-bound (inputs of ~130 KB stay in L2), so the figures are microseconds."""
+    import torch
+    import lossless_kv_compressed_b200 as vc
+    from synth import gen
+    case = gen.attn_case(1)
+    cfg = case["cfg"]
+    t = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
+        torch.bfloat16).to(dev)
+    k, v = t(case["k_bits"]), t(case["v_bits"])
+    cache = vc.IndexedCache(k=k, v=v, S=cfg.S, Hq=cfg.Hq,
+                            idx=torch.from_numpy(case["idx"]).to(dev),
+                            deg=torch.from_numpy(case["deg"]).to(dev),
+                            k_tail=t(gen.bf16_block_rows(case, "k", cfg.k)),
+                            v_tail=t(gen.bf16_block_rows(case, "v", cfg.k)), n_tail=cfg.k)
+    qd, qv = t(case["q_draft_bits"]), t(case["q_verify_bits"])
+    od, ov = torch.empty_like(qd), torch.empty_like(qv)
+    wd = torch.empty(vc.draft_workspace_size(cache), dtype=torch.uint8, device=dev)
+    n_q = cfg.k + 1
+    wv = torch.empty(vc.verify_workspace_size(cfg.B, n_q, cfg.Hq, cfg.Hkv, cfg.D, 0, cfg.P + n_q),
+                     dtype=torch.uint8, device=dev)
+    lg = torch.from_numpy(case["logits"]).to(dev)
+    dr = torch.from_numpy(case["drafts"]).to(dev)
+    clocks = _clock_sampler(dev)
+    clocks.start()
+    d_us = _events_median(lambda: vc.draft_attn(qd, cache, out=od, ws=wd)) * 1e6
+    v_us = _events_median(lambda: vc.verify_attn(qv, k, v, cfg.P, out=ov, ws=wv)) * 1e6
+    a_us = _events_median(lambda: vc.accept(lg, dr)) * 1e6
+    clk = clocks.stop()
+    return {"workload": cfg.name, "bound": "latency",
+            "draft_us": d_us, "verify_us": v_us, "accept_us": a_us,
+            "accept_shape": [cfg.B, n_q, cfg.vocab],
+            "note": "calls back to back on resident inputs (L2-resident), median of 20",
+            "clocks": clk}
+
+
+def workload_int4(dev, peaks, cpu_budget_s: float = 10.0) -> dict:
+    """The 128K-context int4 layer: batch 4, 32/8 heads of 128; K and V i.i.d. N(0, 1)
+    with the workload's 1% outlier channels x10; the first 130944 tokens quantised on the
+    GPU by vc_int4_quantize (4092 blocks of 32 per pair), the last 128 of the prefix kept
+    in bf16.  Times the int4 draft (HBM roofline), the verify of k = 32 over the bf16 full
+    cache (tensor roofline) and the acceptance over [4, 33, 128256] logits; the oracle's
+    int4 draft on a bounded sample of pairs is the CPU baseline."""
+    import torch
+    import lossless_kv_compressed_b200 as vc
+    from synth import device as sd, gen
+    from synth.configs import get_config
+    cfg = get_config(3)
+    B, Hq, Hkv, D, P = cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.P
+    T_q, n_tail, n_q = P - cfg.tail_bf16, cfg.tail_bf16, cfg.k + 1
+    g = sd.generator(cfg.seed + 300, dev)
+    scale = torch.ones(Hkv, D, device=dev)
+    for f in gen.outlier_channels(cfg):
+        scale[int(f) // D, int(f) % D] = 10.0
+    K = torch.empty(B, Hkv, cfg.L_cap, D, dtype=torch.bfloat16, device=dev)
+    V = torch.empty_like(K)
+    for b in range(B):
+        K[b] = (torch.randn(Hkv, cfg.L_cap, D, generator=g, device=dev) * scale[:, None]).bfloat16()
+        V[b] = (torch.randn(Hkv, cfg.L_cap, D, generator=g, device=dev) * scale[:, None]).bfloat16()
+    cache = vc.empty_int4_cache(B, Hq, Hkv, D, T_q, device=dev)
+    vc.int4_quantize(K, V, cache, n_blocks=T_q // 32)
+    cache.S = T_q
+    cache.k_tail = K[:, :, T_q:P].contiguous()
+    cache.v_tail = V[:, :, T_q:P].contiguous()
+    cache.n_tail = n_tail
+    qd = sd.normal_bf16((B, Hq, D), g, dev)
+    qv = sd.normal_bf16((B, n_q, Hq, D), g, dev)
+    od, ov = torch.empty_like(qd), torch.empty_like(qv)
+    wd = torch.empty(vc.draft_workspace_size(cache), dtype=torch.uint8, device=dev)
+    wv = torch.empty(vc.verify_workspace_size(B, n_q, Hq, Hkv, D, 0, P + n_q), dtype=torch.uint8,
+                     device=dev)
+    acc = _accept_case(B, n_q, cfg.vocab, dev, cfg.seed + 301)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    pairs = B * Hkv
+    per_block = 32 * 4 * (D // 32) * 4 + D * 4 * 4 + 2 * D * 2 + 2 * D * 2
+    d_bytes = pairs * (T_q // 32 * per_block + n_tail * D * 4) + 2 * B * Hq * D * 2
+    v_flops = 4 * D * (Hq // Hkv) * sum(P + i + 1 for i in range(n_q)) * pairs
+    v_bytes = pairs * (P + n_q) * D * 4 + 2 * B * n_q * Hq * D * 2
+    torch.cuda.synchronize()
+    clocks = _clock_sampler(dev)
+    clocks.start()
+    d_s = _events_median(lambda: vc.draft_attn(qd, cache, out=od, ws=wd), flush=flush)
+    v_s = _events_median(lambda: vc.verify_attn(qv, K, V, P, out=ov, ws=wv), flush=flush)
+    a_s = _events_median(acc, flush=flush)
+    clk = clocks.stop()
+    d_gbs = d_bytes / d_s / 1e9
+    v_tf = v_flops / v_s / 1e12
+    attain = min(peaks["bf16_tflops"], v_flops / v_bytes * peaks["hbm_gbs"] / 1e3)
+    out = {
+        "workload": cfg.name,
+        "roofline": {"bound": "hbm", "kernel": "vc_draft_attn (int4 + bf16 tail)",
+                     "achieved": d_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": d_gbs / peaks["hbm_gbs"], "traffic": profiled_traffic("draft_int4"),
+                     "peak_source": peaks["source"] + " hbm_gbs",
+                     "algorithmic_bytes_per_launch": d_bytes, "launch_us": d_s * 1e6},
+        "draft": {"us": d_s * 1e6, "GB/s": d_gbs, "frac_hbm": d_gbs / peaks["hbm_gbs"],
+                  "queries_per_s": B / d_s, "bytes": d_bytes},
+        "verify": {"us": v_s * 1e6, "TFLOP/s": v_tf, "frac_tensor": v_tf / peaks["bf16_tflops"],
+                   "frac_attainable": v_tf / attain, "GB/s": v_bytes / v_s / 1e9,
+                   "frac_hbm": v_bytes / v_s / 1e9 / peaks["hbm_gbs"],
+                   "queries_per_s": B * n_q / v_s},
+        "accept_us": a_s * 1e6,
+        "l2": "flushed before each timed call (256 MB write)",
+        "data": "i.i.d. N(0,1) K/V with 1% outlier channels x10, drawn on the GPU "
+                "(torch generator); int4 cache quantised on the GPU",
+        "clocks": clk,
+    }
+    if cpu_budget_s > 0:
+        import oracle
+        f = oracle.bf16_to_f64
+        host = lambda x: x.cpu().numpy()
+        tot_b, tot_t, n = 0, 0.0, 0
+        for b in range(B):
+            for j in range(Hkv):
+                sl = (slice(b, b + 1), slice(j, j + 1))
+                args = [host(cache.kq[sl]).view(np.uint32), host(cache.k_scale[sl]).view(np.uint16),
+                        host(cache.k_zero[sl]).view(np.uint16), host(cache.vq[sl]).view(np.uint32),
+                        host(cache.v_scale[sl]).view(np.uint16), host(cache.v_zero[sl]).view(np.uint16)]
+                qh = f(host(qd[b:b + 1, j * cfg.g:(j + 1) * cfg.g].view(torch.int16)).view(np.uint16))
+                kt = f(host(cache.k_tail[sl].view(torch.int16)).view(np.uint16))
+                vt = f(host(cache.v_tail[sl].view(torch.int16)).view(np.uint16))
+                t0 = time.perf_counter()
+                oracle.draft_attn_int4(qh, *args, kt, vt)
+                tot_t += time.perf_counter() - t0
+                tot_b += d_bytes / pairs
+                n += 1
+                if tot_t > cpu_budget_s:
+                    break
+            if tot_t > cpu_budget_s:
+                break
+        out["cpu_baseline"] = {"value": tot_b / tot_t / 1e9, "unit": "GB/s",
+                               "cores": oracle_threads(), "kind": "oracle",
+                               "sample": f"int4 draft of {n} of {pairs} (batch, kv head) pairs "
+                                         f"(unpack, dequantise, attend), fp64 NumPy "
+                                         f"({tot_t:.1f} s)"}
+    return out
+
+
+def workload_staged(dev, peaks) -> dict:
     """Long-context staging: one request's 1M-token full cache (4 GiB, chunk-major in
     pinned host memory) streams through a 3-slot HBM ring for its k = 40 verify while
     three 256K-context requests draft over their 65536-slot compressed caches."""
     import torch
     import lossless_kv_compressed_b200 as vc
     from lossless_kv_compressed_b200.stagger import StagedVerify, run_alongside
-    from synth import gen
+    from synth import device as sd, gen
     from synth.configs import get_config
     cfg = get_config(4)
-    dev = torch.device("cuda", 0)
     chunk = cfg.chunk_tokens
     n_chunks = cfg.P // chunk
-    case = gen.staged_case(cfg)
     host = torch.empty((n_chunks, 2, cfg.Hkv, chunk, cfg.D), dtype=torch.bfloat16,
                        pin_memory=True)
-    b16 = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
-        torch.bfloat16)
-    for c, (kb, vb) in enumerate(zip(case["chunks_k"], case["chunks_v"])):
-        host[c, 0] = b16(kb)
-        host[c, 1] = b16(vb)
-    bk, bv = b16(case["block_k_bits"]).to(dev), b16(case["block_v_bits"]).to(dev)
-    q = b16(case["q_verify_bits"]).to(dev)
+    g = sd.generator(cfg.seed + 100, dev)
+    ark = sd.AR1((cfg.Hkv,), cfg.D, cfg.rho, g, dev)
+    arv = sd.AR1((cfg.Hkv,), cfg.D, cfg.rho, g, dev)
+    for c in range(n_chunks):
+        host[c, 0].copy_(ark.next(chunk).bfloat16())
+        host[c, 1].copy_(arv.next(chunk).bfloat16())
+    n_q = cfg.k + 1
+    bk = sd.normal_bf16((1, cfg.Hkv, n_q, cfg.D), g, dev)
+    bv = sd.normal_bf16((1, cfg.Hkv, n_q, cfg.D), g, dev)
+    q = sd.normal_bf16((1, n_q, cfg.Hq, cfg.D), g, dev)
     st = StagedVerify(host, cfg.P, bk, bv, n_slots=3)
     out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
     # drafting requests: 3 x 8 kv heads x 65536 compact slots, degrees 1..16
     S = cfg.S
     dc = gen.staged_draft_case(cfg)
-    kc, vcc = b16(dc["kc_bits"]).to(dev), b16(dc["vc_bits"]).to(dev)
-    deg = torch.from_numpy(dc["deg"]).to(dev)
-    dq = b16(dc["q_bits"]).to(dev)
-    dcache = vc.IndexedCache(k=kc, v=vcc, S=S, Hq=cfg.Hq, deg=deg)
+    b16 = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
+        torch.bfloat16).to(dev)
+    dcache = vc.IndexedCache(k=b16(dc["kc_bits"]), v=b16(dc["vc_bits"]), S=S, Hq=cfg.Hq,
+                             deg=torch.from_numpy(dc["deg"]).to(dev))
+    dq = b16(dc["q_bits"])
     dws = torch.empty(vc.draft_workspace_size(dcache), dtype=torch.uint8, device=dev)
     dout = torch.empty_like(dq)
     s_draft = torch.cuda.Stream(dev)
@@ -507,6 +696,9 @@ def run_config4(args) -> int:
         vc.draft_attn(dq, dcache, out=dout, ws=dws, stream=stream)
 
     full_bytes = n_chunks * st.chunk_bytes
+    torch.cuda.synchronize()
+    clocks = _clock_sampler(dev)
+    clocks.start()
     # (1) bare PCIe: the 16 chunk copies alone, back to back
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for rep in range(2):
@@ -538,39 +730,44 @@ def run_config4(args) -> int:
     n_drafts = run_alongside(st, q, out, draft_step, s_draft)
     ev1.record(s_draft)
     torch.cuda.synchronize()
+    clk = clocks.stop()
     round_ms = st.t_start.elapsed_time(st.t_done)
     staged_gbs = full_bytes / (st.t_start.elapsed_time(st.t_staged) * 1e-3) / 1e9
     draft_span_s = ev0.elapsed_time(ev1) * 1e-3
     assert vc.device_error() == 0
-    line = {
-        "metric": METRIC, "value": staged_gbs, "unit": "GB/s", "n_gpus": 1,
-        "higher_is_better": True, "dtype": "bf16", "data": "synthetic", "scaling": "weak",
-        "vs_baseline": None,
-        "config": {"workload": cfg.name, "context": cfg.P, "heads": f"{cfg.Hq}/{cfg.Hkv}",
-                   "head_dim": cfg.D, "verify_rows": cfg.k + 1, "chunk_tokens": chunk,
-                   "ring_slots": 3, "draft_requests": cfg.n_draft_requests,
-                   "draft_slots": S},
+    overlapped = n_drafts * d_bytes / draft_span_s / 1e9
+    return {
+        "workload": cfg.name,
+        "config": {"context": cfg.P, "heads": f"{cfg.Hq}/{cfg.Hkv}", "head_dim": cfg.D,
+                   "verify_rows": n_q, "chunk_tokens": chunk, "ring_slots": 3,
+                   "draft_requests": cfg.n_draft_requests, "draft_slots": S},
+        "roofline": {"bound": "pcie", "kernel": "vc_stage_full_kv (copy engines) while drafting",
+                     "achieved": staged_gbs, "peak": bare_gbs, "unit": "GB/s",
+                     "frac": staged_gbs / bare_gbs, "traffic": None,
+                     "peak_source": "bare pinned H2D of the same 16 chunks, measured here"},
         "pcie": {"bare_h2d_GBs": bare_gbs, "staged_alone_GBs": staged_alone_gbs,
                  "staged_while_drafting_GBs": staged_gbs, "frac_of_bare": staged_gbs / bare_gbs,
                  "bytes_per_round": full_bytes},
         "verify_round_ms": {"alone": verify_alone_ms, "while_drafting": round_ms},
         "draft": {"alone_us": draft_alone_s * 1e6, "alone_GBs": d_bytes / draft_alone_s / 1e9,
-                  "steps_during_round": n_drafts,
-                  "overlapped_GBs": n_drafts * d_bytes / draft_span_s / 1e9},
+                  "alone_frac_hbm": d_bytes / draft_alone_s / 1e9 / peaks["hbm_gbs"],
+                  "steps_during_round": n_drafts, "overlapped_GBs": overlapped,
+                  "overlapped_frac_hbm": overlapped / peaks["hbm_gbs"]},
         # context only: the verified request's committed tokens/s if each round accepted
         # the 25-40 tokens the VeriCache summary reports for trained models
         "modelled_accepted_tokens_per_s_at_25_40": [25 / (round_ms * 1e-3),
                                                     40 / (round_ms * 1e-3)],
+        "data": "AR(1) K/V (rho 0.9) drawn on the GPU (torch generator), staged from pinned "
+                "host memory",
+        "clocks": clk,
     }
-    print(json.dumps(line), flush=True)
-    return 0
 
 
-# ------------------------------------------------------------------ tiny-decoder loop
-def run_config5(args) -> int:
+def workload_loop(dev) -> dict:
     """The loop end to end on the tiny decoder: accepted tokens/s of the VeriCache loop
-    and of full-KV greedy decoding on the same GPU, and the acceptance-length histogram.
-    (The GPU stream against the fp64 oracle's is a GPU test, not a bench figure.)"""
+    and of full-KV greedy decoding on the same GPU, the acceptance-length histogram, and
+    the acceptance call over [1, 33, 8192] logits.  (The GPU stream against the fp64
+    oracle's is a GPU test, not a bench figure.)"""
     import torch
     from lossless_kv_compressed_b200.loop import GpuTinyLM, greedy_loop, vericache_loop
     from synth import gen
@@ -579,7 +776,8 @@ def run_config5(args) -> int:
     w = gen.tinylm_weights(cfg)
     prompt = gen.tinylm_prompt(cfg)
     max_len = cfg.prompt_len + cfg.gen_tokens + cfg.k + 2
-    mk = lambda: GpuTinyLM(w, cfg, max_len, cfg.k, cfg.budget + cfg.gen_tokens + cfg.k + 2)
+    mk = lambda: GpuTinyLM(w, cfg, max_len, cfg.k, cfg.budget + cfg.gen_tokens + cfg.k + 2,
+                           device=dev)
 
     def timed(fn):
         torch.cuda.synchronize()
@@ -590,26 +788,53 @@ def run_config5(args) -> int:
 
     greedy_loop(mk(), prompt, 8)                   # warm-up (module load, allocator)
     g_model, v_model = mk(), mk()
+    clocks = _clock_sampler(dev)
+    clocks.start()
     greedy, tg = timed(lambda: greedy_loop(g_model, prompt, cfg.gen_tokens))
     (toks, alens), tv = timed(lambda: vericache_loop(v_model, prompt, cfg.gen_tokens, cfg.k,
                                                      cfg.budget, cfg.n_sinks, cfg.n_recent,
                                                      cfg.score_window))
+    a_us = _events_median(_accept_case(1, cfg.k + 1, cfg.vocab, dev, cfg.seed + 1)) * 1e6
+    clk = clocks.stop()
     hist = np.bincount(np.asarray(alens), minlength=cfg.k + 1).tolist()
-    line = {
-        "metric": METRIC, "value": cfg.gen_tokens / tv, "unit": "accepted tokens/s",
-        "n_gpus": 1, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
-        "scaling": "weak", "vs_baseline": None,
-        "config": {"workload": cfg.name, "layers": cfg.n_layers, "d_model": cfg.d_model,
-                   "heads": f"{cfg.Hq}/{cfg.Hkv}", "head_dim": cfg.D, "ffn": cfg.ffn,
-                   "vocab": cfg.vocab, "prompt": cfg.prompt_len, "generated": cfg.gen_tokens,
-                   "draft_len": cfg.k, "budget": cfg.budget,
-                   "timing": "wall clock incl. prefill, host-driven launches"},
-        "commits_equal_greedy": toks == greedy,
+    return {
+        "workload": cfg.name, "unit": "accepted tokens/s",
+        "accepted_tokens_per_s": cfg.gen_tokens / tv,
         "greedy_tokens_per_s": cfg.gen_tokens / tg,
+        "commits_equal_greedy": toks == greedy,
         "rounds": len(alens), "mean_accept_len": float(np.mean(alens)),
         "accept_len_histogram": hist,
-        "oracle_fp64": "tests/test_gpu_loop.py::test_tinylm_loop_greedy_follows_oracle_to_a_near_tie",
+        "accept_us": a_us,
+        "config": {"layers": cfg.n_layers, "d_model": cfg.d_model,
+                   "heads": f"{cfg.Hq}/{cfg.Hkv}", "head_dim": cfg.D, "ffn": cfg.ffn,
+                   "vocab": cfg.vocab, "prompt": cfg.prompt_len, "generated": cfg.gen_tokens,
+                   "draft_len": cfg.k, "budget": cfg.budget},
+        "timing": "wall clock incl. prefill and eviction, host-driven launches",
+        "clocks": clk,
     }
+
+
+def run_config4(args) -> int:
+    import torch
+    dev = torch.device("cuda", 0)
+    r = workload_staged(dev, measured_peaks())
+    line = {"metric": METRIC, "value": r["pcie"]["staged_while_drafting_GBs"], "unit": "GB/s",
+            "n_gpus": 1, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None}
+    line.update(r)
+    line["config"] = dict(r["config"], workload=r["workload"])
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_config5(args) -> int:
+    import torch
+    r = workload_loop(torch.device("cuda", 0))
+    line = {"metric": METRIC, "value": r["accepted_tokens_per_s"], "unit": "accepted tokens/s",
+            "n_gpus": 1, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None}
+    line.update(r)
+    line["config"] = dict(r["config"], workload=r["workload"])
     print(json.dumps(line), flush=True)
     return 0
 
@@ -785,12 +1010,49 @@ def run_table(args) -> int:
     return 0
 
 
+def _profile_int4(kind: str) -> int:
+    """Five calls of the 128K-context int4 layer's draft (``int4``) or verify (``verify3``)
+    for an ncu capture: about 3 GB on the device (bf16 full cache + the int4 cache)."""
+    import torch
+    import lossless_kv_compressed_b200 as vc
+    from synth import device as sd
+    from synth.configs import get_config
+    cfg = get_config(3)
+    dev = torch.device("cuda", 0)
+    g = sd.generator(cfg.seed + 300, dev)
+    B, Hq, Hkv, D, P = cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.P
+    T_q, n_q = P - cfg.tail_bf16, cfg.k + 1
+    K = sd.normal_bf16((B, Hkv, cfg.L_cap, D), g, dev)
+    V = sd.normal_bf16((B, Hkv, cfg.L_cap, D), g, dev)
+    if kind == "int4":
+        cache = vc.empty_int4_cache(B, Hq, Hkv, D, T_q, device=dev)
+        vc.int4_quantize(K, V, cache, n_blocks=T_q // 32)
+        cache.S, cache.n_tail = T_q, cfg.tail_bf16
+        cache.k_tail = K[:, :, T_q:P].contiguous()
+        cache.v_tail = V[:, :, T_q:P].contiguous()
+        del K, V
+        q = sd.normal_bf16((B, Hq, D), g, dev)
+        ws = torch.empty(vc.draft_workspace_size(cache), dtype=torch.uint8, device=dev)
+        for _ in range(5):
+            vc.draft_attn(q, cache, ws=ws)
+    else:
+        q = sd.normal_bf16((B, n_q, Hq, D), g, dev)
+        for _ in range(5):
+            vc.verify_attn(q, K, V, P)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": kind, "workload": cfg.name, "ok": True}), flush=True)
+    return 0
+
+
 def run_profile_case(kind: str) -> int:
     """A short run of one call of the 32K-context round for an ncu capture: one copy of
-    the inputs (about 1.2 GB on the device), five calls of the chosen entry point."""
+    the inputs (about 1.2 GB on the device), five calls of the chosen entry point
+    (``int4`` and ``verify3``: the 128K-context int4 layer's draft and verify)."""
     import torch
     import lossless_kv_compressed_b200 as vc
     from synth import gen
+    if kind in ("int4", "verify3"):
+        return _profile_int4(kind)
     case = gen.attn_case(2)
     cfg = case["cfg"]
     dev = torch.device("cuda", 0)
@@ -832,9 +1094,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--table", action="store_true",
                     help="per-kernel rates at every workload's shapes, one JSON line per row")
-    ap.add_argument("--profile-case", choices=["draft", "verify", "accept"], default=None,
+    ap.add_argument("--profile-case", choices=["draft", "verify", "accept", "int4", "verify3"],
+                    default=None,
                     help="run five calls of one entry point on the 32K-context inputs (one "
                          "copy) for an ncu capture, and print no bench line")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the tiny, int4, staged and loop workloads after the timed "
+                         "round (they run by default at N = 1)")
     ap.add_argument("--config", type=int, default=2, choices=[2, 4, 5],
                     help="2: the round of the 32K-context layer (default line); "
                          "4: long-context staging while drafting; 5: the loop end to end")
@@ -923,6 +1189,22 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(case)
+    # The other workloads' figures, measured after the timed steps on the same GPU (one
+    # GPU only: at N > 1 every rank runs the same replica round and nothing else).
+    workloads = None
+    if world == 1 and not args.no_workloads:
+        workloads = {}
+        for name, fn in (("1", lambda: workload_tiny(device)),
+                         ("3", lambda: workload_int4(device, peaks,
+                                                     0.0 if args.no_cpu_baseline else 10.0)),
+                         ("4", lambda: workload_staged(device, peaks)),
+                         ("5", lambda: workload_loop(device))):
+            try:
+                workloads[name] = fn()
+            except Exception as e:          # reported in the line, never hidden
+                workloads[name] = {"error": f"{type(e).__name__}: {e}"}
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
 
     if rank == 0:
         line = {
@@ -958,6 +1240,8 @@ def main():
             "round_bytes": rb,
             "rounds_per_s": world * args.steps / t_max,
         }
+        if workloads is not None:
+            line["workloads"] = workloads
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

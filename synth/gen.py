@@ -116,6 +116,15 @@ def agreeing_logits(rng: Generator, B: int, nq: int, V: int, drafts: np.ndarray,
 
 
 # ---------------------------------------------------------------- workloads
+def outlier_channels(cfg: AttnConfig, rng: Generator | None = None) -> np.ndarray:
+    """The (kv head, channel) pairs scaled x10 in the int4 workload, as flat indices
+    kvh * D + d (unsorted draw order): round(outlier_frac * Hkv * D) distinct pairs."""
+    if rng is None:
+        rng = children(cfg.seed, 12)[2]
+    n_out = int(round(cfg.outlier_frac * cfg.Hkv * cfg.D))
+    return rng.choice(cfg.Hkv * cfg.D, size=n_out, replace=False)
+
+
 def attn_case(cfg: AttnConfig | int, **override) -> dict:
     """Seeded inputs for one attention-layer workload (optionally resized).
 
@@ -135,8 +144,7 @@ def attn_case(cfg: AttnConfig | int, **override) -> dict:
     Kf = ar1(r[0], (B, Hkv), cfg.L_cap, D, cfg.rho)
     Vf = ar1(r[1], (B, Hkv), cfg.L_cap, D, cfg.rho)
     if cfg.outlier_frac > 0.0:
-        n_out = int(round(cfg.outlier_frac * Hkv * D))
-        flat = r[2].choice(Hkv * D, size=n_out, replace=False)
+        flat = outlier_channels(cfg, r[2])
         for f in flat:
             Kf[:, f // D, :, f % D] *= 10.0
             Vf[:, f // D, :, f % D] *= 10.0
