@@ -234,3 +234,97 @@ def vericache_loop(model, prompt, n_gen, k, budget, n_sinks, n_recent, score_win
                 slots[l][j] = np.concatenate([slots[l][j], np.arange(P, P + a + 1)])
         P += a + 1
     return out[:n_gen], accept_lens
+
+
+def vericache_loop_csm(model, prompt, n_gen, k, budget, n_sinks, n_recent, chunk, r_init,
+                       delta_r, r_floor, recluster_every):
+    """Draft-then-verify decoding whose compressed cache is built by CentroidKV's Chunked
+    Soft Matching ("Riassunto Tecnico: CentroidKV", section "Metodologia": item 2, the
+    inference pipeline -- a clustering round after prefill when the cache exceeds the
+    budget, re-clustering every g decoding steps, sinks and recent tokens preserved;
+    item 3, the progressive schedule r_j = r_init - j * delta_r; item 4, drafting over
+    degree-weighted centroids with ln n_t in the softmax).  Returns (generated tokens,
+    accept lengths, cache sizes after each clustering round).
+
+    Readings: after prefill, rounds run until the cache is within the budget (each round
+    can at most halve a chunk, so one may not suffice); r_j never drops below r_floor;
+    the accepted tokens' verify-pass K/V join the compressed cache with degree 1 (the
+    draft tail is dropped, as in ``vericache_loop``); after every ``recluster_every``
+    committed tokens one more round runs if the cache is over the budget."""
+    from . import csm
+    c = model.cfg
+    n = len(prompt)
+    L_cap = n + n_gen + k + 2
+    logits, Ks, Vs, _ = model.prefill(prompt, L_cap)
+    comp = [[[Ks[l][j, :n].copy(), Vs[l][j, :n].copy(), np.ones(n, np.int64)]
+             for j in range(c.Hkv)] for l in range(c.n_layers)]
+    state = {"j": 0}
+    sizes = []
+
+    def cluster_round():
+        r = max(r_floor, r_init - state["j"] * delta_r)
+        for l in range(c.n_layers):
+            for j in range(c.Hkv):
+                Kc, Vc, nc = comp[l][j]
+                Ko, Vo, no, _ = csm.compress(Kc, Vc, nc, n_sinks, n_recent, chunk, r)
+                comp[l][j] = [Ko, Vo, no]
+        state["j"] += 1
+        sizes.append(len(comp[0][0][2]))
+
+    while len(comp[0][0][2]) > budget:
+        before = len(comp[0][0][2])
+        cluster_round()
+        if len(comp[0][0][2]) == before:       # nothing left to merge
+            break
+    out = [int(accept(logits[None, None])["target"][0, 0])]
+    P = n
+    accept_lens = []
+    since = 0
+    while len(out) < n_gen:
+        pending = out[-1]
+        tails_k = [np.zeros((c.Hkv, 0, c.D)) for _ in range(c.n_layers)]
+        tails_v = [np.zeros((c.Hkv, 0, c.D)) for _ in range(c.n_layers)]
+        drafts = []
+        x_tok = pending
+        for jd in range(k):
+            x = model.w["embed"][[x_tok]]
+            for l in range(c.n_layers):
+                q, kk, vv = model.qkv(l, x, [P + jd])
+                tails_k[l] = np.concatenate([tails_k[l], kk.transpose(1, 0, 2)], axis=1)
+                tails_v[l] = np.concatenate([tails_v[l], vv.transpose(1, 0, 2)], axis=1)
+                Kc = np.stack([comp[l][j][0] for j in range(c.Hkv)])[None]
+                Vc = np.stack([comp[l][j][1] for j in range(c.Hkv)])[None]
+                deg = np.stack([comp[l][j][2] for j in range(c.Hkv)])[None]
+                o, _ = draft_attn(q, Kc, Vc, Kc.shape[2], None, deg, tails_k[l][None],
+                                  tails_v[l][None])
+                x = model.finish_layer(l, x, o)
+            d = int(accept(model.logits(x)[None])["target"][0, 0])
+            drafts.append(d)
+            x_tok = d
+        toks = [pending] + drafts
+        pos = np.arange(P, P + k + 1)
+        x = model.w["embed"][toks]
+        for l in range(c.n_layers):
+            q, kk, vv = model.qkv(l, x, pos)
+            Ks[l][:, P:P + k + 1] = kk.transpose(1, 0, 2)
+            Vs[l][:, P:P + k + 1] = vv.transpose(1, 0, 2)
+            o = verify_attn(q[None], Ks[l][None, :, :P + k + 1], Vs[l][None, :, :P + k + 1], P)
+            x = model.finish_layer(l, x, o[0])
+        r = accept(model.logits(x)[None], np.array([drafts]))
+        a = int(r["accept_len"][0])
+        accept_lens.append(a)
+        out.extend(int(t) for t in r["commit"][0, :a + 1])
+        for l in range(c.n_layers):
+            Ks[l][:, P + a + 1:P + k + 1] = 0.0
+            Vs[l][:, P + a + 1:P + k + 1] = 0.0
+            for j in range(c.Hkv):
+                comp[l][j][0] = np.concatenate([comp[l][j][0], Ks[l][j, P:P + a + 1]])
+                comp[l][j][1] = np.concatenate([comp[l][j][1], Vs[l][j, P:P + a + 1]])
+                comp[l][j][2] = np.concatenate([comp[l][j][2], np.ones(a + 1, np.int64)])
+        P += a + 1
+        since += a + 1
+        if since >= recluster_every:
+            since = 0
+            if len(comp[0][0][2]) > budget:
+                cluster_round()
+    return out[:n_gen], accept_lens, sizes

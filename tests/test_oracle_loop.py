@@ -147,3 +147,40 @@ def test_no_compression_accepts_every_draft_plus_bonus():
     full_rounds = (cfg.gen_tokens - 1) // (cfg.k + 1)
     assert alens[:full_rounds] == [cfg.k] * full_rounds
     assert vc == tinylm.greedy_loop(model, prompt, cfg.gen_tokens)
+
+
+def _csm_loop(cfg, **kw):
+    model, _ = _model(cfg)
+    prompt = gen.tinylm_prompt(cfg)
+    args = dict(budget=20, n_sinks=2, n_recent=4, chunk=8, r_init=1.0, delta_r=0.25,
+                r_floor=0.25, recluster_every=6)
+    args.update(kw)
+    return model, prompt, tinylm.vericache_loop_csm(model, prompt, cfg.gen_tokens, cfg.k,
+                                                    **args)
+
+
+def test_csm_loop_commits_equal_greedy_and_reclusters():
+    """CentroidKV's pipeline inside the loop: clustering after prefill until within the
+    budget, re-clustering as the cache grows, drafting over centroids with ln n; the
+    committed stream is still full-KV greedy decoding (VeriCache summary, "Risultati
+    Sperimentali")."""
+    cfg = SMALL
+    model, prompt, (toks, alens, sizes) = _csm_loop(cfg)
+    assert toks == tinylm.greedy_loop(model, prompt, cfg.gen_tokens)
+    assert len(sizes) >= 3                      # prefill rounds plus at least one re-cluster
+    assert sizes[0] < cfg.prompt_len
+    # the schedule's first rounds halve every full chunk of the middle
+    from oracle import csm
+    assert sizes[0] == csm.out_len(cfg.prompt_len, 2, 4, 8, 1.0)
+
+
+def test_csm_loop_without_merging_accepts_every_draft():
+    """r = 0 merges nothing and a budget above the prompt never clusters: the drafter
+    sees the whole context, so every round accepts all k drafts plus the bonus."""
+    cfg = dataclasses.replace(SMALL, gen_tokens=19)
+    model, prompt, (toks, alens, sizes) = _csm_loop(cfg, budget=1000, r_init=0.0, delta_r=0.0,
+                                                    r_floor=0.0)
+    assert sizes == []
+    full = (cfg.gen_tokens - 1) // (cfg.k + 1)
+    assert alens[:full] == [cfg.k] * full
+    assert toks == tinylm.greedy_loop(model, prompt, cfg.gen_tokens)
