@@ -769,7 +769,8 @@ def workload_loop(dev) -> dict:
     the acceptance call over [1, 33, 8192] logits.  (The GPU stream against the fp64
     oracle's is a GPU test, not a bench figure.)"""
     import torch
-    from lossless_kv_compressed_b200.loop import GpuTinyLM, greedy_loop, vericache_loop
+    from lossless_kv_compressed_b200.loop import (GpuTinyLM, greedy_loop, vericache_loop,
+                                                  vericache_loop_csm)
     from synth import gen
     from synth.configs import get_config
     cfg = get_config(5)
@@ -794,6 +795,13 @@ def workload_loop(dev) -> dict:
     (toks, alens), tv = timed(lambda: vericache_loop(v_model, prompt, cfg.gen_tokens, cfg.k,
                                                      cfg.budget, cfg.n_sinks, cfg.n_recent,
                                                      cfg.score_window))
+    # the same loop over a Chunked Soft Matching cache (CentroidKV) instead of eviction
+    cap = cfg.prompt_len + cfg.gen_tokens + cfg.k + 2
+    c_model = GpuTinyLM(w, cfg, max_len, cfg.k, cap, device=dev)
+    (ctoks, calens, csizes), tc = timed(lambda: vericache_loop_csm(
+        c_model, prompt, cfg.gen_tokens, cfg.k, cfg.budget, cfg.n_sinks, cfg.n_recent,
+        chunk=cfg.csm_chunk, r_init=cfg.csm_r_init, delta_r=cfg.csm_delta_r,
+        r_floor=cfg.csm_r_floor, recluster_every=cfg.csm_recluster_every))
     a_us = _events_median(_accept_case(1, cfg.k + 1, cfg.vocab, dev, cfg.seed + 1)) * 1e6
     clk = clocks.stop()
     hist = np.bincount(np.asarray(alens), minlength=cfg.k + 1).tolist()
@@ -805,6 +813,15 @@ def workload_loop(dev) -> dict:
         "rounds": len(alens), "mean_accept_len": float(np.mean(alens)),
         "accept_len_histogram": hist,
         "accept_us": a_us,
+        "csm": {"accepted_tokens_per_s": cfg.gen_tokens / tc,
+                "commits_equal_greedy": ctoks == greedy, "rounds": len(calens),
+                "mean_accept_len": float(np.mean(calens)),
+                "accept_len_histogram": np.bincount(np.asarray(calens),
+                                                    minlength=cfg.k + 1).tolist(),
+                "cache_rows_after_each_clustering": csizes,
+                "schedule": {"chunk": cfg.csm_chunk, "r_init": cfg.csm_r_init,
+                             "delta_r": cfg.csm_delta_r, "r_floor": cfg.csm_r_floor,
+                             "recluster_every": cfg.csm_recluster_every}},
         "config": {"layers": cfg.n_layers, "d_model": cfg.d_model,
                    "heads": f"{cfg.Hq}/{cfg.Hkv}", "head_dim": cfg.D, "ffn": cfg.ffn,
                    "vocab": cfg.vocab, "prompt": cfg.prompt_len, "generated": cfg.gen_tokens,

@@ -61,6 +61,73 @@ vc_status vc_glue_swiglu(const float* gu, int n, int F, void* out, cudaStream_t 
 vc_status vc_glue_append_slots(int32_t* idx, int32_t* deg, int Hkv, int S_cap, int S,
                                int start, int count, cudaStream_t stream);
 
+/* ----------------------------------------------------------------------------------
+ * Host-side drivers of the loop: one call enqueues every kernel of k draft steps, of a
+ * verify (or prefill) pass, or of n greedy steps, so a round costs a handful of calls
+ * from the host instead of one per kernel.  They run the same kernels as the calls above
+ * and the attention / acceptance calls of vericache.h, in the same order.
+ *
+ * vc_tinylm describes the model and its buffers (batch 1).  Per-layer arrays are HOST
+ * arrays of n_layers device pointers.  Weights bf16, matrices [in, out]:
+ *   wqkv [d, (Hq + 2 Hkv) D] (q | k | v), wo [Hq D, d], wgu [d, 2 ffn] (gate | up),
+ *   wdown [ffn, d], embed [vocab, d], lm_head [d, vocab].
+ * Caches: k_full / v_full bf16 [Hkv, cap, D] (position p in row p); k_tail / v_tail bf16
+ * [Hkv, tail_cap, D] (draft step j stores its K/V in row j).  positions: device int32
+ * [>= cap] with positions[i] = i.  Work buffers for rows_cap rows: x fp32 [rows, d], h
+ * bf16 [rows, d], qkv fp32 [rows, (Hq + 2 Hkv) D], q, att bf16 [rows, Hq, D], gu fp32
+ * [rows, 2 ffn], act bf16 [rows, ffn], logits fp32 [rows, vocab].  ws: device workspace
+ * for the attention calls of one pass (large enough for vc_draft_workspace_size of every
+ * draft cache and vc_verify_workspace_size(1, min(rows_cap, 1024 / g), Hq, Hkv, D, 0,
+ * cap)).
+ * -------------------------------------------------------------------------------- */
+typedef struct vc_tinylm {
+  int32_t n_layers, d_model, Hq, Hkv, D, ffn, vocab;
+  float rms_eps, rope_theta;
+  const void* embed;
+  const void* lm_head;
+  const void* const* wqkv;
+  const void* const* wo;
+  const void* const* wgu;
+  const void* const* wdown;
+  void* const* k_full;
+  void* const* v_full;
+  int32_t cap;
+  void* const* k_tail;
+  void* const* v_tail;
+  int32_t tail_cap;
+  const int32_t* positions;
+  float* x;
+  void* h;
+  float* qkv;
+  void* q;
+  void* att;
+  float* gu;
+  void* act;
+  float* logits;
+  int32_t rows_cap;
+  void* ws;
+  size_t ws_bytes;
+} vc_tinylm;
+
+/* Tokens ids[0 .. n-1] (device int32) at positions pos0 .. pos0+n-1 through the whole
+ * model over the full cache (their K/V stored at their positions, rows attending
+ * causally): logits fp32 [n, vocab] in m->logits.  n <= rows_cap, pos0 + n <= cap. */
+vc_status vc_glue_forward_full(const vc_tinylm* m, const int32_t* ids, int n, int pos0,
+                               cudaStream_t stream);
+
+/* k draft steps ([VC] "Algoritmo Principale", step 1): step j feeds ids[j] at position
+ * P + j through the model, attending layer l's compressed cache caches[l] (a host array
+ * of n_layers descriptors; their tail fields are replaced by the model's draft tail with
+ * j + 1 rows) and writes the argmax of its logits to ids[j + 1].  ids device int32
+ * [k + 1]; k + 1 <= tail_cap; P + k <= cap. */
+vc_status vc_glue_draft_steps(const vc_tinylm* m, const vc_comp_cache* caches, int32_t* ids,
+                              int k, int P, cudaStream_t stream);
+
+/* n greedy steps over the full cache: step t feeds ids[t] at position pos0 + t and writes
+ * the argmax of its logits to ids[t + 1].  ids device int32 [n + 1]. */
+vc_status vc_glue_greedy_steps(const vc_tinylm* m, int32_t* ids, int n, int pos0,
+                               cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -28,7 +28,8 @@ EXPORTS = (
 # Model glue of the end-to-end loop (include/vericache_glue.h).
 GLUE_EXPORTS = (
     "vc_glue_embed", "vc_glue_rmsnorm", "vc_glue_gemm", "vc_glue_rope_store",
-    "vc_glue_swiglu", "vc_glue_append_slots",
+    "vc_glue_swiglu", "vc_glue_append_slots", "vc_glue_forward_full", "vc_glue_draft_steps",
+    "vc_glue_greedy_steps",
 )
 
 _p = ctypes.c_void_p
@@ -48,6 +49,22 @@ class CompCache(ctypes.Structure):
         ("vq", _p), ("v_scale", _p), ("v_zero", _p),
         ("k_tail", _p), ("v_tail", _p), ("R_cap", _i32), ("n_tail", _i32),
         ("err_flag", _p),
+    ]
+
+
+class TinyLM(ctypes.Structure):
+    """Mirror of ``vc_tinylm`` (vericache_glue.h)."""
+
+    _fields_ = [
+        ("n_layers", _i32), ("d_model", _i32), ("Hq", _i32), ("Hkv", _i32), ("D", _i32),
+        ("ffn", _i32), ("vocab", _i32), ("rms_eps", ctypes.c_float),
+        ("rope_theta", ctypes.c_float), ("embed", _p), ("lm_head", _p),
+        ("wqkv", ctypes.POINTER(_p)), ("wo", ctypes.POINTER(_p)), ("wgu", ctypes.POINTER(_p)),
+        ("wdown", ctypes.POINTER(_p)), ("k_full", ctypes.POINTER(_p)),
+        ("v_full", ctypes.POINTER(_p)), ("cap", _i32), ("k_tail", ctypes.POINTER(_p)),
+        ("v_tail", ctypes.POINTER(_p)), ("tail_cap", _i32), ("positions", _p),
+        ("x", _p), ("h", _p), ("qkv", _p), ("q", _p), ("att", _p), ("gu", _p), ("act", _p),
+        ("logits", _p), ("rows_cap", _i32), ("ws", _p), ("ws_bytes", _sz),
     ]
 
 
@@ -126,6 +143,12 @@ def lib() -> ctypes.CDLL:
                                                                              ctypes.c_int, _p]
         L.vc_glue_swiglu.argtypes = [_p, ctypes.c_int, ctypes.c_int, _p, _p]
         L.vc_glue_append_slots.argtypes = [_p, _p] + [ctypes.c_int] * 5 + [_p]
+        L.vc_glue_forward_full.argtypes = [ctypes.POINTER(TinyLM), _p, ctypes.c_int,
+                                           ctypes.c_int, _p]
+        L.vc_glue_draft_steps.argtypes = [ctypes.POINTER(TinyLM), ctypes.POINTER(CompCache), _p,
+                                          ctypes.c_int, ctypes.c_int, _p]
+        L.vc_glue_greedy_steps.argtypes = [ctypes.POINTER(TinyLM), _p, ctypes.c_int,
+                                           ctypes.c_int, _p]
         _lib = L
     return _lib
 

@@ -13,7 +13,8 @@
 //
 // Design: one CTA per (chunk, pair) -- a chunk is <= 256 rows, so everything after the
 // loads stays in shared memory.  The chunk's key rows land once in a swizzled tile
-// (cp.async); the |A| x |B| dot products run on mma.sync (bf16 in, fp32 accumulate,
+// (cp.async), its value rows in a second tile whose copies complete while the matching
+// runs (the centroids read both from shared memory); the |A| x |B| dot products run on mma.sync (bf16 in, fp32 accumulate,
 // each warp one 16-row A tile against all B rows) and every A row keeps its best
 // dot / |b| with a quad reduction; the top-m selection is a rank count over the
 // chunk's <= 128 candidates; the centroids sum in a fixed order (the B row, then its
@@ -49,7 +50,8 @@ template <int D>
 struct CsmSmem {
   static constexpr int kRowB = D * 2;
   static constexpr int kK = 0;                                     // [256][D] bf16
-  static constexpr int kInvN = kK + kCsmMaxChunk * kRowB;          // float [256]
+  static constexpr int kV = kK + kCsmMaxChunk * kRowB;             // [256][D] bf16
+  static constexpr int kInvN = kV + kCsmMaxChunk * kRowB;          // float [256]
   static constexpr int kBestB = kInvN + kCsmMaxChunk * 4;          // int [128]
   static constexpr int kBestS = kBestB + 128 * 4;                  // float [128]
   static constexpr int kMerged = kBestS + 128 * 4;                 // int [128]
@@ -113,7 +115,9 @@ __global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
   int* merged = reinterpret_cast<int*>(smem + SM::kMerged);
   int* scan = reinterpret_cast<int*>(smem + SM::kScan);
 
-  // ---- key rows of the chunk -> shared memory (rows past the chunk zeroed)
+  // ---- key rows of the chunk -> shared memory (rows past the chunk zeroed), then the
+  //      value rows in a second group that lands while the matching runs
+  const uint32_t vs = smem_u32(smem + SM::kV);
   for (int e = tid; e < kCsmMaxChunk * CH; e += kCsmThreads) {
     const int r = e / CH, c = e - r * CH;
     const bool ok = r < len;
@@ -121,7 +125,12 @@ __global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
                ok ? 16u : 0u);
   }
   cp_async_commit();
-  cp_async_wait<0>();
+  for (int e = tid; e < len * CH; e += kCsmThreads) {
+    const int r = e / CH, c = e - r * CH;
+    cp_async16(csm_row_addr<D>(vs, r, c), vin + (int64_t)(r0 + r) * D + c * 8, 16u);
+  }
+  cp_async_commit();
+  cp_async_wait<1>();
   __syncthreads();
 
   // ---- 1 / |k| of every row (0 for an all-zero row: its cosines are 0)
@@ -233,6 +242,8 @@ __global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
   }
 
   // ---- write the kept rows: unmerged A rows as they are, B rows as centroids
+  cp_async_wait<0>();                             // the value rows
+  __syncthreads();
   constexpr int DPL = D / 32;                     // channels per lane
   for (int t = warp; t < len; t += kCsmThreads / 32) {
     if ((t & 1) == 0 && merged[t >> 1]) continue;  // warp-uniform
@@ -241,9 +252,9 @@ __global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
     float ak[DPL], av[DPL];
     int ntot = deg_of(row);
     const float nb = (float)ntot;
-    auto load_k = [&](int r, float (&x)[DPL]) {     // channels lane*DPL .. from shared
+    auto load_row = [&](int tile, int r, float (&x)[DPL]) {   // channels lane*DPL ..
       const int d0 = lane * DPL;
-      const uint8_t* src = smem + SM::kK + r * SM::kRowB + (((d0 >> 3) ^ (r & 7)) << 4) +
+      const uint8_t* src = smem + tile + r * SM::kRowB + (((d0 >> 3) ^ (r & 7)) << 4) +
                            (d0 & 7) * 2;
       if constexpr (DPL == 4) {
         const uint2 w = *reinterpret_cast<const uint2*>(src);
@@ -253,16 +264,8 @@ __global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
         x[0] = bf16_lo(w); x[1] = bf16_hi(w);
       }
     };
-    auto load_v = [&](int r, float (&x)[DPL]) {     // from global
-      const __nv_bfloat16* src = vin + (int64_t)(r0 + r) * D + lane * DPL;
-      if constexpr (DPL == 4) {
-        const uint2 w = *reinterpret_cast<const uint2*>(src);
-        x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
-      } else {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(src);
-        x[0] = bf16_lo(w); x[1] = bf16_hi(w);
-      }
-    };
+    auto load_k = [&](int r, float (&x)[DPL]) { load_row(SM::kK, r, x); };
+    auto load_v = [&](int r, float (&x)[DPL]) { load_row(SM::kV, r, x); };
     load_k(t, ak);
     load_v(t, av);
     if (t & 1) {

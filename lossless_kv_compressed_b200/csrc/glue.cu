@@ -224,4 +224,125 @@ vc_status vc_glue_append_slots(int32_t* idx, int32_t* deg, int Hkv, int S_cap, i
   return VC_OK;
 }
 
+// ------------------------------------------------------------------ loop drivers
+namespace {
+
+vc_status check_model(const vc_tinylm* m) {
+  if (!m || m->n_layers <= 0 || !m->wqkv || !m->wo || !m->wgu || !m->wdown || !m->k_full ||
+      !m->v_full || !m->positions || !m->x || !m->h || !m->qkv || !m->q || !m->att ||
+      !m->gu || !m->act || !m->logits || !m->ws || !m->embed || !m->lm_head)
+    return fail(VC_ERR_INVALID, "tinylm: NULL field");
+  if (m->Hq % m->Hkv || m->d_model % 256 || (m->D != 64 && m->D != 128))
+    return fail(VC_ERR_UNSUPPORTED, "tinylm: shape");
+  return VC_OK;
+}
+
+// One layer's work after the attention output is in m->att: output projection with the
+// residual, the MLP with its residual.
+vc_status layer_tail(const vc_tinylm* m, int l, int n, cudaStream_t s) {
+  vc_status st;
+  if ((st = vc_glue_gemm(m->att, m->wo[l], n, m->Hq * m->D, m->d_model, m->x, 1, s))) return st;
+  if ((st = vc_glue_rmsnorm(m->x, n, m->d_model, m->rms_eps, m->h, s))) return st;
+  if ((st = vc_glue_gemm(m->h, m->wgu[l], n, m->d_model, 2 * m->ffn, m->gu, 0, s))) return st;
+  if ((st = vc_glue_swiglu(m->gu, n, m->ffn, m->act, s))) return st;
+  return vc_glue_gemm(m->act, m->wdown[l], n, m->ffn, m->d_model, m->x, 1, s);
+}
+
+vc_status layer_head(const vc_tinylm* m, int l, int n, const int32_t* pos, const int32_t* dst,
+                     void* kc, void* vcache, int cap, cudaStream_t s) {
+  vc_status st;
+  const int nqkv = (m->Hq + 2 * m->Hkv) * m->D;
+  if ((st = vc_glue_rmsnorm(m->x, n, m->d_model, m->rms_eps, m->h, s))) return st;
+  if ((st = vc_glue_gemm(m->h, m->wqkv[l], n, m->d_model, nqkv, m->qkv, 0, s))) return st;
+  return vc_glue_rope_store(m->qkv, pos, dst, n, m->Hq, m->Hkv, m->D, m->rope_theta, m->q, kc,
+                            vcache, cap, s);
+}
+
+vc_status logits_of(const vc_tinylm* m, int n, cudaStream_t s) {
+  vc_status st;
+  if ((st = vc_glue_rmsnorm(m->x, n, m->d_model, m->rms_eps, m->h, s))) return st;
+  return vc_glue_gemm(m->h, m->lm_head, n, m->d_model, m->vocab, m->logits, 0, s);
+}
+
+vc_status forward_full(const vc_tinylm* m, const int32_t* ids, int n, int pos0, cudaStream_t s) {
+  vc_status st;
+  if ((st = vc_glue_embed(m->embed, ids, n, m->d_model, m->x, s))) return st;
+  const int g = m->Hq / m->Hkv;
+  const int chunk = 1024 / g;
+  const size_t qrow = (size_t)m->Hq * m->D * 2;          // bytes of one row of q / att
+  for (int l = 0; l < m->n_layers; ++l) {
+    const int32_t* pos = m->positions + pos0;
+    if ((st = layer_head(m, l, n, pos, pos, m->k_full[l], m->v_full[l], m->cap, s))) return st;
+    for (int r0 = 0; r0 < n; r0 += chunk) {
+      const int r1 = n < r0 + chunk ? n : r0 + chunk;
+      const int nq = r1 - r0;
+      const int64_t P = pos0 + r0;
+      st = vc_verify_attn(static_cast<const char*>(m->q) + r0 * qrow, 1, nq, m->Hq, m->Hkv,
+                          m->D, m->k_full[l], m->v_full[l], m->cap, 0, P + nq, P, nullptr,
+                          nullptr, nullptr, 0, 0.f, static_cast<char*>(m->att) + r0 * qrow,
+                          m->ws, m->ws_bytes, s);
+      if (st) return st;
+    }
+    if ((st = layer_tail(m, l, n, s))) return st;
+  }
+  return logits_of(m, n, s);
+}
+
+}  // namespace
+
+vc_status vc_glue_forward_full(const vc_tinylm* m, const int32_t* ids, int n, int pos0,
+                               cudaStream_t stream) {
+  vc_status st = check_model(m);
+  if (st) return st;
+  if (!ids || n <= 0 || n > m->rows_cap || pos0 < 0 || pos0 + n > m->cap)
+    return fail(VC_ERR_INVALID, "forward_full: rows or positions");
+  return forward_full(m, ids, n, pos0, stream);
+}
+
+vc_status vc_glue_draft_steps(const vc_tinylm* m, const vc_comp_cache* caches, int32_t* ids,
+                              int k, int P, cudaStream_t stream) {
+  vc_status st = check_model(m);
+  if (st) return st;
+  if (!caches || !ids || k < 0 || k + 1 > m->tail_cap || P < 0 || P + k > m->cap ||
+      !m->k_tail || !m->v_tail)
+    return fail(VC_ERR_INVALID, "draft_steps: arguments");
+  for (int j = 0; j < k; ++j) {
+    if ((st = vc_glue_embed(m->embed, ids + j, 1, m->d_model, m->x, stream))) return st;
+    for (int l = 0; l < m->n_layers; ++l) {
+      // this step's K/V go to row j of the draft tail
+      if ((st = layer_head(m, l, 1, m->positions + P + j, m->positions + j, m->k_tail[l],
+                           m->v_tail[l], m->tail_cap, stream)))
+        return st;
+      vc_comp_cache c = caches[l];
+      c.k_tail = m->k_tail[l];
+      c.v_tail = m->v_tail[l];
+      c.R_cap = m->tail_cap;
+      c.n_tail = j + 1;
+      if ((st = vc_draft_attn(m->q, &c, 0.f, 0, m->att, nullptr, m->ws, m->ws_bytes, stream)))
+        return st;
+      if ((st = layer_tail(m, l, 1, stream))) return st;
+    }
+    if ((st = logits_of(m, 1, stream))) return st;
+    if ((st = vc_accept(m->logits, nullptr, 1, 1, m->vocab, ids + j + 1, nullptr, nullptr,
+                        nullptr, nullptr, stream)))
+      return st;
+  }
+  return VC_OK;
+}
+
+vc_status vc_glue_greedy_steps(const vc_tinylm* m, int32_t* ids, int n, int pos0,
+                               cudaStream_t stream) {
+  vc_status st = check_model(m);
+  if (st) return st;
+  if (!ids || n < 0 || pos0 < 0 || pos0 + n > m->cap)
+    return fail(VC_ERR_INVALID, "greedy_steps: arguments");
+  for (int t = 0; t < n; ++t) {
+    if ((st = forward_full(m, ids + t, 1, pos0 + t, stream))) return st;
+    if ((st = vc_accept(m->logits, nullptr, 1, 1, m->vocab, ids + t + 1, nullptr, nullptr,
+                        nullptr, nullptr, stream)))
+      return st;
+  }
+  return VC_OK;
+}
+
 }  // extern "C"

@@ -48,18 +48,30 @@ __device__ __forceinline__ uint64_t globaltimer() {
 
 // Bounded wait: returns false after ~limit_ns of wall time or once *abort is set
 // by another role of the CTA (so one stuck role cannot hang the others).  abort may be
-// null (teardown waits that must not be cut short by the flag).  Each test suspends the
-// thread for at most min(limit_ns, 1 ms), so the limit and the flag are checked at least
-// that often whatever the hardware's own suspend time.
+// null (teardown waits that must not be cut short by the flag).  Ordinary limits use the
+// plain test (the thread wakes as soon as the phase completes) and look at the clock and
+// the flag every 64 tests; a limit under 1 ms (a test of the error path) bounds each
+// test's suspend time by the limit itself, so the wait really gives up that early.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns = 2000000000ull) {
-  const uint32_t hint = limit_ns < 1000000ull ? (uint32_t)limit_ns : 1000000u;
-  if (mbar_try_for(bar, parity, hint)) return true;
-  const uint64_t t0 = globaltimer();
-  for (;;) {
+  if (limit_ns < 1000000ull) {
+    const uint32_t hint = (uint32_t)limit_ns;
     if (mbar_try_for(bar, parity, hint)) return true;
-    if (abort != nullptr && *abort) return false;
-    if (globaltimer() - t0 > limit_ns) return false;
+    const uint64_t t0 = globaltimer();
+    for (;;) {
+      if (mbar_try_for(bar, parity, hint)) return true;
+      if (abort != nullptr && *abort) return false;
+      if (globaltimer() - t0 > limit_ns) return false;
+    }
+  }
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (abort != nullptr && *abort) return false;
+      if (globaltimer() - t0 > limit_ns) return false;
+    }
   }
 }
 
@@ -132,6 +144,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+// 32 lanes x 16 consecutive 32-bit columns, all set to zero.
+__device__ __forceinline__ void tmem_st16_zero(uint32_t taddr) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
+      "%1,%1};"
+      :: "r"(taddr), "r"(0u) : "memory");
+}
+
 // ---------------------------------------------------------------- UMMA
 // Shared-memory matrix descriptor, 128-byte swizzle (tiles 1024-byte aligned):
 // start address >> 4 in bits 0-13, leading byte offset >> 4 in 16-29, stride byte
@@ -147,11 +167,14 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
 }
 
 // Instruction descriptor of kind::f16 with bf16 A and B and an fp32 accumulator.
-// b_mn_major: B stored with N contiguous (e.g. V rows [keys][dims] as the B of P.V).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+// a_mn_major / b_mn_major: the operand is stored with its M (N) index contiguous instead
+// of K (e.g. V rows [keys][dims] read as V^T, the A of V^T P^T).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
+                                                      bool b_mn_major) {
   return (1u << 4)                       // accumulator fp32
          | (1u << 7)                     // A bf16
          | (1u << 10)                    // B bf16
+         | ((a_mn_major ? 1u : 0u) << 15)
          | ((b_mn_major ? 1u : 0u) << 16)
          | ((uint32_t)(N >> 3) << 17)
          | ((uint32_t)(M >> 4) << 24);

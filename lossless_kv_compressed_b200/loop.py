@@ -10,11 +10,12 @@ section "Problematica").
 
 Everything per token runs in libvericache.so: glue kernels (vericache_glue.h) for
 embedding, RMSNorm, fused QKV / O / gate-up / down / LM-head GEMMs, RoPE with the cache
-store and SwiGLU; vc_draft_attn / vc_verify_attn / vc_accept for the method.  Token ids
-stay on the device between draft steps (each argmax is written straight into the next
-step's input); the host reads back only the accepted length and the commits, once per
-round.  Eviction after the prefill (attention-mass scores of the last prompt queries and
-the top-budget selection) runs in the library too.
+store and SwiGLU; vc_draft_attn / vc_verify_attn / vc_accept for the method.  A round is
+three library calls from the host -- vc_glue_draft_steps (the k draft steps, each argmax
+written straight into the next step's input on the device), vc_glue_forward_full (the
+verify pass) and vc_accept -- and the host reads back only the accepted length and the
+commits.  Eviction after the prefill (attention-mass scores of the last prompt queries
+and the top-budget selection) and CentroidKV's clustering run in the library too.
 
 Readings (same as the fp64 oracle in oracle/tinylm.py): k+1 verify rows (pending token +
 k drafts); on a disagreement the full-KV prediction is committed as the correction; the
@@ -29,8 +30,8 @@ import numpy as np
 import torch
 
 from . import _lib
-from .api import (IndexedCache, accept, draft_attn, draft_workspace_size, evict_scores,
-                  evict_select, verify_attn)
+from .api import (IndexedCache, accept, csm_compress, draft_attn, draft_workspace_size,
+                  evict_scores, evict_select, verify_attn, verify_workspace_size)
 from ._lib import check, lib
 
 
@@ -69,6 +70,9 @@ class GpuTinyLM:
         self.VT = [z(1, Hkv, k + 1, D) for _ in range(L)]
         self.idx = [z(1, Hkv, s_cap, dt=i32) for _ in range(L)]  # compressed slots
         self.S = 0
+        # Chunked Soft Matching caches (compact rows + degrees), two buffers per layer:
+        # a clustering round reads one and writes the other (allocated on first use)
+        self.csm = None
         self.arange = torch.arange(max_len + k + 2, dtype=i32, device=self.dev)
         rows = max(self.PREFILL_ROWS, k + 1)
         self._alloc(rows)
@@ -129,10 +133,15 @@ class GpuTinyLM:
                   "vc_glue_rope_store")
             if keep_last:
                 self.qlast.append(self.q[n - keep_last:n].clone())
-            if mode == "draft":
+            if mode == "draft" and self.csm is not None:
+                kc, vcc, dc = self.csm["cur"][l]
+                cache = IndexedCache(k=kc, v=vcc, S=self.S, Hq=c.Hq, deg=dc,
+                                     k_tail=self.KT[l], v_tail=self.VT[l], n_tail=n_tail)
+            elif mode == "draft":
                 cache = IndexedCache(k=self.K[l], v=self.V[l], S=self.S, Hq=c.Hq,
                                      idx=self.idx[l], k_tail=self.KT[l], v_tail=self.VT[l],
                                      n_tail=n_tail)
+            if mode == "draft":
                 draft_attn(self.q[:1].view(1, c.Hq, c.D), cache,
                            out=self.att[:1].view(1, c.Hq, c.D))
             else:
@@ -174,17 +183,127 @@ class GpuTinyLM:
         self.S = min(budget, n)
 
 
+    # ---------------------------------------------------------------- C-side drivers
+    def _native(self):
+        """The model descriptor of the C drivers (vericache_glue.h), rebuilt when the work
+        buffers change; its workspace covers every attention call of the loop."""
+        key = (self.x.data_ptr(), self.rows)
+        if getattr(self, "_nat_key", None) == key:
+            return self._nat
+        c = self.cfg
+        P = ctypes.c_void_p
+        arr = lambda ts: (P * len(ts))(*[t.data_ptr() for t in ts])
+        g = c.Hq // c.Hkv
+        need = verify_workspace_size(1, min(self.rows, 1024 // g), c.Hq, c.Hkv, c.D, 0,
+                                     self.max_len)
+        probe = IndexedCache(k=self.K[0], v=self.V[0], S=self.s_cap, Hq=c.Hq,
+                             idx=self.idx[0], k_tail=self.KT[0], v_tail=self.VT[0],
+                             n_tail=self.k + 1)
+        need = max(need, draft_workspace_size(probe))
+        self._nat_ws = torch.empty(need, dtype=torch.uint8, device=self.dev)
+        self._nat_arrays = [arr(self.wqkv), arr(self.wo), arr(self.wgu), arr(self.wdown),
+                            arr(self.K), arr(self.V), arr(self.KT), arr(self.VT)]
+        a = self._nat_arrays
+        m = _lib.TinyLM()
+        m.n_layers, m.d_model, m.Hq, m.Hkv, m.D = c.n_layers, c.d_model, c.Hq, c.Hkv, c.D
+        m.ffn, m.vocab, m.rms_eps, m.rope_theta = c.ffn, c.vocab, c.rms_eps, c.rope_theta
+        m.embed, m.lm_head = self.embed.data_ptr(), self.lm_head.data_ptr()
+        m.wqkv, m.wo, m.wgu, m.wdown = a[0], a[1], a[2], a[3]
+        m.k_full, m.v_full, m.cap = a[4], a[5], self.max_len
+        m.k_tail, m.v_tail, m.tail_cap = a[6], a[7], self.k + 1
+        m.positions = self.arange.data_ptr()
+        m.x, m.h, m.qkv, m.q = (self.x.data_ptr(), self.h.data_ptr(), self.qkv.data_ptr(),
+                                self.q.data_ptr())
+        m.att, m.gu, m.act, m.logits = (self.att.data_ptr(), self.gu.data_ptr(),
+                                        self.act.data_ptr(), self.logits.data_ptr())
+        m.rows_cap = self.rows
+        m.ws, m.ws_bytes = self._nat_ws.data_ptr(), self._nat_ws.numel()
+        self._nat, self._nat_key = m, key
+        return m
+
+    def _draft_caches(self):
+        c = self.cfg
+        out = []
+        for l in range(c.n_layers):
+            if self.csm is not None:
+                kc, vcc, dc = self.csm["cur"][l]
+                out.append(IndexedCache(k=kc, v=vcc, S=self.S, Hq=c.Hq, deg=dc).struct())
+            else:
+                out.append(IndexedCache(k=self.K[l], v=self.V[l], S=self.S, Hq=c.Hq,
+                                        idx=self.idx[l]).struct())
+        return (_lib.CompCache * len(out))(*out)
+
+    def draft_steps(self, ids: torch.Tensor, k: int, P: int) -> None:
+        """k draft steps in one library call: ids[j] at position P + j -> ids[j + 1]."""
+        check(lib().vc_glue_draft_steps(ctypes.byref(self._native()), self._draft_caches(),
+                                        ids.data_ptr(), k, P, self._s()), "vc_glue_draft_steps")
+
+    def forward_full(self, ids: torch.Tensor, n: int, pos0: int) -> torch.Tensor:
+        """n tokens over the full cache in one library call; logits fp32 [n, V]."""
+        check(lib().vc_glue_forward_full(ctypes.byref(self._native()), ids.data_ptr(), n, pos0,
+                                         self._s()), "vc_glue_forward_full")
+        return self.logits[:n]
+
+    def greedy_steps(self, ids: torch.Tensor, n: int, pos0: int) -> None:
+        """n greedy steps in one library call: ids[t] at position pos0 + t -> ids[t + 1]."""
+        check(lib().vc_glue_greedy_steps(ctypes.byref(self._native()), ids.data_ptr(), n, pos0,
+                                         self._s()), "vc_glue_greedy_steps")
+
+    # ---------------------------------------------------------------- CentroidKV
+    def csm_init(self, n: int):
+        """The compressed cache starts as the prompt's own rows, degree 1."""
+        c = self.cfg
+        cap = self.s_cap
+        if n > cap:
+            raise ValueError(f"compressed-cache capacity {cap} < prompt length {n}")
+        bf, i32 = torch.bfloat16, torch.int32
+        mk = lambda: [(torch.empty((1, c.Hkv, cap, c.D), dtype=bf, device=self.dev),
+                       torch.empty((1, c.Hkv, cap, c.D), dtype=bf, device=self.dev),
+                       torch.empty((1, c.Hkv, cap), dtype=i32, device=self.dev))
+                      for _ in range(c.n_layers)]
+        self.csm = {"cur": mk(), "alt": mk(), "round": 0}
+        for l in range(c.n_layers):
+            kc, vcc, dc = self.csm["cur"][l]
+            kc[:, :, :n].copy_(self.K[l][:, :, :n])
+            vcc[:, :, :n].copy_(self.V[l][:, :, :n])
+            dc[:, :, :n].fill_(1)
+        self.S = n
+
+    def csm_round(self, n_sinks: int, n_recent: int, chunk: int, r: float) -> int:
+        """One Chunked Soft Matching round (vc_csm_compress) over every layer's compressed
+        cache; returns the new size."""
+        n_out = 0
+        for l in range(self.cfg.n_layers):
+            kc, vcc, dc = self.csm["cur"][l]
+            ko, vo, do = self.csm["alt"][l]
+            _, _, _, n_out = csm_compress(kc, vcc, n_sinks, n_recent, chunk, r, deg=dc,
+                                          T=self.S, k_out=ko, v_out=vo, deg_out=do)
+        self.csm["cur"], self.csm["alt"] = self.csm["alt"], self.csm["cur"]
+        self.csm["round"] += 1
+        self.S = n_out
+        return n_out
+
+    def csm_append(self, P: int, n: int):
+        """The accepted tokens' verify-pass K/V (rows P .. P+n-1 of the full cache) join
+        the compressed cache with degree 1."""
+        if self.S + n > self.s_cap:
+            raise ValueError("compressed cache full")
+        for l in range(self.cfg.n_layers):
+            kc, vcc, dc = self.csm["cur"][l]
+            kc[:, :, self.S:self.S + n].copy_(self.K[l][:, :, P:P + n])
+            vcc[:, :, self.S:self.S + n].copy_(self.V[l][:, :, P:P + n])
+            dc[:, :, self.S:self.S + n].fill_(1)
+        self.S += n
+
+
 def greedy_loop(model: GpuTinyLM, prompt: np.ndarray, n_gen: int) -> list:
     """Full-KV greedy decoding on the GPU: one token per step through the verify
-    attention (n_q = 1), argmax on the device, one read-back at the end."""
+    attention (n_q = 1), argmax on the device, one read-back at the end; the steps after
+    the prefill are enqueued by one library call."""
     logits = model.prefill(prompt)
     out = torch.empty(n_gen, dtype=torch.int32, device=model.dev)
     accept(logits.view(1, 1, -1), target=out[0:1].view(1, 1))
-    p = len(prompt)
-    for t in range(1, n_gen):
-        lg = model.forward(out[t - 1:t], 1, p, "full")
-        accept(lg.view(1, 1, -1), target=out[t:t + 1].view(1, 1))
-        p += 1
+    model.greedy_steps(out, n_gen - 1, len(prompt))
     return out.cpu().tolist()
 
 
@@ -204,10 +323,8 @@ def vericache_loop(model: GpuTinyLM, prompt: np.ndarray, n_gen: int, k: int, bud
     alens = []
     while len(out) < n_gen:
         vids[0] = out[-1]
-        for j in range(k):
-            lg = model.forward(vids[j:j + 1], 1, P + j, "draft", n_tail=j + 1)
-            accept(lg.view(1, 1, -1), target=vids[j + 1:j + 2].view(1, 1))
-        lg = model.forward(vids, k + 1, P, "full")
+        model.draft_steps(vids, k, P)
+        lg = model.forward_full(vids, k + 1, P)
         drafts = vids[1:].view(1, k)
         r = accept(lg.view(1, k + 1, -1), drafts)
         a = int(r["accept_len"].item())
@@ -224,3 +341,59 @@ def vericache_loop(model: GpuTinyLM, prompt: np.ndarray, n_gen: int, k: int, bud
         model.S += a + 1
         P += a + 1
     return out[:n_gen], alens
+
+
+def vericache_loop_csm(model: GpuTinyLM, prompt: np.ndarray, n_gen: int, k: int, budget: int,
+                       n_sinks: int, n_recent: int, chunk: int, r_init: float, delta_r: float,
+                       r_floor: float, recluster_every: int, record=None):
+    """Draft-then-verify decoding over a Chunked Soft Matching cache (CentroidKV summary,
+    "Riassunto Tecnico: CentroidKV", section "Metodologia", items 2-4): after prefill the
+    prompt's cache is clustered by vc_csm_compress until it fits the budget, with
+    r_j = max(r_floor, r_init - j * delta_r) for round j; the drafts attend the centroids
+    with their ln n_t bias; the accepted tokens join the cache with degree 1, and after
+    every ``recluster_every`` committed tokens one more round runs if the cache is over
+    the budget.  The same readings as the fp64 oracle's ``vericache_loop_csm``.
+    Returns (tokens, accept lengths, cache sizes after each clustering round)."""
+    n = len(prompt)
+    logits = model.prefill(prompt)
+    model.csm_init(n)
+    sizes = []
+
+    def cluster():
+        r = max(r_floor, r_init - model.csm["round"] * delta_r)
+        sizes.append(model.csm_round(n_sinks, n_recent, chunk, r))
+
+    while model.S > budget:
+        before = model.S
+        cluster()
+        if model.S == before:
+            break
+    dev = model.dev
+    first = torch.empty((1, 1), dtype=torch.int32, device=dev)
+    accept(logits.view(1, 1, -1), target=first)
+    out = [int(first.item())]
+    P = n
+    vids = torch.empty(k + 1, dtype=torch.int32, device=dev)
+    alens = []
+    since = 0
+    while len(out) < n_gen:
+        vids[0] = out[-1]
+        model.draft_steps(vids, k, P)
+        lg = model.forward_full(vids, k + 1, P)
+        drafts = vids[1:].view(1, k)
+        r = accept(lg.view(1, k + 1, -1), drafts)
+        a = int(r["accept_len"].item())
+        commit = r["commit"][0, :a + 1].cpu().tolist()
+        if record is not None:
+            record.append((lg.detach().cpu().numpy().copy(), drafts.cpu().numpy().copy(),
+                           {key: v.cpu().numpy().copy() for key, v in r.items() if v is not None}))
+        alens.append(a)
+        out.extend(commit)
+        model.csm_append(P, a + 1)
+        P += a + 1
+        since += a + 1
+        if since >= recluster_every:
+            since = 0
+            if model.S > budget:
+                cluster()
+    return out[:n_gen], alens, sizes

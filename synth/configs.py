@@ -74,6 +74,13 @@ class LoopConfig:
     rope_theta: float = 10000.0
     rms_eps: float = 1e-5
     init_std: float = 0.02
+    # Chunked Soft Matching variant of the compressed cache (CentroidKV): chunk size,
+    # ratio schedule r_j = max(r_floor, r_init - j * delta_r), re-clustering interval
+    csm_chunk: int = 256
+    csm_r_init: float = 1.0
+    csm_delta_r: float = 0.1
+    csm_r_floor: float = 0.1
+    csm_recluster_every: int = 128
     extra: dict = field(default_factory=dict)
 
     @property

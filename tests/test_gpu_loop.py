@@ -18,7 +18,8 @@ import torch
 import lossless_kv_compressed_b200 as vc
 import oracle
 from lossless_kv_compressed_b200._lib import check, lib
-from lossless_kv_compressed_b200.loop import GpuTinyLM, greedy_loop, vericache_loop
+from lossless_kv_compressed_b200.loop import (GpuTinyLM, greedy_loop, vericache_loop,
+                                              vericache_loop_csm)
 from oracle import tinylm
 from synth import gen
 from synth.configs import LoopConfig, get_config
@@ -174,3 +175,57 @@ def test_tinylm_loop_greedy_follows_oracle_to_a_near_tie():
         g = m.forward(ids, 1, p, "full").double().cpu().numpy()[0]
         o = tinylm._decode_full(om, tg, p, Ks, Vs)
         p += 1
+
+
+CSM_ARGS = dict(chunk=32, r_init=1.0, delta_r=0.2, r_floor=0.2, recluster_every=16)
+
+
+def test_csm_loop_commits_equal_greedy_and_accept_is_exact():
+    """CentroidKV's pipeline in the loop on the GPU: vc_csm_compress clusters the prompt's
+    cache until it fits the budget (r_j = r_init - j delta_r), the drafts attend the
+    centroids with ln n_t, accepted tokens join with degree 1 and the cache is
+    re-clustered as it grows; the committed stream still equals full-KV greedy decoding
+    and every round's acceptance is exact against the oracle."""
+    from oracle import csm
+    cfg = SMALL
+    w = gen.tinylm_weights(cfg)
+    prompt = gen.tinylm_prompt(cfg)
+    greedy = greedy_loop(_model(cfg, w), prompt, cfg.gen_tokens)
+    cap = cfg.prompt_len + cfg.gen_tokens + cfg.k + 2
+    m = GpuTinyLM(w, cfg, cap, cfg.k, cap)
+    rec = []
+    toks, alens, sizes = vericache_loop_csm(m, prompt, cfg.gen_tokens, cfg.k, cfg.budget,
+                                            cfg.n_sinks, cfg.n_recent, record=rec, **CSM_ARGS)
+    assert toks == greedy
+    # clustering after prefill: the sizes follow the schedule exactly (they depend on the
+    # row counts only), down to the budget; then at least one re-clustering
+    T, j, want = cfg.prompt_len, 0, []
+    while T > cfg.budget:
+        r = max(CSM_ARGS["r_floor"], CSM_ARGS["r_init"] - j * CSM_ARGS["delta_r"])
+        T = csm.out_len(T, cfg.n_sinks, cfg.n_recent, CSM_ARGS["chunk"], r)
+        want.append(T)
+        j += 1
+    assert sizes[:len(want)] == want
+    assert len(sizes) > len(want)
+    for logits, drafts, got in rec:
+        ref = oracle.accept(logits[None], drafts)
+        for key in ("target", "accept_len", "commit", "n_commit", "err"):
+            assert np.array_equal(got[key], ref[key]), key
+    assert vc.device_error() == 0
+
+
+def test_csm_loop_full_size():
+    """The tiny-decoder loop at full size with the Chunked Soft Matching cache: 8192-token
+    prompt clustered to the 2048-slot budget (chunk 256), 512 tokens, k = 32."""
+    cfg = get_config(5)
+    w = gen.tinylm_weights(cfg)
+    prompt = gen.tinylm_prompt(cfg)
+    greedy = greedy_loop(_model(cfg, w), prompt, cfg.gen_tokens)
+    cap = cfg.prompt_len + cfg.gen_tokens + cfg.k + 2
+    m = GpuTinyLM(w, cfg, cap, cfg.k, cap)
+    toks, alens, sizes = vericache_loop_csm(
+        m, prompt, cfg.gen_tokens, cfg.k, cfg.budget, cfg.n_sinks, cfg.n_recent,
+        chunk=cfg.csm_chunk, r_init=cfg.csm_r_init, delta_r=cfg.csm_delta_r,
+        r_floor=cfg.csm_r_floor, recluster_every=cfg.csm_recluster_every)
+    assert toks == greedy
+    assert sizes and sizes[0] < cfg.prompt_len
