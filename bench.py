@@ -1070,6 +1070,26 @@ def run_profile_case(kind: str) -> int:
     from synth import gen
     if kind in ("int4", "verify3"):
         return _profile_int4(kind)
+    if kind == "csm":
+        # one Chunked Soft Matching round over the 32K-context caches (chunk 256, r 0.5),
+        # five times: about 2 GB on the device
+        from synth import device as sd
+        from synth.configs import get_config
+        c = get_config(2)
+        dev = torch.device("cuda", 0)
+        g = sd.generator(c.seed + 400, dev)
+        kc = sd.normal_bf16((c.B, c.Hkv, c.P, c.D), g, dev)
+        vcc = sd.normal_bf16((c.B, c.Hkv, c.P, c.D), g, dev)
+        deg = torch.randint(1, 17, (c.B, c.Hkv, c.P), device=dev, generator=g, dtype=torch.int32)
+        n_out = vc.csm_out_len(c.P, 4, 512, 256, 0.5)
+        ko = torch.empty(c.B, c.Hkv, n_out, c.D, dtype=torch.bfloat16, device=dev)
+        vo = torch.empty_like(ko)
+        do = torch.empty(c.B, c.Hkv, n_out, dtype=torch.int32, device=dev)
+        for _ in range(5):
+            vc.csm_compress(kc, vcc, 4, 512, 256, 0.5, deg=deg, k_out=ko, v_out=vo, deg_out=do)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_case": kind, "workload": c.name, "ok": True}), flush=True)
+        return 0
     case = gen.attn_case(2)
     cfg = case["cfg"]
     dev = torch.device("cuda", 0)
@@ -1111,7 +1131,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--table", action="store_true",
                     help="per-kernel rates at every workload's shapes, one JSON line per row")
-    ap.add_argument("--profile-case", choices=["draft", "verify", "accept", "int4", "verify3"],
+    ap.add_argument("--profile-case",
+                    choices=["draft", "verify", "accept", "int4", "verify3", "csm"],
                     default=None,
                     help="run five calls of one entry point on the 32K-context inputs (one "
                          "copy) for an ncu capture, and print no bench line")

@@ -363,20 +363,21 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
 
 // ------------------------------------------------------------------ int4 cache
 // Draft attention over the 4-bit cache (layout in vericache.h): the same persistent
-// per-warp ranges, over (pair, 32-token block) units.  A block's packed K and V words and
-// its fp16 scales / zeros are five contiguous runs (5 KB at D = 128) copied into a
+// per-warp ranges, over (pair, 32-token block) units.  A block's packed K and V words
+// and its fp16 scales / zeros are five contiguous runs (5 KB at D = 128) copied into a
 // per-warp cp.async ring.  The word layout matches the mma.sync fragments, so a thread
 // reads exactly its own nibbles: one 16-byte load per token for K, one word per channel
-// for V.  Each nibble pair becomes an fp16 pair x_hat = n s + z in four instructions (the
-// nibbles ORed into the mantissa of fp16 1024, 1024 subtracted exactly, one fused
-// multiply-add with the group's scale and zero, a single rounding to fp16), and the
-// dequantised K and V are the B operands of f16 mma.sync:
-//   S = (q_hi + q_lo) . K_hat^T     (q split into fp16 high and low parts once per pair,
-//                                    placed in A rows 0-7 and 8-15: ~22-bit q)
-//   O += (p_hi + p_lo) . V_hat       (p split once per block the same way)
-// The accumulator rows of the two halves add up to the result.  The only rounding beyond
-// fp32 accumulation is that of x_hat to fp16 (relative 2^-11, below the bf16 rounding of
-// the full cache the draft approximates); scale and zero enter exactly.
+// for V.  The nibbles stay exact (ORed into the mantissa of fp16 1024, then 1024
+// subtracted) and the scales move to the other operand, so nothing proportional to a
+// dequantised value is ever rounded to fp16:
+//   q . k_hat = sum_d (q_d s_d) n_d + sum_d q_d z_d              (K: per channel)
+//   sum_t p_t v_hat_t = sum_t (p_t s_t / 2)(2 n_t - 15) + sum_t p_t (z_t + 7.5 s_t)
+//                                                                 (V: per token, group;
+//   centred so that neither sum is much larger than the result)
+// q_d s_d and p_t s_t are split into fp16 high and low parts placed in A rows 0-7 and
+// 8-15 (rows 8-15 are padding: g <= 8), so one f16 mma.sync carries both and the two
+// accumulator halves add up to ~22 mantissa bits.  The zero-point sum over tokens is
+// one more mma per 16 tokens; sum_d q_d z_d is an fp32 dot product.
 struct DraftInt4Params {
   const __nv_bfloat16* q;
   const uint32_t* kq;            // [pairs, nblk_cap, 32, 4, D/32]
@@ -403,14 +404,22 @@ struct Int4Smem {
   static constexpr int kStageB = kKW + kVW + 4 * kSZ;
 };
 
-// Nibble pair j of word w (nibbles j and j + 4) dequantised: (n0 s0 + z0, n1 s1 + z1) as
-// fp16x2, with s2 = (s0, s1), z2 = (z0, z1).
-__device__ __forceinline__ uint32_t deq_pair(uint32_t w, int j, uint32_t s2, uint32_t z2) {
-  const uint32_t x = ((w >> (4 * j)) & 0x000F000Fu) | 0x64006400u;   // 1024 + n, exact
-  uint32_t n, r;
+// Nibble pair j of word w as exact fp16x2 integers (n0, n1).
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int j) {
+  const uint32_t x = ((w >> (4 * j)) & 0x000F000Fu) | 0x64006400u;   // 1024 + n
+  uint32_t n;
   asm("sub.f16x2 %0, %1, %2;" : "=r"(n) : "r"(x), "r"(0x64006400u));
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(n), "r"(s2), "r"(z2));
-  return r;
+  return n;
+}
+// Same, centred on the middle of the 4-bit range and doubled: (2 n0 - 15, 2 n1 - 15),
+// exact.  2n + 1 goes into the mantissa of fp16 1024 (the nibble shifted up one bit,
+// the low bit set) and 1040 is subtracted, so one subtraction does both steps.
+__device__ __forceinline__ uint32_t nib_pair_c2(uint32_t w, int j) {
+  const uint32_t sh = j == 0 ? (w << 1) : (w >> (4 * j - 1));
+  const uint32_t x = (sh & 0x001E001Eu) | 0x64016401u;     // 1024 + 2n + 1
+  uint32_t c;
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(c) : "r"(x), "r"(0x64106410u));   // - 1040
+  return c;
 }
 __device__ __forceinline__ float2 h2f(uint32_t h) {
   return __half22float2(*reinterpret_cast<const __half2*>(&h));
@@ -469,36 +478,45 @@ __global__ void __launch_bounds__(128, 3) draft_int4_kernel(const DraftInt4Param
     for (int i = 0; i < (4 * SZC) / 32; ++i) cp_async16(zd + i * 16, zb + i * 16, 16u);
   };
 
-  // q of the pair's heads as fp16 high / low A fragments (rows 0-7 / 8-15)
   const int qr = lane >> 2, qc = lane & 3;
-  uint32_t qh[D / 16][2], ql[D / 16][2];
-  auto load_q = [&](int64_t pair) {
+  uint32_t qa[D / 16][2], qn[D / 16][2];
+  auto load_q = [&](int64_t pair, uint32_t (&dst)[D / 16][2]) {
     const int64_t b = pair / p.Hkv, j = pair - b * p.Hkv;
     const bool ok = qr < p.g;
     const uint32_t* qp =
         reinterpret_cast<const uint32_t*>(p.q + (b * p.Hq + j * p.g + (ok ? qr : 0)) * D);
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t w = ok ? __ldg(qp + (16 * ks + 8 * h + 2 * qc) / 2) : 0u;
-        split_f16(bf16_lo(w), bf16_hi(w), qh[ks][h], ql[ks][h]);
-      }
+    for (int ks = 0; ks < D / 16; ++ks) {       // raw bf16 pairs, widened when used
+      dst[ks][0] = ok ? __ldg(qp + (16 * ks + 2 * qc) / 2) : 0u;
+      dst[ks][1] = ok ? __ldg(qp + (16 * ks + 8 + 2 * qc) / 2) : 0u;
+    }
   };
   const int64_t pair_last = (x0 + n - 1) / nblk;
-  load_q(pair_first);
+  load_q(pair_first, qa);
+  if (pair_last > pair_first) load_q(pair_first + 1, qn);
 
   float o[NT][4];
+  float zacc[4];
   float m_run, l_run;
   auto reset = [&]() {
 #pragma unroll
     for (int nn = 0; nn < NT; ++nn) o[nn][0] = o[nn][1] = o[nn][2] = o[nn][3] = 0.f;
+    zacc[0] = zacc[1] = zacc[2] = zacc[3] = 0.f;
     m_run = -INFINITY;
     l_run = 0.f;
   };
   auto flush = [&](int64_t pair) {
     float l = l_run + __shfl_xor_sync(0xffffffffu, l_run, 1);
     l += __shfl_xor_sync(0xffffffffu, l, 2);
+    // zero-point term of group G for row qr: columns G of the zacc tile (lane qr*4 + G/2)
+    const float zc0 = zacc[0] + zacc[2], zc1 = zacc[1] + zacc[3];
+    float zt[NW];
+#pragma unroll
+    for (int G = 0; G < NW; ++G) {
+      const float a = __shfl_sync(0xffffffffu, zc0, qr * 4 + G / 2);
+      const float b = __shfl_sync(0xffffffffu, zc1, qr * 4 + G / 2);
+      zt[G] = (G & 1) ? b : a;
+    }
     const int64_t seg = gw - warp_of_tile(pair * p.nblk, p.T, p.W);
     const int64_t part = (pair * p.maxseg + seg) * p.g;
     if (qr < p.g) {
@@ -506,7 +524,7 @@ __global__ void __launch_bounds__(128, 3) draft_int4_kernel(const DraftInt4Param
 #pragma unroll
       for (int nn = 0; nn < NT; ++nn)
         *reinterpret_cast<float2*>(dst + nn * 8 + 2 * qc) =
-            make_float2(o[nn][0] + o[nn][2], o[nn][1] + o[nn][3]);
+            make_float2(o[nn][0] + o[nn][2] + zt[nn / 4], o[nn][1] + o[nn][3] + zt[nn / 4]);
       if (qc == 0) *reinterpret_cast<float2*>(p.ws_ml + (part + qr) * 2) = make_float2(m_run, l);
     }
   };
@@ -529,7 +547,9 @@ __global__ void __launch_bounds__(128, 3) draft_int4_kernel(const DraftInt4Param
       flush(cur);
       reset();
       ++cur;
-      load_q(cur);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) { qa[ks][0] = qn[ks][0]; qa[ks][1] = qn[ks][1]; }
+      if (cur < pair_last) load_q(cur + 1, qn);
     }
     ++c_rem;
     const uint8_t* sbase = wbuf + (it % NST) * SM::kStageB;
@@ -540,40 +560,52 @@ __global__ void __launch_bounds__(128, 3) draft_int4_kernel(const DraftInt4Param
     const uint32_t* vsc = kzr + SM::kSZ / 4;
     const uint32_t* vzr = vsc + SM::kSZ / 4;
 
-    // ---- S = Q K_hat^T over 4 n-tiles of 8 tokens: this thread's key words of tokens
-    //      8 nt + qr (word (t, qc, w) holds channels 16 (2w + hk) + 2qc (+8) as pairs)
-    uint32_t w[4][NW];
+    // ---- q'_d = q_d * s_d (per channel of this block) as hi/lo A fragments, and the
+    //      zero-point term c = sum_d q_d z_d of this thread's head (fp32)
+    uint32_t ah[D / 16][2], al[D / 16][2];
+    float cz = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      const uint32_t* src = kw + ((nt * 8 + qr) * 4 + qc) * NW;
-      if constexpr (NW == 4) {
-        const uint4 v4 = *reinterpret_cast<const uint4*>(src);
-        w[nt][0] = v4.x; w[nt][1] = v4.y; w[nt][2] = v4.z; w[nt][3] = v4.w;
-      } else {
-        const uint2 v2 = *reinterpret_cast<const uint2*>(src);
-        w[nt][0] = v2.x; w[nt][1] = v2.y;
+    for (int ks = 0; ks < D / 16; ++ks)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int d0 = 16 * ks + 8 * h + 2 * qc;
+        const float2 sc = h2f(ksc[d0 / 2]), zc = h2f(kzr[d0 / 2]);
+        const float q0 = bf16_lo(qa[ks][h]), q1 = bf16_hi(qa[ks][h]);
+        split_f16(q0 * sc.x, q1 * sc.y, ah[ks][h], al[ks][h]);
+        cz = fmaf(q0, zc.x, fmaf(q1, zc.y, cz));
       }
-    }
+    cz += __shfl_xor_sync(0xffffffffu, cz, 1);
+    cz += __shfl_xor_sync(0xffffffffu, cz, 2);
+
+    // ---- S = Q K^T over 4 n-tiles of 8 tokens (B = exact nibbles)
     float s[4][4];
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+    for (int nt = 0; nt < 4; ++nt) {
+      s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+      const int t = nt * 8 + qr;
+      uint32_t w[NW];
+      if constexpr (NW == 4) {
+        const uint4 v4 = *reinterpret_cast<const uint4*>(kw + (t * 4 + qc) * NW);
+        w[0] = v4.x; w[1] = v4.y; w[2] = v4.z; w[3] = v4.w;
+      } else {
+        const uint2 v2 = *reinterpret_cast<const uint2*>(kw + (t * 4 + qc) * NW);
+        w[0] = v2.x; w[1] = v2.y;
+      }
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      const int wi = ks >> 1, hk = ks & 1;
-      // per-channel scale / zero of the pairs (16 ks + 2qc, +1) and (16 ks + 8 + 2qc, +1)
-      const uint32_t s0 = ksc[8 * ks + qc], s1 = ksc[8 * ks + 4 + qc];
-      const uint32_t z0 = kzr[8 * ks + qc], z1 = kzr[8 * ks + 4 + qc];
+      for (int wi = 0; wi < NW; ++wi)
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
-        mma_f16(s[nt], qh[ks][0], ql[ks][0], qh[ks][1], ql[ks][1],
-                deq_pair(w[nt][wi], 2 * hk, s0, z0), deq_pair(w[nt][wi], 2 * hk + 1, s1, z1));
+        for (int hk = 0; hk < 2; ++hk) {            // k-step 2wi + hk
+          const int ks = 2 * wi + hk;
+          mma_f16(s[nt], ah[ks][0], al[ks][0], ah[ks][1], al[ks][1], nib_pair(w[wi], 2 * hk),
+                  nib_pair(w[wi], 2 * hk + 1));
+        }
     }
-    // rows qr (high part) + rows qr+8 (low part)
+    // rows qr (high part) + rows qr+8 (low part) + zero-point term
     float mx = -INFINITY;
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
-      s[nt][0] = (s[nt][0] + s[nt][2]) * p.qk_scale2;
-      s[nt][1] = (s[nt][1] + s[nt][3]) * p.qk_scale2;
+      s[nt][0] = (s[nt][0] + s[nt][2] + cz) * p.qk_scale2;
+      s[nt][1] = (s[nt][1] + s[nt][3] + cz) * p.qk_scale2;
       mx = fmaxf(mx, fmaxf(s[nt][0], s[nt][1]));
     }
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -587,35 +619,58 @@ __global__ void __launch_bounds__(128, 3) draft_int4_kernel(const DraftInt4Param
       for (int nn = 0; nn < NT; ++nn) {
         o[nn][0] *= alpha; o[nn][1] *= alpha; o[nn][2] *= alpha; o[nn][3] *= alpha;
       }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) zacc[e] *= alpha;
       m_run = m_new;
     }
     float psum = 0.f;
-    uint32_t ph[4], pl[4];
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
-      const float e0 = ex2(s[nt][0] - m_new), e1 = ex2(s[nt][1] - m_new);
-      psum += e0 + e1;
-      split_f16(e0, e1, ph[nt], pl[nt]);
+      s[nt][0] = ex2(s[nt][0] - m_new);
+      s[nt][1] = ex2(s[nt][1] - m_new);
+      psum += s[nt][0] + s[nt][1];
     }
     l_run += psum;
 
-    // ---- O += P V_hat: word (channel 8 nn + qr, qc), pair j = tokens 2qc + 8j, +1; the
-    //      value group of channel 8 nn + qr is nn / 4, its scales per token pair
+    // ---- zero-point term sum_t p_t z_t: A = p (hi/lo), B = zeros [tokens x groups]
+    {
+      uint32_t ph[4], pl[4];
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) split_f16(s[nt][0], s[nt][1], ph[nt], pl[nt]);
+      // B = z + 7.5 s, the value of the middle of each group's grid (the nibbles of V
+      // enter centred, so both sums stay of the size of the result: no cancellation)
+      auto zmid = [&](int t0) -> uint32_t {
+        const int o = (qr * 32 + t0) / 2;
+        const float2 z = h2f(vzr[o]), sc = h2f(vsc[o]);
+        return pack_f16x2(fmaf(7.5f, sc.x, z.x), fmaf(7.5f, sc.y, z.y));
+      };
+#pragma unroll
+      for (int kt = 0; kt < 2; ++kt) {
+        uint32_t z0 = 0u, z1 = 0u;
+        if (qr < NW) {
+          z0 = zmid(16 * kt + 2 * qc);
+          z1 = zmid(16 * kt + 8 + 2 * qc);
+        }
+        mma_f16(zacc, ph[2 * kt], pl[2 * kt], ph[2 * kt + 1], pl[2 * kt + 1], z0, z1);
+      }
+    }
+    // ---- O += (p s / 2) (2N - 15) per channel group, B = exact doubled centred nibbles
+    float sh[4][2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) { sh[j][0] = 0.5f * s[j][0]; sh[j][1] = 0.5f * s[j][1]; }
 #pragma unroll
     for (int G = 0; G < NW; ++G) {
-      uint32_t vs2[4], vz2[4];
+      uint32_t pah[4], pal[4];                      // [kt * 2 + half]
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        vs2[j] = vsc[(G * 32 + 2 * qc + 8 * j) / 2];
-        vz2[j] = vzr[(G * 32 + 2 * qc + 8 * j) / 2];
+      for (int j = 0; j < 4; ++j) {                 // token pair 2qc + 8j: n-tile j
+        const float2 sv = h2f(vsc[(G * 32 + 2 * qc + 8 * j) / 2]);
+        split_f16(sh[j][0] * sv.x, sh[j][1] * sv.y, pah[j], pal[j]);
       }
 #pragma unroll
       for (int nn = 4 * G; nn < 4 * G + 4; ++nn) {
         const uint32_t wv = vw[(nn * 8 + qr) * 4 + qc];
-        mma_f16(o[nn], ph[0], pl[0], ph[1], pl[1], deq_pair(wv, 0, vs2[0], vz2[0]),
-                deq_pair(wv, 1, vs2[1], vz2[1]));
-        mma_f16(o[nn], ph[2], pl[2], ph[3], pl[3], deq_pair(wv, 2, vs2[2], vz2[2]),
-                deq_pair(wv, 3, vs2[3], vz2[3]));
+        mma_f16(o[nn], pah[0], pal[0], pah[1], pal[1], nib_pair_c2(wv, 0), nib_pair_c2(wv, 1));
+        mma_f16(o[nn], pah[2], pal[2], pah[3], pal[3], nib_pair_c2(wv, 2), nib_pair_c2(wv, 3));
       }
     }
     __syncwarp();

@@ -6,48 +6,37 @@
 // [0, n_q), head h of the GQA group -- sits at absolute position P + i and attends every
 // key at position <= P + i: the whole prefix plus the block, causal inside the block.
 //
-// Decomposition.  A CTA owns one pair, one group of N <= 160 query rows (row r = i * g +
-// h; N is the UMMA N, a multiple of 16, the same for every group of a call) and one split
-// of the keys: the intersection of the call's key range with an absolute window
-// [s * 4096, (s + 1) * 4096).  Split windows and 128-key tiles sit at fixed absolute
-// positions, so a row's result does not depend on n_q or on the other rows (a verify row
-// equals the same token decoded alone).
+// Decomposition.  A CTA owns one pair, one group of <= 256 query rows (two M = 128
+// UMMA tiles; row r = i * g + h) and one split of the keys: the intersection of the
+// call's key range with an absolute window [s * 4096, (s + 1) * 4096).  Split windows
+// and 64-key tiles sit at fixed absolute positions, so a row's result does not depend
+// on n_q or on the other rows (a verify row equals the same token decoded alone).
 //
-// Orientation.  Key positions are the UMMA M = 128 and query rows the N: per 128-key tile
-//     S^T [128 keys x N] = K [128 x D] . Q^T          (A = K tile, B = Q, both K-major)
-//     O^T [D x N]      += V^T [D x 128] . P^T [128 x N]  (A = V tile read MN-major, B = P^T)
-// so a group of 132 rows (k = 32 at g = 4) costs 144 columns of tensor work instead of two
-// M = 128 tiles, and the softmax of a tile is spread over all four TMEM sub-partitions.
-//
-// Per CTA (256 threads):
-//   warp 0, lane 0   TMA producer of K tiles, warp 3 lane 0 of V tiles ([128 keys x 64
-//                    dims] boxes, 128-byte swizzle), each into its own 2-slot ring with a
-//                    full / empty mbarrier pair per slot.
-//   warp 1           TMEM allocator; lane 0 issues every UMMA: QK of tile t as soon as the
-//                    softmax has copied S of tile t-1 out of TMEM, then PV of tile t-1 once
-//                    its P^T is in shared memory.
-//   warps 4-7        softmax: thread (w, lane) owns key 32 (w - 4) + lane of the tile (its
-//                    TMEM lane) and holds that key's N scores.  Scores are in the log2
-//                    domain against a per-row reference maximum m_r that is raised only
-//                    when a tile's scores exceed it by more than 2^8 (the four warps vote
-//                    once per tile; the rare raise finds the exact column maxima with warp
-//                    reductions, then rescales O^T and the sums).  p = 2^(s - m_r) is
-//                    written as bf16 P^T (MN-major, 128-byte swizzle) and summed per
-//                    (key lane, row) in TMEM; the lanes' sums are added in a fixed order at
-//                    the end.  A split's partial (m_r, l_r, unnormalised O) goes to the
-//                    workspace.
-// TMEM columns: O^T [0, 160), S^T [160, 320), per-lane row sums [320, 480).
+// Per CTA (384 threads):
+//   warp 0      TMA producer: K and V tiles [64 keys x D] (128-byte swizzle) into a
+//               6-stage ring, one mbarrier per stage with the transaction byte count.
+//   warp 1      TMEM allocator; one thread of warp 1 (M-tile 0) and one of warp 2
+//   warp 2      (M-tile 1) issue the UMMAs: the tile's next S = Q K^T as soon as its
+//               softmax has copied the current S out of TMEM, then O += P V once its
+//               P is in.  Q of M-tile 0 is read from TMEM, Q of M-tile 1 from shared
+//               memory; P from TMEM, K and V from shared memory (V as an N-major B).
+//   warps 4-7   softmax of M-tile 0, warps 8-11 of M-tile 1: one thread per query row
+//               (TMEM lane); M-tile 1 keeps row r in lane (r + 64) % 128, so a part-
+//               filled second tile lands on sub-partitions 2-3.  Scores in the log2
+//               domain, running max kept unless it grows by more than 2^8 (then O in
+//               TMEM is rescaled after the previous P.V), P written as bf16 into the
+//               M-tile's P columns once the previous P.V has read them.
+// TMEM columns: O0 [0,D), O1 [D,2D), S0, S1 (64 each), P0, P1 (32 each), Q0 (D/2).
 // Every mbarrier wait is bounded in time (pipeline waits by a launch parameter, 2 s
 // unless vc_set_wait_limit changed it; teardown waits by 1 s); on expiry the CTA raises
 // the library's device error word, lets its copies and products in flight land,
 // releases TMEM and exits.
-// The split partials are merged by a second kernel in split order, optionally together
-// with a carried state for chunked (streamed) keys.
+// The split partials (max, sum, unnormalised O) are merged by a second kernel in
+// split order, optionally together with a carried state for chunked (streamed) keys.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <atomic>
-#include <climits>
 
 #include "tc05.cuh"
 #include "vc_common.cuh"
@@ -58,16 +47,14 @@ namespace vc {
 __device__ int g_vc_dev_error;   // bit 0: a bounded wait in the verify kernel expired
 
 constexpr int kSplitKeys = 4096;
-constexpr int kBN = 128;          // keys per tile (UMMA M)
-constexpr int kNMax = 160;        // query rows per CTA (UMMA N <= kNMax)
-constexpr int kVThreads = 256;
+constexpr int kBN = 64;
+constexpr int kVThreads = 384;
+constexpr int kNSt = 6;
 constexpr float kRescaleLog2 = 8.f;
-constexpr float kPadRowMax = 1e30f;   // reference maximum of padding rows: p = 0, no votes
 
 struct VerifyParams {
   const __nv_bfloat16* q;   // [B, n_q, Hq, D]
   int n_q, Hq, Hkv, g, R;   // R = n_q * g rows per pair
-  int N;                    // rows per CTA group (multiple of 16, <= kNMax)
   int64_t kv_start, kv_len, P;
   int split0, n_split;
   float qk_scale2;          // scale * log2(e)
@@ -78,42 +65,25 @@ struct VerifyParams {
 
 template <int D>
 struct VLayout {
-  static constexpr int kQBlk = kNMax * 128;             // 64 dims of the group's Q rows
-  static constexpr int kKVBlk = kBN * 128;              // 64 dims of a K or V tile
-  static constexpr int kKVSlot = (D / 64) * kKVBlk;
-  static constexpr int kPBlk = kBN * 128;               // 64 rows of P^T (one 128 B row per key)
-  static constexpr int kPBlocks = (kNMax + 63) / 64;
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + (D / 64) * kQBlk;
-  static constexpr int kV = kK + 2 * kKVSlot;
-  static constexpr int kP = kV + 2 * kKVSlot;
-  static constexpr int kBar = kP + kPBlocks * kPBlk;
-  static constexpr int kNBar = 17;
+  static constexpr int kQTile = 128 * D * 2;        // Q of M-tile 1 (128-byte swizzle)
+  static constexpr int kKVTile = kBN * D * 2;
+  static constexpr int kQ1 = 0;
+  static constexpr int kK = kQ1 + kQTile;
+  static constexpr int kV = kK + kNSt * kKVTile;
+  static constexpr int kBar = kV + kNSt * kKVTile;
+  static constexpr int kNBar = 2 * kNSt + 2 + 2 + 2 + 2 + 1;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
-  static constexpr int kFlags = kAbort + 4;              // int [2][4] votes
-  static constexpr int kMUsed = kFlags + 48;             // float [kNMax] reference maxima
-  static constexpr int kAlpha = kMUsed + kNMax * 4;      // float [kNMax] rescale factors
-  static constexpr int kWMax = kAlpha + kNMax * 4;       // float [4][kNMax] warp maxima
-  static constexpr int kTotal = kWMax + 4 * kNMax * 4;
+  static constexpr int kTotal = kAbort + 4;
   static constexpr int kAlloc = kTotal + 1024;
-  static constexpr int kRedStride = kNMax + 1;           // row sums, per key lane (floats)
-  static constexpr uint32_t kColO = 0, kColS = kNMax, kColL = 2 * kNMax;
+  static constexpr uint32_t kColO = 0;
+  static constexpr uint32_t kColS = 2 * D;
+  static constexpr uint32_t kColP = 2 * D + 2 * kBN;
+  static constexpr uint32_t kColQ0 = kColP + 2 * (kBN / 2);
   static constexpr uint32_t kTmemCols = 512;
-  static_assert(kColL + kNMax <= kTmemCols, "TMEM columns");
-  static_assert(kK % 1024 == 0 && kV % 1024 == 0 && kP % 1024 == 0, "align");
-  static_assert(kMUsed % 16 == 0, "align");
-  static_assert(kAlloc <= 232448, "shared memory");
-  static_assert(128 * kRedStride * 4 <= kBar - kK, "row-sum staging fits the idle K/V/P buffers");
+  static_assert(kColQ0 + D / 2 <= kTmemCols, "TMEM columns");
+  static_assert(kQTile % 1024 == 0 && kKVTile % 1024 == 0, "align");
 };
-
-// Largest value over the warp (no NaN), through the order-preserving integer image.
-__device__ __forceinline__ float warp_max_f32(float v) {
-  const int i = __float_as_int(v);
-  int key = i >= 0 ? i : (i ^ 0x7fffffff);
-  key = __reduce_max_sync(0xffffffffu, key);
-  return __int_as_float(key >= 0 ? key : (key ^ 0x7fffffff));
-}
 
 template <int D>
 __global__ void __launch_bounds__(kVThreads, 1)
@@ -129,9 +99,9 @@ __global__ void __launch_bounds__(kVThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s_local = blockIdx.x, rg = blockIdx.y, pair = blockIdx.z;
   const int b = pair / p.Hkv, kvh = pair - b * p.Hkv;
-  const int N = p.N;
-  const int row0 = rg * N;
-  const int rows_here = min(N, p.R - row0);
+  const int row0 = rg * 256;
+  const int rows_here = min(256, p.R - row0);
+  const int n_mt = (rows_here + 127) >> 7;
   const int64_t part = (int64_t)pair * p.n_split + s_local;
 
   // key range of this split seen by this row group
@@ -153,151 +123,168 @@ __global__ void __launch_bounds__(kVThreads, 1)
   }
 
   auto bar = [&](int i) -> uint32_t { return sb + L::kBar + 8 * i; };
-  auto b_k_full = [&](int s) { return bar(s); };
-  auto b_k_empty = [&](int s) { return bar(2 + s); };
-  auto b_v_full = [&](int s) { return bar(4 + s); };
-  auto b_v_empty = [&](int s) { return bar(6 + s); };
-  const uint32_t b_s_full = bar(8), b_s_free = bar(9), b_p_full = bar(10), b_o_done = bar(11);
-  const uint32_t b_teardown = bar(12);
-  // syncs of the four softmax warps (one arrival per warp): the tile's vote, the raise of
-  // the reference maxima (two steps, only in tiles that raise), the end of the row sums
-  const uint32_t b_vote = bar(13), b_wmax = bar(14), b_mnew = bar(15), b_sums = bar(16);
+  auto b_kv_full = [&](int st) { return bar(st); };
+  auto b_kv_empty = [&](int st) { return bar(kNSt + st); };
+  auto b_s_full = [&](int mt) { return bar(2 * kNSt + mt); };
+  auto b_s_free = [&](int mt) { return bar(2 * kNSt + 2 + mt); };
+  auto b_p_full = [&](int mt) { return bar(2 * kNSt + 4 + mt); };
+  auto b_o_done = [&](int mt) { return bar(2 * kNSt + 6 + mt); };
+  const uint32_t b_teardown = bar(2 * kNSt + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
-  volatile int* votes = reinterpret_cast<volatile int*>(smem + L::kFlags);
-  float* m_used = reinterpret_cast<float*>(smem + L::kMUsed);
-  float* alpha = reinterpret_cast<float*>(smem + L::kAlpha);
-  float* wmax = reinterpret_cast<float*>(smem + L::kWMax);
+  auto nw_active = [&](int mt) {
+    const int v = min(128, rows_here - mt * 128);
+    return v > 0 ? (v + 31) >> 5 : 0;
+  };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(b_k_full(s), 1);
-      tc::mbar_init(b_k_empty(s), 1);
-      tc::mbar_init(b_v_full(s), 1);
-      tc::mbar_init(b_v_empty(s), 1);
+    for (int st = 0; st < kNSt; ++st) {
+      tc::mbar_init(b_kv_full(st), 1);
+      tc::mbar_init(b_kv_empty(st), n_mt);      // released by each M-tile's issuer
     }
-    tc::mbar_init(b_s_full, 1);
-    tc::mbar_init(b_s_free, 4);
-    tc::mbar_init(b_p_full, 4);
-    tc::mbar_init(b_o_done, 1);
-    tc::mbar_init(b_teardown, 1);
-    tc::mbar_init(b_vote, 4);
-    tc::mbar_init(b_wmax, 4);
-    tc::mbar_init(b_mnew, 4);
-    tc::mbar_init(b_sums, 4);
+    for (int mt = 0; mt < 2; ++mt) {
+      tc::mbar_init(b_s_full(mt), 1);
+      tc::mbar_init(b_s_free(mt), max(1, nw_active(mt)));
+      tc::mbar_init(b_p_full(mt), max(1, nw_active(mt)));
+      tc::mbar_init(b_o_done(mt), 1);
+    }
+    tc::mbar_init(b_teardown, n_mt);
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
-  for (int c = threadIdx.x; c < kNMax; c += kVThreads)
-    m_used[c] = c < rows_here ? -INFINITY : kPadRowMax;
-  // Q rows of this group into shared memory: K-major, 128-byte swizzle, one 128 B row per
-  // query row and 64 dims; rows past the group's are zero
-  for (int idx = threadIdx.x; idx < kNMax * (D / 8); idx += kVThreads) {
-    const int r = idx / (D / 8), ch = idx - r * (D / 8);
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < rows_here) {
-      const int grow = row0 + r;
-      const int i = grow / p.g, hl = grow - i * p.g;
-      v = __ldg(reinterpret_cast<const uint4*>(
-                    p.q + (((int64_t)b * p.n_q + i) * p.Hq + kvh * p.g + hl) * D) + ch);
-    }
-    const int cb = ch >> 3, cc = ch & 7;
-    *reinterpret_cast<uint4*>(smem + L::kQ + cb * L::kQBlk + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
-  }
-  tc::fence_proxy_async();
   if (warp == 1) tc::tmem_alloc(sb + L::kTmemSlot, L::kTmemCols);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlot);
 
+  // Q rows of this group: M-tile 0 into TMEM (row r in lane r, two bf16 per column), M-tile
+  // 1 into shared memory (K-major, 128-byte swizzle, row r at row (r + 64) % 128);
+  // padding rows are zero.
+  if (warp >= 4) {
+    const int mt = (warp - 4) >> 2, q4 = warp & 3;
+    const int rl = 32 * q4 + lane;                       // TMEM lane / UMMA row
+    const int grow = row0 + mt * 128 + ((rl + (mt ? 64 : 0)) & 127);
+    const bool ok = mt < n_mt && grow < row0 + rows_here;
+    const uint4* src = nullptr;
+    if (ok) {
+      const int i = grow / p.g, hl = grow - i * p.g;
+      src = reinterpret_cast<const uint4*>(p.q + (((int64_t)b * p.n_q + i) * p.Hq + kvh * p.g + hl) * D);
+    }
+    if (mt == 0) {
+      const uint32_t q_t = tmem + ((uint32_t)(32 * q4) << 16) + L::kColQ0;
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t w[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 v = ok ? __ldg(src + 8 * c + u) : make_uint4(0u, 0u, 0u, 0u);
+          w[4 * u] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
+        }
+        tc::tmem_st32(q_t + 32 * c, w);
+      }
+      tc::tmem_wait_st();
+    } else {
+#pragma unroll
+      for (int ch = 0; ch < D / 8; ++ch) {
+        const uint4 v = ok ? __ldg(src + ch) : make_uint4(0u, 0u, 0u, 0u);
+        const int cb = ch >> 3, cc = ch & 7;
+        *reinterpret_cast<uint4*>(smem + L::kQ1 + cb * (128 * 128) + rl * 128 +
+                                  ((cc ^ (rl & 7)) << 4)) = v;
+      }
+      tc::fence_proxy_async();
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+
   auto raise = [&]() {
     *abort_flag = 1;
     atomicOr(&g_vc_dev_error, 1);
   };
 
-  if ((warp == 0 || warp == 3) && lane == 0) {
-    // ------------------------------------------------------------ TMA producers
-    const bool is_k = warp == 0;
-    const CUtensorMap* map = is_k ? &tmK : &tmV;
-    const uint32_t base = sb + (is_k ? L::kK : L::kV);
-    tc::prefetch_tmap(map);
-    int issued = 0;
-    for (int t = 0; t < n_tiles; ++t) {
-      const int s = t & 1;
-      const uint32_t fb = is_k ? b_k_full(s) : b_v_full(s);
-      const uint32_t eb = is_k ? b_k_empty(s) : b_v_empty(s);
-      if (t >= 2 && !tc::mbar_wait(eb, ((t >> 1) - 1) & 1, abort_flag, p.wait_ns)) {
-        raise();
-        break;
-      }
-      tc::mbar_expect_tx(fb, L::kKVSlot);
-      const int y = (int)((tile0 + t) * kBN - p.kv_start);
-#pragma unroll
-      for (int cb = 0; cb < D / 64; ++cb)
-        tc::tma_load_3d(base + s * L::kKVSlot + cb * L::kKVBlk, map, fb, cb * 64, y, pair);
-      issued = t + 1;
-    }
-    // loads still in flight must land before shared memory is released
-    for (int t = max(0, issued - 2); t < issued; ++t)
-      tc::mbar_wait(is_k ? b_k_full(t & 1) : b_v_full(t & 1), (t >> 1) & 1, nullptr,
-                    1000000000ull);
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ UMMA issuer
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const uint32_t id_qk = tc::idesc_bf16_f32(128, N, false, false);
-      const uint32_t id_pv = tc::idesc_bf16_f32(128, N, true, true);
+      tc::prefetch_tmap(&tmK);
+      tc::prefetch_tmap(&tmV);
+      int issued = 0;
+      for (int t = 0; t < n_tiles; ++t) {
+        const int st = t % kNSt;
+        if (t >= kNSt && !tc::mbar_wait(b_kv_empty(st), ((t / kNSt) - 1) & 1, abort_flag, p.wait_ns)) {
+          raise();
+          break;
+        }
+        const uint32_t fb = b_kv_full(st);
+        tc::mbar_expect_tx(fb, 2 * L::kKVTile);
+        const int y = (int)((tile0 + t) * kBN - p.kv_start);
+#pragma unroll
+        for (int cb = 0; cb < D / 64; ++cb) {
+          tc::tma_load_3d(sb + L::kK + st * L::kKVTile + cb * (kBN * 128), &tmK, fb, cb * 64, y,
+                          pair);
+          tc::tma_load_3d(sb + L::kV + st * L::kKVTile + cb * (kBN * 128), &tmV, fb, cb * 64, y,
+                          pair);
+        }
+        issued = t + 1;
+      }
+      // loads still in flight must land before shared memory is released
+      for (int t = max(0, issued - kNSt); t < issued; ++t)
+        tc::mbar_wait(b_kv_full(t % kNSt), (t / kNSt) & 1, nullptr, 1000000000ull);
+    }
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ UMMA issuers
+    // One thread per M-tile (warp 1: M-tile 0, warp 2: M-tile 1), so neither tile's
+    // products wait behind the other tile's softmax.
+    const int mt = warp - 1;
+    if (lane == 0 && mt < n_mt) {
+      const uint32_t id_qk = tc::idesc_bf16_f32(128, kBN, false, false);
+      const uint32_t id_pv = tc::idesc_bf16_f32(128, D, false, true);
       auto qk = [&](int t) {
-        const int s = t & 1;
+        const int st = t % kNSt;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t a = sb + L::kK + s * L::kKVSlot + (ks >> 2) * L::kKVBlk + (ks & 3) * 32;
-          const uint32_t bq = sb + L::kQ + (ks >> 2) * L::kQBlk + (ks & 3) * 32;
-          tc::umma_ss(tmem + L::kColS, tc::sdesc_sw128(a, 16, 1024), tc::sdesc_sw128(bq, 16, 1024),
-                      id_qk, ks > 0 ? 1u : 0u);
+          const uint32_t bb = sb + L::kK + st * L::kKVTile + (ks >> 2) * (kBN * 128) + (ks & 3) * 32;
+          const uint64_t bdesc = tc::sdesc_sw128(bb, 16, 1024);
+          if (mt == 0) {
+            tc::umma_ts(tmem + L::kColS, tmem + L::kColQ0 + ks * 8, bdesc, id_qk, ks > 0 ? 1u : 0u);
+          } else {
+            const uint32_t a = sb + L::kQ1 + (ks >> 2) * (128 * 128) + (ks & 3) * 32;
+            tc::umma_ss(tmem + L::kColS + kBN, tc::sdesc_sw128(a, 16, 1024), bdesc, id_qk,
+                        ks > 0 ? 1u : 0u);
+          }
         }
       };
       auto pv = [&](int t) {
-        const int s = t & 1;
+        const int st = t % kNSt;
 #pragma unroll
         for (int ks = 0; ks < kBN / 16; ++ks) {
-          // A = V^T: dims contiguous in each key's 128 B row (64 dims per block, blocks
-          // L::kKVBlk apart; at D = 64 the second half of M re-reads the first block)
-          const uint32_t a = sb + L::kV + s * L::kKVSlot + ks * 16 * 128;
-          const uint32_t bp = sb + L::kP + ks * 16 * 128;
-          tc::umma_ss(tmem + L::kColO, tc::sdesc_sw128(a, D == 128 ? L::kKVBlk : 0, 1024),
-                      tc::sdesc_sw128(bp, L::kPBlk, 1024), id_pv,
-                      (t > 0 || ks > 0) ? 1u : 0u);
+          const uint32_t bb = sb + L::kV + st * L::kKVTile + ks * 16 * 128;
+          tc::umma_ts(tmem + L::kColO + mt * D, tmem + L::kColP + mt * (kBN / 2) + ks * 8,
+                      tc::sdesc_sw128(bb, kBN * 128, 1024), id_pv, (t > 0 || ks > 0) ? 1u : 0u);
         }
       };
-      bool ok = true;
-      for (int t = 0; t < n_tiles && ok; ++t) {
-        if (!(ok = tc::mbar_wait(b_k_full(t & 1), (t >> 1) & 1, abort_flag, p.wait_ns))) break;
-        if (t > 0 && !(ok = tc::mbar_wait(b_s_free, (t - 1) & 1, abort_flag, p.wait_ns))) break;
-        tc::tc_fence_after();
-        qk(t);
-        tc::umma_commit(b_s_full);
-        tc::umma_commit(b_k_empty(t & 1));
-        if (t > 0) {
-          if (!(ok = tc::mbar_wait(b_p_full, (t - 1) & 1, abort_flag, p.wait_ns))) break;
-          if (!(ok = tc::mbar_wait(b_v_full((t - 1) & 1), ((t - 1) >> 1) & 1, abort_flag,
-                                   p.wait_ns)))
-            break;
-          tc::tc_fence_after();
-          pv(t - 1);
-          tc::umma_commit(b_o_done);
-          tc::umma_commit(b_v_empty((t - 1) & 1));
-        }
-      }
+      bool ok = tc::mbar_wait(b_kv_full(0), 0, abort_flag, p.wait_ns);
       if (ok) {
-        const int t = n_tiles - 1;
-        ok = tc::mbar_wait(b_p_full, t & 1, abort_flag, p.wait_ns) &&
-             tc::mbar_wait(b_v_full(t & 1), (t >> 1) & 1, abort_flag, p.wait_ns);
-        if (ok) {
+        tc::tc_fence_after();
+        qk(0);
+        tc::umma_commit(b_s_full(mt));
+      }
+      for (int t = 0; ok && t < n_tiles; ++t) {
+        if (t + 1 < n_tiles) {
+          // the next Q K^T as soon as the softmax has copied this S out of TMEM
+          if (!(ok = tc::mbar_wait(b_kv_full((t + 1) % kNSt), ((t + 1) / kNSt) & 1,
+                                   abort_flag, p.wait_ns)))
+            break;
+          if (!(ok = tc::mbar_wait(b_s_free(mt), t & 1, abort_flag, p.wait_ns))) break;
           tc::tc_fence_after();
-          pv(t);
-          tc::umma_commit(b_o_done);
-          tc::umma_commit(b_v_empty(t & 1));
+          qk(t + 1);
+          tc::umma_commit(b_s_full(mt));
         }
+        if (!(ok = tc::mbar_wait(b_p_full(mt), t & 1, abort_flag, p.wait_ns))) break;
+        tc::tc_fence_after();
+        pv(t);
+        tc::umma_commit(b_o_done(mt));
+        tc::umma_commit(b_kv_empty(t % kNSt));   // one arrival per M-tile
       }
       if (!ok) raise();
       // every UMMA issued must retire before TMEM is released
@@ -307,225 +294,130 @@ __global__ void __launch_bounds__(kVThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
-    const int q4 = warp - 4;
-    const int key_lane = 32 * q4 + lane;
-    const int tid_s = threadIdx.x - 128;
-    const uint32_t lane_t = tmem + ((uint32_t)(32 * q4) << 16);
-    const uint32_t s_t = lane_t + L::kColS, o_t = lane_t + L::kColO, l_t = lane_t + L::kColL;
-    const int nch = (N + 31) >> 5;
-    const float sc2 = p.qk_scale2;
-    // the four softmax warps meet on an mbarrier (bounded wait: a warp that gave up never
-    // arrives, and the others give up in turn instead of hanging)
-    auto sync4 = [&](uint32_t bar4, uint32_t phase) -> bool {
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar4);
-      return __all_sync(0xffffffffu, tc::mbar_wait(bar4, phase, abort_flag, p.wait_ns));
-    };
-    // S columns [N, 32 nch) are read with the last 32-column load but never written by
-    // the UMMA: zero them once (disjoint from the columns Q K^T writes)
-    if (N & 16) {
-      tc::tmem_st16_zero(s_t + N);
-      tc::tmem_wait_st();
-    }
-    bool ok = true;
-    int n_raise = 0;                          // tiles that raised a reference maximum
-    for (int t = 0; t < n_tiles; ++t) {
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(b_s_full, t & 1, abort_flag, p.wait_ns));
-      if (!ok) break;
-      tc::tc_fence_after();
-      float s[kNMax];
+    const int mt = (warp - 4) >> 2, q4 = warp & 3;
+    const int valid_mt = min(128, rows_here - mt * 128);
+    const int rot = mt ? 64 : 0;
+    if (mt < n_mt && ((32 * q4 + rot) & 127) < valid_mt) {
+      const int r = (32 * q4 + lane + rot) & 127;
+      const int grow = row0 + mt * 128 + r;
+      const bool row_ok = r < valid_mt;
+      const int64_t limit = p.P + grow / p.g;
+      const uint32_t lane_t = tmem + ((uint32_t)(32 * q4) << 16);
+      const uint32_t s_t = lane_t + L::kColS + mt * kBN;
+      const uint32_t p_t = lane_t + L::kColP + mt * (kBN / 2);
+      const uint32_t o_t = lane_t + L::kColO + mt * D;
+      float m_used = -INFINITY, lsum = 0.f;
+      bool ok = true;
+      for (int t = 0; t < n_tiles; ++t) {
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(b_s_full(mt), t & 1, abort_flag, p.wait_ns));
+        if (!ok) break;
+        tc::tc_fence_after();
+        uint32_t sr[64];
+        tc::tmem_ld32(s_t, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tc::tmem_ld32(s_t + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tc::tmem_wait_ld();
+        // S is in registers: the next Q K^T may overwrite it
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(b_s_free(mt));
+        // visible columns j in [lo, hi] of this tile for this row (int32, clamped); a
+        // padding row counts as seeing the whole tile (its values are never used)
+        const int64_t key0 = (tile0 + t) * kBN;
+        const int lo = row_ok ? (int)max((int64_t)0, min((int64_t)kBN, a0 - key0)) : 0;
+        const int hi = row_ok
+            ? (int)max((int64_t)-1, min((int64_t)(kBN - 1), min(a1 - 1, limit) - key0))
+            : kBN - 1;
+        // Row max on the raw scores (the scale is positive, so it commutes with max);
+        // a tile every row of the warp sees whole skips the per-column mask.
+        // (eight independent partial maxima: a short dependency chain)
+        float mx8[8];
 #pragma unroll
-      for (int c = 0; c < kNMax / 32; ++c)
-        if (c < nch) tc::tmem_ld32(s_t + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
-      tc::tmem_wait_ld();
-      // S is in registers: the next Q K^T may overwrite it
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(b_s_free);
-
-      // the group's columns c >= r_min see this thread's key: row row0 + c sits at
-      // position P + (row0 + c) / g (none if the key is outside the split's range)
-      const int64_t key = (tile0 + t) * kBN + key_lane;
-      const bool kv_ok = key >= a0 && key < a1;
-      const int64_t rm = (key - p.P) * p.g - row0;
-      const int r_min = !kv_ok ? INT_MAX : rm <= 0 ? 0 : (int)min((int64_t)INT_MAX, rm);
-      const bool whole = __all_sync(0xffffffffu, r_min == 0);
-      auto valid = [&](int c) { return whole || c >= r_min; };
-
-      // vote: does any score exceed its row's reference maximum by more than 2^8?
-      float mx = -INFINITY;
+        for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
+        if (__all_sync(0xffffffffu, lo == 0 && hi == kBN - 1)) {
 #pragma unroll
-      for (int c = 0; c < kNMax; c += 4) {
-        if (c < 32 * nch) {
-          const float4 m4 = *reinterpret_cast<const float4*>(m_used + c);
-          const float e0 = fmaf(s[c], sc2, -m4.x), e1 = fmaf(s[c + 1], sc2, -m4.y);
-          const float e2 = fmaf(s[c + 2], sc2, -m4.z), e3 = fmaf(s[c + 3], sc2, -m4.w);
-          if (whole) {
-            mx = fmaxf(mx, fmaxf(fmaxf(e0, e1), fmaxf(e2, e3)));
-          } else {
-            if (valid(c)) mx = fmaxf(mx, e0);
-            if (valid(c + 1)) mx = fmaxf(mx, e1);
-            if (valid(c + 2)) mx = fmaxf(mx, e2);
-            if (valid(c + 3)) mx = fmaxf(mx, e3);
+          for (int j = 0; j < 64; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(sr[j]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            const float v = (j >= lo && j <= hi) ? __uint_as_float(sr[j]) : -INFINITY;
+            sr[j] = __float_as_uint(v);
+            mx8[j & 7] = fmaxf(mx8[j & 7], v);
           }
         }
-      }
-      const int vote = __any_sync(0xffffffffu, mx > kRescaleLog2) ? 1 : 0;
-      if (lane == 0) votes[(t & 1) * 4 + q4] = vote;
-      if (!(ok = sync4(b_vote, t & 1))) break;
-      const bool exceed = (votes[(t & 1) * 4] | votes[(t & 1) * 4 + 1] | votes[(t & 1) * 4 + 2] |
-                           votes[(t & 1) * 4 + 3]) != 0;
-      bool waited_o = false;
-      if (exceed) {
-        // exact maxima of this tile per row, then raise the rows that need it
+        const float mraw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float mx = mraw * p.qk_scale2;
+        const float m_new = fmaxf(m_used, mx);
+        const bool resc = m_new > m_used + kRescaleLog2;
+        const float alpha = resc ? ex2(m_used - m_new) : 1.f;
+        if (resc) m_used = m_new;
+        const float m_safe = m_used == -INFINITY ? 0.f : m_used;
+        // P (bf16, keys packed two per column) in registers first -- it does not depend on
+        // O -- so the exponentials overlap the previous P.V; row sum in eight partial sums
+        // added in a fixed order
+        uint32_t pw[32];
+        float rs8[8];
 #pragma unroll
-        for (int c = 0; c < kNMax; ++c) {
-          if (c < 32 * nch) {
-            const float v = warp_max_f32(valid(c) ? s[c] * sc2 : -INFINITY);
-            if (lane == 0) wmax[q4 * kNMax + c] = v;
-          }
+        for (int u = 0; u < 8; ++u) rs8[u] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float e0 = ex2(fmaf(__uint_as_float(sr[2 * c]), p.qk_scale2, -m_safe));
+          const float e1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), p.qk_scale2, -m_safe));
+          rs8[(2 * c) & 7] += e0;
+          rs8[(2 * c + 1) & 7] += e1;
+          pw[c] = pack_bf16x2(e0, e1);
         }
-        if (!(ok = sync4(b_wmax, n_raise & 1))) break;
-        for (int c = tid_s; c < 32 * nch; c += 128) {
-          const float m_old = m_used[c];
-          const float tm = fmaxf(fmaxf(wmax[c], wmax[kNMax + c]),
-                                 fmaxf(wmax[2 * kNMax + c], wmax[3 * kNMax + c]));
-          const float m_new = fmaxf(m_old, tm);
-          float a = 1.f;
-          if (m_new > m_old + kRescaleLog2) {
-            a = m_old == -INFINITY ? 0.f : ex2(m_old - m_new);
-            m_used[c] = m_new;
-          }
-          alpha[c] = a;
-        }
-        if (!(ok = sync4(b_mnew, n_raise & 1))) break;
-        ++n_raise;
+        // the previous P.V must be done before O is rescaled or P overwritten
         if (t > 0) {
-          // O^T (lane = head dim) scaled per row once the previous P.V is done
-          ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done, (t - 1) & 1, abort_flag, p.wait_ns));
+          ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt), (t - 1) & 1, abort_flag, p.wait_ns));
           if (!ok) break;
           tc::tc_fence_after();
-          waited_o = true;
+        }
+        if (t > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll
-          for (int c = 0; c < kNMax / 32; ++c) {
-            if (c < nch) {
-              uint32_t o[32];
-              tc::tmem_ld32(o_t + 32 * c, o);
-              tc::tmem_wait_ld();
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tc::tmem_ld32(o_t + 32 * c, o);
+            tc::tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 32; ++e)
-                o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha[32 * c + e]);
-              tc::tmem_st32(o_t + 32 * c, o);
-            }
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tc::tmem_st32(o_t + 32 * c, o);
           }
           tc::tmem_wait_st();
         }
+        lsum *= alpha;
+        tc::tmem_st32(p_t, pw);
+        lsum += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(b_p_full(mt));
       }
-      // p = 2^(s - m_r), 0 where the key is not visible
-#pragma unroll
-      for (int c = 0; c < kNMax; c += 4) {
-        if (c < 32 * nch) {
-          const float4 m4 = *reinterpret_cast<const float4*>(m_used + c);
-          const float e0 = ex2(fmaf(s[c], sc2, -m4.x)), e1 = ex2(fmaf(s[c + 1], sc2, -m4.y));
-          const float e2 = ex2(fmaf(s[c + 2], sc2, -m4.z)), e3 = ex2(fmaf(s[c + 3], sc2, -m4.w));
-          s[c] = valid(c) ? e0 : 0.f;
-          s[c + 1] = valid(c + 1) ? e1 : 0.f;
-          s[c + 2] = valid(c + 2) ? e2 : 0.f;
-          s[c + 3] = valid(c + 3) ? e3 : 0.f;
-        }
+      if (ok) {
+        const int tl = n_tiles - 1;
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done(mt), tl & 1, abort_flag, p.wait_ns));
       }
-      // the previous P.V must be done before P^T is overwritten
-      if (t > 0 && !waited_o) {
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(b_o_done, (t - 1) & 1, abort_flag, p.wait_ns));
-        if (!ok) break;
+      if (!ok) {
+        raise();
+      } else {
         tc::tc_fence_after();
-      }
-      // this lane's row sums: L = L * alpha + p
+        const int64_t o_row = part * p.R + grow;
 #pragma unroll
-      for (int c = 0; c < kNMax / 32; ++c) {
-        if (c < nch) {
-          uint32_t lr[32];
-          if (t > 0) {
-            tc::tmem_ld32(l_t + 32 * c, lr);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float a = exceed ? alpha[32 * c + e] : 1.f;
-              lr[e] = __float_as_uint(fmaf(__uint_as_float(lr[e]), a, s[32 * c + e]));
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) lr[e] = __float_as_uint(s[32 * c + e]);
-          }
-          tc::tmem_st32(l_t + 32 * c, lr);
-        }
-      }
-      // P^T: bf16, MN-major with 128-byte swizzle: 64-row blocks, key k's 64 rows in one
-      // 128-byte line of its block, 16-byte chunk j at position j ^ (k & 7)
-      uint8_t* pbase = smem + L::kP + key_lane * 128;
-#pragma unroll
-      for (int c8 = 0; c8 < kNMax / 8; ++c8) {
-        if (c8 < (N >> 3)) {
-          const int c = 8 * c8;
-          const uint4 w = make_uint4(pack_bf16x2(s[c], s[c + 1]), pack_bf16x2(s[c + 2], s[c + 3]),
-                                     pack_bf16x2(s[c + 4], s[c + 5]),
-                                     pack_bf16x2(s[c + 6], s[c + 7]));
-          *reinterpret_cast<uint4*>(pbase + (c8 >> 3) * L::kPBlk +
-                                    (((c8 & 7) ^ (key_lane & 7)) << 4)) = w;
-        }
-      }
-      tc::tmem_wait_st();
-      tc::fence_proxy_async();
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(b_p_full);
-    }
-    if (ok)
-      ok = __all_sync(0xffffffffu,
-                      tc::mbar_wait(b_o_done, (n_tiles - 1) & 1, abort_flag, p.wait_ns));
-    if (ok && *abort_flag) ok = false;       // another role gave up: loads may be in flight
-    float* red = reinterpret_cast<float*>(smem + L::kK);
-    if (ok) {
-      tc::tc_fence_after();
-      // row sums: each key lane's partial sums to shared memory (the K/V and P buffers are idle
-      // now), then every row added over the 128 lanes in order
-#pragma unroll
-      for (int c = 0; c < kNMax / 32; ++c) {
-        if (c < nch) {
-          uint32_t lr[32];
-          tc::tmem_ld32(l_t + 32 * c, lr);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) red[key_lane * L::kRedStride + 32 * c + e] = __uint_as_float(lr[e]);
-        }
-      }
-      ok = sync4(b_sums, 0);
-    }
-    if (!ok) {
-      raise();
-    } else {
-      for (int c = tid_s; c < rows_here; c += 128) {
-        float l = 0.f;
-        for (int k = 0; k < kBN; ++k) l += red[k * L::kRedStride + c];
-        const int64_t o_row = part * p.R + row0 + c;
-        p.ws_ml[o_row * 2] = m_used[c];
-        p.ws_ml[o_row * 2 + 1] = l;
-      }
-      // O^T: lane = head dim; a warp writes 32 consecutive dims of one row per store
-#pragma unroll
-      for (int c = 0; c < kNMax / 32; ++c) {
-        if (c < nch) {
+        for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
           tc::tmem_ld32(o_t + 32 * c, o);
           tc::tmem_wait_ld();
-          if (key_lane < D) {
+          if (row_ok) {
+            float4* dst = reinterpret_cast<float4*>(p.ws_o + o_row * D + 32 * c);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int col = 32 * c + e;
-              if (col < rows_here)
-                p.ws_o[(part * p.R + row0 + col) * D + key_lane] = __uint_as_float(o[e]);
-            }
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                   __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
           }
+        }
+        if (row_ok) {
+          p.ws_ml[o_row * 2] = m_used;
+          p.ws_ml[o_row * 2 + 1] = lsum;
         }
       }
     }
@@ -662,7 +554,7 @@ bool make_kv_map(CUtensorMap* m, const void* base, int D, int64_t kv_len, int64_
 }
 
 struct Plan {
-  int pairs, g, R, split0, n_split, n_rg, N;
+  int pairs, g, R, split0, n_split, n_rg;
   size_t ws_bytes;
 };
 
@@ -673,10 +565,7 @@ Plan plan(int B, int n_q, int Hq, int Hkv, int D, int64_t kv_start, int64_t kv_l
   pl.R = n_q * pl.g;
   pl.split0 = (int)(kv_start / kSplitKeys);
   pl.n_split = (int)((kv_start + kv_len - 1) / kSplitKeys) - pl.split0 + 1;
-  // row groups of at most kNMax rows, all of the same size N (a multiple of 16)
-  pl.n_rg = (pl.R + kNMax - 1) / kNMax;
-  const int per = (pl.R + pl.n_rg - 1) / pl.n_rg;
-  pl.N = (per + 15) / 16 * 16;
+  pl.n_rg = (pl.R + 255) / 256;
   pl.ws_bytes = (size_t)pl.pairs * pl.n_split * pl.R * ((size_t)D + 2) * sizeof(float);
   return pl;
 }
@@ -737,7 +626,6 @@ vc_status launch_verify(const void* q, int B, int n_q, int Hq, int Hkv, int D, c
   vp.Hkv = Hkv;
   vp.g = pl.g;
   vp.R = pl.R;
-  vp.N = pl.N;
   vp.kv_start = kv_start;
   vp.kv_len = kv_len;
   vp.P = P;
