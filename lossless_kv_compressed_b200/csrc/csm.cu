@@ -13,16 +13,17 @@
 //
 // Design: one CTA per (chunk, pair) -- a chunk is <= 256 rows, so everything after the
 // loads stays in shared memory.  The chunk's key rows land once in a swizzled tile
-// (cp.async), its value rows in a second tile whose copies complete while the matching
-// runs (the centroids read both from shared memory); the |A| x |B| dot products run on mma.sync (bf16 in, fp32 accumulate,
+// (cp.async); the |A| x |B| dot products run on mma.sync (bf16 in, fp32 accumulate,
 // each warp one 16-row A tile against all B rows) and every A row keeps its best
 // dot / |b| with a quad reduction; the top-m selection is a rank count over the
 // chunk's <= 128 candidates; the centroids sum in a fixed order (the B row, then its
-// merged A rows in ascending order) in fp32 and round to bf16 once.  One extra CTA per
+// merged A rows in ascending order) in fp32 and round to bf16 once, each warp loading the
+// value rows of four output rows at a time.  One extra CTA per
 // pair copies the sinks and recent rows.  The rows a chunk keeps and their output
 // places depend only on that chunk, so every CTA writes its own output rows.
 #include <climits>
 #include <cmath>
+#include <type_traits>
 
 #include "vc_common.cuh"
 #include "vc_internal.h"
@@ -50,8 +51,7 @@ template <int D>
 struct CsmSmem {
   static constexpr int kRowB = D * 2;
   static constexpr int kK = 0;                                     // [256][D] bf16
-  static constexpr int kV = kK + kCsmMaxChunk * kRowB;             // [256][D] bf16
-  static constexpr int kInvN = kV + kCsmMaxChunk * kRowB;          // float [256]
+  static constexpr int kInvN = kK + kCsmMaxChunk * kRowB;          // float [256]
   static constexpr int kBestB = kInvN + kCsmMaxChunk * 4;          // int [128]
   static constexpr int kBestS = kBestB + 128 * 4;                  // float [128]
   static constexpr int kMerged = kBestS + 128 * 4;                 // int [128]
@@ -115,9 +115,7 @@ __global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
   int* merged = reinterpret_cast<int*>(smem + SM::kMerged);
   int* scan = reinterpret_cast<int*>(smem + SM::kScan);
 
-  // ---- key rows of the chunk -> shared memory (rows past the chunk zeroed), then the
-  //      value rows in a second group that lands while the matching runs
-  const uint32_t vs = smem_u32(smem + SM::kV);
+  // ---- key rows of the chunk -> shared memory (rows past the chunk zeroed)
   for (int e = tid; e < kCsmMaxChunk * CH; e += kCsmThreads) {
     const int r = e / CH, c = e - r * CH;
     const bool ok = r < len;
@@ -125,12 +123,7 @@ __global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
                ok ? 16u : 0u);
   }
   cp_async_commit();
-  for (int e = tid; e < len * CH; e += kCsmThreads) {
-    const int r = e / CH, c = e - r * CH;
-    cp_async16(csm_row_addr<D>(vs, r, c), vin + (int64_t)(r0 + r) * D + c * 8, 16u);
-  }
-  cp_async_commit();
-  cp_async_wait<1>();
+  cp_async_wait<0>();
   __syncthreads();
 
   // ---- 1 / |k| of every row (0 for an all-zero row: its cosines are 0)
@@ -241,71 +234,93 @@ __global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
     dst[r0 + tid] = base + scan[own] - 1;
   }
 
-  // ---- write the kept rows: unmerged A rows as they are, B rows as centroids
-  cp_async_wait<0>();                             // the value rows
-  __syncthreads();
+  // ---- write the kept rows: unmerged A rows as they are, B rows as centroids.  A warp
+  //      takes its rows four at a time and loads their value rows from global memory
+  //      together, so the four loads' latencies overlap.
   constexpr int DPL = D / 32;                     // channels per lane
-  for (int t = warp; t < len; t += kCsmThreads / 32) {
-    if ((t & 1) == 0 && merged[t >> 1]) continue;  // warp-uniform
-    const int orow = base + scan[t] - 1;
-    const int row = r0 + t;
-    float ak[DPL], av[DPL];
-    int ntot = deg_of(row);
-    const float nb = (float)ntot;
-    auto load_row = [&](int tile, int r, float (&x)[DPL]) {   // channels lane*DPL ..
-      const int d0 = lane * DPL;
-      const uint8_t* src = smem + tile + r * SM::kRowB + (((d0 >> 3) ^ (r & 7)) << 4) +
-                           (d0 & 7) * 2;
-      if constexpr (DPL == 4) {
-        const uint2 w = *reinterpret_cast<const uint2*>(src);
-        x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
-      } else {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(src);
-        x[0] = bf16_lo(w); x[1] = bf16_hi(w);
-      }
-    };
-    auto load_k = [&](int r, float (&x)[DPL]) { load_row(SM::kK, r, x); };
-    auto load_v = [&](int r, float (&x)[DPL]) { load_row(SM::kV, r, x); };
-    load_k(t, ak);
-    load_v(t, av);
-    if (t & 1) {
-      // a B row: add the A rows merged into it, in ascending order
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) { ak[e] *= nb; av[e] *= nb; }
-      const int j = t >> 1;
-      for (int i0 = 0; i0 < nA; i0 += 32) {
-        const int i = i0 + lane;
-        const bool in = i < nA && merged[i] && best_b[i] == j;
-        unsigned bal = __ballot_sync(0xffffffffu, in);
-        while (bal) {
-          const int a = i0 + __ffs(bal) - 1;
-          bal &= bal - 1;
-          const int na = deg_of(r0 + 2 * a);
-          float xk[DPL], xv[DPL];
-          load_k(2 * a, xk);
-          load_v(2 * a, xv);
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) {
-            ak[e] = fmaf((float)na, xk[e], ak[e]);
-            av[e] = fmaf((float)na, xv[e], av[e]);
-          }
-          ntot += na;
-        }
-      }
-      const float inv = (float)ntot;
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) { ak[e] = ak[e] / inv; av[e] = av[e] / inv; }
-    }
-    __nv_bfloat16* ko = kout + (int64_t)orow * D + lane * DPL;
-    __nv_bfloat16* vo = vout + (int64_t)orow * D + lane * DPL;
+  constexpr int kBatch = 4;
+  auto load_k = [&](int r, float (&x)[DPL]) {     // channels lane*DPL .. from shared
+    const int d0 = lane * DPL;
+    const uint8_t* src = smem + SM::kK + r * SM::kRowB + (((d0 >> 3) ^ (r & 7)) << 4) +
+                         (d0 & 7) * 2;
     if constexpr (DPL == 4) {
-      *reinterpret_cast<uint2*>(ko) = make_uint2(pack_bf16x2(ak[0], ak[1]), pack_bf16x2(ak[2], ak[3]));
-      *reinterpret_cast<uint2*>(vo) = make_uint2(pack_bf16x2(av[0], av[1]), pack_bf16x2(av[2], av[3]));
+      const uint2 w = *reinterpret_cast<const uint2*>(src);
+      x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
     } else {
-      *reinterpret_cast<uint32_t*>(ko) = pack_bf16x2(ak[0], ak[1]);
-      *reinterpret_cast<uint32_t*>(vo) = pack_bf16x2(av[0], av[1]);
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(src);
+      x[0] = bf16_lo(w); x[1] = bf16_hi(w);
     }
-    if (lane == 0) dout[orow] = ntot;
+  };
+  using VRaw = typename std::conditional<DPL == 4, uint2, uint32_t>::type;
+  auto raw_v = [&](int r) -> VRaw {               // from global
+    return *reinterpret_cast<const VRaw*>(vin + (int64_t)(r0 + r) * D + lane * DPL);
+  };
+  auto unpack = [&](VRaw w, float (&x)[DPL]) {
+    if constexpr (DPL == 4) {
+      x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+    } else {
+      x[0] = bf16_lo(w); x[1] = bf16_hi(w);
+    }
+  };
+  constexpr int kWarps = kCsmThreads / 32;
+  for (int t0 = warp; t0 < len; t0 += kWarps * kBatch) {
+    VRaw vr[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int t = t0 + b * kWarps;
+      vr[b] = raw_v(t < len ? t : 0);
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int t = t0 + b * kWarps;
+      if (t >= len) break;
+      if ((t & 1) == 0 && merged[t >> 1]) continue;  // warp-uniform
+      const int orow = base + scan[t] - 1;
+      const int row = r0 + t;
+      float ak[DPL], av[DPL];
+      int ntot = deg_of(row);
+      const float nb = (float)ntot;
+      load_k(t, ak);
+      unpack(vr[b], av);
+      if (t & 1) {
+        // a B row: add the A rows merged into it, in ascending order
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) { ak[e] *= nb; av[e] *= nb; }
+        const int j = t >> 1;
+        for (int i0 = 0; i0 < nA; i0 += 32) {
+          const int i = i0 + lane;
+          const bool in = i < nA && merged[i] && best_b[i] == j;
+          unsigned bal = __ballot_sync(0xffffffffu, in);
+          while (bal) {
+            const int a = i0 + __ffs(bal) - 1;
+            bal &= bal - 1;
+            const int na = deg_of(r0 + 2 * a);
+            float xk[DPL], xv[DPL];
+            load_k(2 * a, xk);
+            unpack(raw_v(2 * a), xv);
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) {
+              ak[e] = fmaf((float)na, xk[e], ak[e]);
+              av[e] = fmaf((float)na, xv[e], av[e]);
+            }
+            ntot += na;
+          }
+        }
+        const float inv = (float)ntot;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) { ak[e] = ak[e] / inv; av[e] = av[e] / inv; }
+      }
+      __nv_bfloat16* ko = kout + (int64_t)orow * D + lane * DPL;
+      __nv_bfloat16* vo = vout + (int64_t)orow * D + lane * DPL;
+      if constexpr (DPL == 4) {
+        *reinterpret_cast<uint2*>(ko) = make_uint2(pack_bf16x2(ak[0], ak[1]), pack_bf16x2(ak[2], ak[3]));
+        *reinterpret_cast<uint2*>(vo) = make_uint2(pack_bf16x2(av[0], av[1]), pack_bf16x2(av[2], av[3]));
+      } else {
+        *reinterpret_cast<uint32_t*>(ko) = pack_bf16x2(ak[0], ak[1]);
+        *reinterpret_cast<uint32_t*>(vo) = pack_bf16x2(av[0], av[1]);
+      }
+      if (lane == 0) dout[orow] = ntot;
+    }
   }
 }
 

@@ -50,7 +50,7 @@ __device__ __forceinline__ uint64_t globaltimer() {
 // by another role of the CTA (so one stuck role cannot hang the others).  abort may be
 // null (teardown waits that must not be cut short by the flag).  Ordinary limits use the
 // plain test (the thread wakes as soon as the phase completes) and look at the clock and
-// the flag every 64 tests; a limit under 1 ms (a test of the error path) bounds each
+// the flag every 256 tests; a limit under 1 ms (a test of the error path) bounds each
 // test's suspend time by the limit itself, so the wait really gives up that early.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns = 2000000000ull) {
@@ -68,7 +68,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
-    if ((it & 63u) == 0) {
+    if ((it & 255u) == 0) {
       if (abort != nullptr && *abort) return false;
       if (globaltimer() - t0 > limit_ns) return false;
     }
