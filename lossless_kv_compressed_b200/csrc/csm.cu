@@ -11,15 +11,16 @@
 // degree-weighted mean of K and V with the summed degree and takes its B row's place;
 // the output keeps sinks, then the survivors of each chunk in order, then recent rows.
 //
-// Design: one CTA per (chunk, pair) -- a chunk is <= 256 rows, so everything after the
-// loads stays in shared memory.  The chunk's key rows land once in a swizzled tile
-// (cp.async); the |A| x |B| dot products run on mma.sync (bf16 in, fp32 accumulate,
+// Design: one CTA per (chunk, pair) -- a chunk is <= 256 rows, so its key rows and
+// degrees stay in shared memory (3 CTAs per SM).  The key rows land once in a swizzled
+// tile (cp.async); the |A| x |B| dot products run on mma.sync (bf16 in, fp32 accumulate,
 // each warp one 16-row A tile against all B rows) and every A row keeps its best
 // dot / |b| with a quad reduction; the top-m selection is a rank count over the
-// chunk's <= 128 candidates; the centroids sum in a fixed order (the B row, then its
-// merged A rows in ascending order) in fp32 and round to bf16 once, each warp loading the
-// value rows of four output rows at a time.  One extra CTA per
-// pair copies the sinks and recent rows.  The rows a chunk keeps and their output
+// chunk's <= 128 candidates.  A scan then lays the chunk's rows out as a source list
+// grouped by output row, and the centroids sum in a fixed order (the B row, then its
+// merged A rows in ascending order) in fp32 and round to bf16 once; a warp folds a
+// contiguous span of the list with eight value-row loads from global memory in
+// flight.  One extra CTA per pair copies the sinks and recent rows.  The rows a chunk keeps and their output
 // places depend only on that chunk, so every CTA writes its own output rows.
 #include <climits>
 #include <cmath>
@@ -56,7 +57,10 @@ struct CsmSmem {
   static constexpr int kBestS = kBestB + 128 * 4;                  // float [128]
   static constexpr int kMerged = kBestS + 128 * 4;                 // int [128]
   static constexpr int kScan = kMerged + 128 * 4;                  // int [256]
-  static constexpr int kTotal = kScan + kCsmMaxChunk * 4;
+  static constexpr int kDeg = kScan + kCsmMaxChunk * 4;            // int [256]
+  static constexpr int kSrc = kDeg + kCsmMaxChunk * 4;             // int [256]
+  static constexpr int kNm = kSrc + kCsmMaxChunk * 4;              // int [128]
+  static constexpr int kTotal = kNm + 128 * 4;
 };
 
 template <int D>
@@ -65,7 +69,7 @@ __device__ __forceinline__ uint32_t csm_row_addr(uint32_t base, int r, int c) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
+__global__ void __launch_bounds__(kCsmThreads, 3) csm_kernel(const CsmParams p) {
   pdl_wait();
   pdl_trigger();
   using SM = CsmSmem<D>;
@@ -83,21 +87,39 @@ __global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
   auto deg_of = [&](int row) { return din ? din[row] : 1; };
 
   if ((int)blockIdx.x == p.n_chunks) {
-    // ---- sinks and recent rows: copied unchanged
+    // ---- sinks and recent rows: copied unchanged, eight 16-byte pieces in flight per
+    //      thread (piece e: row e / (2 CH), K for the first CH pieces of a row, then V)
     const int n_copy = p.n_sinks + p.n_recent;
-    for (int e = warp; e < n_copy; e += kCsmThreads / 32) {
-      const int row = e < p.n_sinks ? e : p.T - p.n_recent + (e - p.n_sinks);
-      const int orow = e < p.n_sinks ? e : p.out_len - p.n_recent + (e - p.n_sinks);
-      for (int c = lane; c < CH; c += 32) {
-        reinterpret_cast<uint4*>(kout + (int64_t)orow * D)[c] =
-            reinterpret_cast<const uint4*>(kin + (int64_t)row * D)[c];
-        reinterpret_cast<uint4*>(vout + (int64_t)orow * D)[c] =
-            reinterpret_cast<const uint4*>(vin + (int64_t)row * D)[c];
+    const int total = n_copy * 2 * CH;
+    auto in_row = [&](int e) { return e < p.n_sinks ? e : p.T - p.n_recent + (e - p.n_sinks); };
+    auto out_row = [&](int e) {
+      return e < p.n_sinks ? e : p.out_len - p.n_recent + (e - p.n_sinks);
+    };
+    constexpr int kInFlight = 8;
+    for (int e0 = tid; e0 < total; e0 += kCsmThreads * kInFlight) {
+      uint4 w[kInFlight];
+#pragma unroll
+      for (int u = 0; u < kInFlight; ++u) {
+        const int e = e0 + u * kCsmThreads;
+        if (e < total) {
+          const int r = e / (2 * CH), c = e - r * 2 * CH;
+          const __nv_bfloat16* src = c < CH ? kin : vin;
+          w[u] = reinterpret_cast<const uint4*>(src + (int64_t)in_row(r) * D)[c % CH];
+        }
       }
-      if (lane == 0) {
-        dout[orow] = deg_of(row);
-        if (dst) dst[row] = orow;
+#pragma unroll
+      for (int u = 0; u < kInFlight; ++u) {
+        const int e = e0 + u * kCsmThreads;
+        if (e < total) {
+          const int r = e / (2 * CH), c = e - r * 2 * CH;
+          __nv_bfloat16* dst_t = c < CH ? kout : vout;
+          reinterpret_cast<uint4*>(dst_t + (int64_t)out_row(r) * D)[c % CH] = w[u];
+        }
       }
+    }
+    for (int e = tid; e < n_copy; e += kCsmThreads) {
+      dout[out_row(e)] = deg_of(in_row(e));
+      if (dst) dst[in_row(e)] = out_row(e);
     }
     return;
   }
@@ -123,6 +145,8 @@ __global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
                ok ? 16u : 0u);
   }
   cp_async_commit();
+  int* deg_s = reinterpret_cast<int*>(smem + SM::kDeg);
+  deg_s[tid] = tid < len ? deg_of(r0 + tid) : 0;   // kCsmThreads == kCsmMaxChunk
   cp_async_wait<0>();
   __syncthreads();
 
@@ -203,6 +227,7 @@ __global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
   __syncthreads();
 
   // ---- the m most similar A rows merge (higher cosine first, lower row on ties)
+  int* nm = reinterpret_cast<int*>(smem + SM::kNm);       // A rows merged into B row j
   if (tid < 128) {
     int mg = 0;
     if (tid < nA && m > 0) {
@@ -215,12 +240,22 @@ __global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
       mg = rank < m ? 1 : 0;
     }
     merged[tid] = mg;
+    nm[tid] = 0;
   }
   __syncthreads();
+  if (tid < nA && merged[tid]) atomicAdd(&nm[best_b[tid]], 1);
+  __syncthreads();
 
-  // ---- output places: exclusive prefix count of the kept rows of the chunk
-  const bool keep = tid < len && !((tid & 1) == 0 && merged[tid >> 1]);
-  scan[tid] = keep ? 1 : 0;
+  // ---- output places and the source list.  Every chunk row either is kept (an output
+  //      row of its own) or is an A row merged into a kept B row.  The source list holds
+  //      the chunk's rows grouped by output row, in output order: the kept row first,
+  //      then the A rows merged into it in ascending order (the centroid's summation
+  //      order).  One inclusive scan counts both: kept rows in the high half-word
+  //      (output places), list entries in the low half-word (list places).
+  auto kept = [&](int t) { return !((t & 1) == 0 && merged[t >> 1]); };
+  const bool keep = tid < len && kept(tid);
+  const int cnt = keep ? ((tid & 1) ? 1 + nm[tid >> 1] : 1) : 0;
+  scan[tid] = (keep ? 1 << 16 : 0) | cnt;
   __syncthreads();
   for (int off = 1; off < kCsmMaxChunk; off <<= 1) {
     const int add = tid >= off ? scan[tid - off] : 0;
@@ -228,26 +263,41 @@ __global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
     scan[tid] += add;
     __syncthreads();
   }
-  // scan[t] is now the inclusive count: kept row t goes to base + scan[t] - 1
-  if (dst && tid < len) {
-    const int own = tid & 1 ? tid : (merged[tid >> 1] ? 2 * best_b[tid >> 1] + 1 : tid);
-    dst[r0 + tid] = base + scan[own] - 1;
+  // kept row t goes to output row base + (scan[t] >> 16) - 1; its list entries start at
+  // (scan[t] & 0xffff) minus its own count
+  int* src = reinterpret_cast<int*>(smem + SM::kSrc);
+  if (keep) src[(scan[tid] & 0xffff) - cnt] = tid;
+  if (tid < len && !keep) {
+    const int a = tid >> 1, j = best_b[a];
+    int before = 0;                                   // merged A rows of j below a
+    for (int u = 0; u < a; ++u) before += (merged[u] && best_b[u] == j) ? 1 : 0;
+    const int b_row = 2 * j + 1;
+    src[(scan[b_row] & 0xffff) - 1 - nm[j] + 1 + before] = tid;
   }
+  if (dst && tid < len) {
+    const int own = keep ? tid : 2 * best_b[tid >> 1] + 1;
+    dst[r0 + tid] = base + (scan[own] >> 16) - 1;
+  }
+  __syncthreads();
 
-  // ---- write the kept rows: unmerged A rows as they are, B rows as centroids.  A warp
-  //      takes its rows four at a time and loads their value rows from global memory
-  //      together, so the four loads' latencies overlap.
+  // ---- write the kept rows: unmerged A rows as they are, B rows as centroids (B row
+  //      times its degree, plus each merged A row times its degree in ascending order,
+  //      over the summed degree, in fp32, rounded to bf16 once).  Warp w folds the
+  //      list entries of the output rows that start in [w len / 8, (w + 1) len / 8), so
+  //      every output row is one warp's; the value rows of eight entries are loaded
+  //      from global memory together, so their latencies overlap.
   constexpr int DPL = D / 32;                     // channels per lane
-  constexpr int kBatch = 4;
+  constexpr int kWarps = kCsmThreads / 32;
+  constexpr int kBatch = 8;
   auto load_k = [&](int r, float (&x)[DPL]) {     // channels lane*DPL .. from shared
     const int d0 = lane * DPL;
-    const uint8_t* src = smem + SM::kK + r * SM::kRowB + (((d0 >> 3) ^ (r & 7)) << 4) +
-                         (d0 & 7) * 2;
+    const uint8_t* srcp = smem + SM::kK + r * SM::kRowB + (((d0 >> 3) ^ (r & 7)) << 4) +
+                          (d0 & 7) * 2;
     if constexpr (DPL == 4) {
-      const uint2 w = *reinterpret_cast<const uint2*>(src);
+      const uint2 w = *reinterpret_cast<const uint2*>(srcp);
       x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
     } else {
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(src);
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(srcp);
       x[0] = bf16_lo(w); x[1] = bf16_hi(w);
     }
   };
@@ -262,66 +312,63 @@ __global__ void __launch_bounds__(kCsmThreads) csm_kernel(const CsmParams p) {
       x[0] = bf16_lo(w); x[1] = bf16_hi(w);
     }
   };
-  constexpr int kWarps = kCsmThreads / 32;
-  for (int t0 = warp; t0 < len; t0 += kWarps * kBatch) {
+  auto span_edge = [&](int e) {                   // first output-row start at or after e
+    while (e < len && !kept(src[e])) ++e;
+    return e;
+  };
+  const int lo = span_edge(min(len, (warp * len) / kWarps));
+  const int hi = span_edge(min(len, ((warp + 1) * len) / kWarps));
+
+  float ak[DPL], av[DPL];
+  int cur = -1, ntot = 0;
+  auto flush = [&]() {
+    if (cur & 1) {
+      const float inv = (float)ntot;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) { ak[e] = ak[e] / inv; av[e] = av[e] / inv; }
+    }
+    const int orow = base + (scan[cur] >> 16) - 1;
+    __nv_bfloat16* ko = kout + (int64_t)orow * D + lane * DPL;
+    __nv_bfloat16* vo = vout + (int64_t)orow * D + lane * DPL;
+    if constexpr (DPL == 4) {
+      *reinterpret_cast<uint2*>(ko) = make_uint2(pack_bf16x2(ak[0], ak[1]), pack_bf16x2(ak[2], ak[3]));
+      *reinterpret_cast<uint2*>(vo) = make_uint2(pack_bf16x2(av[0], av[1]), pack_bf16x2(av[2], av[3]));
+    } else {
+      *reinterpret_cast<uint32_t*>(ko) = pack_bf16x2(ak[0], ak[1]);
+      *reinterpret_cast<uint32_t*>(vo) = pack_bf16x2(av[0], av[1]);
+    }
+    if (lane == 0) dout[orow] = ntot;
+  };
+  for (int e0 = lo; e0 < hi; e0 += kBatch) {
     VRaw vr[kBatch];
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-      const int t = t0 + b * kWarps;
-      vr[b] = raw_v(t < len ? t : 0);
-    }
+    for (int b = 0; b < kBatch; ++b) vr[b] = raw_v(e0 + b < hi ? src[e0 + b] : src[lo]);
 #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
-      const int t = t0 + b * kWarps;
-      if (t >= len) break;
-      if ((t & 1) == 0 && merged[t >> 1]) continue;  // warp-uniform
-      const int orow = base + scan[t] - 1;
-      const int row = r0 + t;
-      float ak[DPL], av[DPL];
-      int ntot = deg_of(row);
-      const float nb = (float)ntot;
-      load_k(t, ak);
-      unpack(vr[b], av);
-      if (t & 1) {
-        // a B row: add the A rows merged into it, in ascending order
+      if (e0 + b >= hi) break;
+      const int t = src[e0 + b];                  // warp-uniform
+      const int n = deg_s[t];
+      float xk[DPL], xv[DPL];
+      load_k(t, xk);
+      unpack(vr[b], xv);
+      if (kept(t)) {
+        if (cur >= 0) flush();
+        cur = t;
+        ntot = n;
+        const float nb = (t & 1) ? (float)n : 1.f;   // an A row is copied as it is
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) { ak[e] *= nb; av[e] *= nb; }
-        const int j = t >> 1;
-        for (int i0 = 0; i0 < nA; i0 += 32) {
-          const int i = i0 + lane;
-          const bool in = i < nA && merged[i] && best_b[i] == j;
-          unsigned bal = __ballot_sync(0xffffffffu, in);
-          while (bal) {
-            const int a = i0 + __ffs(bal) - 1;
-            bal &= bal - 1;
-            const int na = deg_of(r0 + 2 * a);
-            float xk[DPL], xv[DPL];
-            load_k(2 * a, xk);
-            unpack(raw_v(2 * a), xv);
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) {
-              ak[e] = fmaf((float)na, xk[e], ak[e]);
-              av[e] = fmaf((float)na, xv[e], av[e]);
-            }
-            ntot += na;
-          }
-        }
-        const float inv = (float)ntot;
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) { ak[e] = ak[e] / inv; av[e] = av[e] / inv; }
-      }
-      __nv_bfloat16* ko = kout + (int64_t)orow * D + lane * DPL;
-      __nv_bfloat16* vo = vout + (int64_t)orow * D + lane * DPL;
-      if constexpr (DPL == 4) {
-        *reinterpret_cast<uint2*>(ko) = make_uint2(pack_bf16x2(ak[0], ak[1]), pack_bf16x2(ak[2], ak[3]));
-        *reinterpret_cast<uint2*>(vo) = make_uint2(pack_bf16x2(av[0], av[1]), pack_bf16x2(av[2], av[3]));
+        for (int e = 0; e < DPL; ++e) { ak[e] = xk[e] * nb; av[e] = xv[e] * nb; }
       } else {
-        *reinterpret_cast<uint32_t*>(ko) = pack_bf16x2(ak[0], ak[1]);
-        *reinterpret_cast<uint32_t*>(vo) = pack_bf16x2(av[0], av[1]);
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) {
+          ak[e] = fmaf((float)n, xk[e], ak[e]);
+          av[e] = fmaf((float)n, xv[e], av[e]);
+        }
+        ntot += n;
       }
-      if (lane == 0) dout[orow] = ntot;
     }
   }
+  if (cur >= 0) flush();
 }
 
 int64_t csm_out_len(int64_t T, int n_sinks, int n_recent, int chunk, double r) {
