@@ -60,7 +60,8 @@ struct CsmSmem {
   static constexpr int kDeg = kScan + kCsmMaxChunk * 4;            // int [256]
   static constexpr int kSrc = kDeg + kCsmMaxChunk * 4;             // int [256]
   static constexpr int kNm = kSrc + kCsmMaxChunk * 4;              // int [128]
-  static constexpr int kTotal = kNm + 128 * 4;
+  static constexpr int kInvB = kNm + 128 * 4;                      // float [128]
+  static constexpr int kTotal = kInvB + 128 * 4;
 };
 
 template <int D>
@@ -168,7 +169,10 @@ __global__ void __launch_bounds__(kCsmThreads, 3) csm_kernel(const CsmParams p) 
         }
       }
     }
-    invn[r] = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+    const float in = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+    invn[r] = in;
+    if (r & 1) reinterpret_cast<float*>(smem + SM::kInvB)[r >> 1] = in;   // B rows, compact
+    if (r < 128 && r >= nA) best_s[r] = -INFINITY;   // candidates past the chunk never rank
   }
   __syncthreads();
 
@@ -199,12 +203,13 @@ __global__ void __launch_bounds__(kCsmThreads, 3) csm_kernel(const CsmParams p) 
                  af[2 * kk + 1][3], b2, b3);
       }
       // accumulator: rows qr, qr + 8; columns (B rows) 8nt + 2qc, +1
+      const float2 ib = reinterpret_cast<const float2*>(smem + SM::kInvB)[4 * nt + qc];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int jj = 8 * nt + 2 * qc + (e & 1);
         const int h = e >> 1;
         if (jj < nB) {
-          const float val = s[e] * invn[2 * jj + 1];
+          const float val = s[e] * ((e & 1) ? ib.y : ib.x);
           if (val > bv[h] || (val == bv[h] && jj < bj[h])) { bv[h] = val; bj[h] = jj; }
         }
       }
@@ -226,24 +231,52 @@ __global__ void __launch_bounds__(kCsmThreads, 3) csm_kernel(const CsmParams p) 
   }
   __syncthreads();
 
-  // ---- the m most similar A rows merge (higher cosine first, lower row on ties)
+  // ---- the m most similar A rows merge (higher cosine first, lower row on ties): the
+  //      rank of candidate i counted by two threads, each over half of the candidates
+  //      (entries past nA hold -inf and never count)
+  int* part = scan;                                       // free until the scan below
+  {
+    const int i = tid & 127, half = tid >> 7;
+    const float st = best_s[i];
+    const float4* bs4 = reinterpret_cast<const float4*>(best_s + 64 * half);
+    int rank = 0;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const float4 v = bs4[q];
+      const int u = 64 * half + 4 * q;
+      rank += (v.x > st || (v.x == st && u < i)) ? 1 : 0;
+      rank += (v.y > st || (v.y == st && u + 1 < i)) ? 1 : 0;
+      rank += (v.z > st || (v.z == st && u + 2 < i)) ? 1 : 0;
+      rank += (v.w > st || (v.w == st && u + 3 < i)) ? 1 : 0;
+    }
+    part[tid] = rank;
+  }
+  __syncthreads();
   int* nm = reinterpret_cast<int*>(smem + SM::kNm);       // A rows merged into B row j
   if (tid < 128) {
-    int mg = 0;
-    if (tid < nA && m > 0) {
-      const float st = best_s[tid];
-      int rank = 0;
-      for (int u = 0; u < nA; ++u) {
-        const float su = best_s[u];
-        rank += (su > st || (su == st && u < tid)) ? 1 : 0;
-      }
-      mg = rank < m ? 1 : 0;
-    }
-    merged[tid] = mg;
+    merged[tid] = (tid < nA && m > 0 && part[tid] + part[tid + 128] < m) ? 1 : 0;
     nm[tid] = 0;
   }
   __syncthreads();
-  if (tid < nA && merged[tid]) atomicAdd(&nm[best_b[tid]], 1);
+  // per merged A row, how many merged A rows below it share its B row (its place among
+  // them), and per B row the count: one warp walks the A rows in ascending order
+  int* before = reinterpret_cast<int*>(best_s);           // best_s is no longer needed
+  if (warp == 0) {
+    for (int c = 0; c < 4; ++c) {
+      const int a = 32 * c + lane;
+      const bool mg = a < nA && merged[a];
+      const int j = mg ? best_b[a] : -1 - lane;           // unmerged lanes: groups of one
+      const unsigned same = __match_any_sync(0xffffffffu, j);
+      const int below = __popc(same & ((1u << lane) - 1u));
+      const int run = mg ? nm[j] : 0;
+      __syncwarp();
+      if (mg) {
+        before[a] = run + below;
+        if ((same >> lane) == 1u) nm[j] = run + below + 1;   // the group's highest lane
+      }
+      __syncwarp();
+    }
+  }
   __syncthreads();
 
   // ---- output places and the source list.  Every chunk row either is kept (an output
@@ -269,10 +302,7 @@ __global__ void __launch_bounds__(kCsmThreads, 3) csm_kernel(const CsmParams p) 
   if (keep) src[(scan[tid] & 0xffff) - cnt] = tid;
   if (tid < len && !keep) {
     const int a = tid >> 1, j = best_b[a];
-    int before = 0;                                   // merged A rows of j below a
-    for (int u = 0; u < a; ++u) before += (merged[u] && best_b[u] == j) ? 1 : 0;
-    const int b_row = 2 * j + 1;
-    src[(scan[b_row] & 0xffff) - 1 - nm[j] + 1 + before] = tid;
+    src[(scan[2 * j + 1] & 0xffff) - nm[j] + before[a]] = tid;   // after its B row
   }
   if (dst && tid < len) {
     const int own = keep ? tid : 2 * best_b[tid >> 1] + 1;
@@ -321,8 +351,9 @@ __global__ void __launch_bounds__(kCsmThreads, 3) csm_kernel(const CsmParams p) 
 
   float ak[DPL], av[DPL];
   int cur = -1, ntot = 0;
+  bool centroid = false;                          // a B row with merged A rows
   auto flush = [&]() {
-    if (cur & 1) {
+    if (centroid) {
       const float inv = (float)ntot;
 #pragma unroll
       for (int e = 0; e < DPL; ++e) { ak[e] = ak[e] / inv; av[e] = av[e] / inv; }
@@ -355,7 +386,9 @@ __global__ void __launch_bounds__(kCsmThreads, 3) csm_kernel(const CsmParams p) 
         if (cur >= 0) flush();
         cur = t;
         ntot = n;
-        const float nb = (t & 1) ? (float)n : 1.f;   // an A row is copied as it is
+        // a row nothing merges into is copied as it is (n x / n is x exactly)
+        centroid = (t & 1) && nm[t >> 1] > 0;
+        const float nb = centroid ? (float)n : 1.f;
 #pragma unroll
         for (int e = 0; e < DPL; ++e) { ak[e] = xk[e] * nb; av[e] = xv[e] * nb; }
       } else {

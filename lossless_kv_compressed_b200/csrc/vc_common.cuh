@@ -34,23 +34,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Base-2 exponential on the FMA pipe, for softmax probabilities that are rounded to bf16
-// afterwards (relative error <= 7.5e-5 over the normal range; inputs below -126 give
-// 2^-126 p(f), not 0).  Cody and Waite's reduction: x = j + f with j = rint(x) (the
-// 1.5 * 2^23 rounding constant) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
-// coefficients are this library's own Remez fit of 2^f on [-1/2, 1/2] for minimal
-// relative error; 2^j added to the exponent field.  Moves work off the MUFU pipe when
-// that pipe, not the issue slots, bounds a softmax.
-__device__ __forceinline__ float exp2_poly3(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;                 // 1.5 * 2^23: rint(x) in the low bits
-  const float f = x - (t - 12582912.f);
-  float p = fmaf(0.0551716685f, f, 0.2426111251f);
-  p = fmaf(p, f, 0.6932609677f);
-  p = fmaf(p, f, 0.9999280572f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // ------------------------------------------------------------------ shared memory
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
