@@ -371,7 +371,7 @@ __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexe
 // subtracted) and the scales move to the other operand, so nothing proportional to a
 // dequantised value is ever rounded to fp16:
 //   q . k_hat = sum_d (q_d s_d) n_d + sum_d q_d z_d              (K: per channel)
-//   sum_t p_t v_hat_t = sum_t (p_t s_t / 2)(2 n_t - 15) + sum_t p_t (z_t + 7.5 s_t)
+//   sum_t p_t v_hat_t = sum_t (p_t s_t)(n_t - 8) + sum_t p_t (z_t + 8 s_t)
 //                                                                 (V: per token, group;
 //   centred so that neither sum is much larger than the result)
 // q_d s_d and p_t s_t are split into fp16 high and low parts placed in A rows 0-7 and
@@ -404,22 +404,30 @@ struct Int4Smem {
   static constexpr int kStageB = kKW + kVW + 4 * kSZ;
 };
 
-// Nibble pair j of word w as exact fp16x2 integers (n0, n1).
+// Nibble pair j of word w as exact fp16x2 integers (n0, n1): nibble j of the low and of
+// the high half-word, put into the mantissa of fp16 1024, then 1024 subtracted.
 __device__ __forceinline__ uint32_t nib_pair(uint32_t w, int j) {
   const uint32_t x = ((w >> (4 * j)) & 0x000F000Fu) | 0x64006400u;   // 1024 + n
   uint32_t n;
   asm("sub.f16x2 %0, %1, %2;" : "=r"(n) : "r"(x), "r"(0x64006400u));
   return n;
 }
-// Same, centred on the middle of the 4-bit range and doubled: (2 n0 - 15, 2 n1 - 15),
-// exact.  2n + 1 goes into the mantissa of fp16 1024 (the nibble shifted up one bit,
-// the low bit set) and 1040 is subtracted, so one subtraction does both steps.
-__device__ __forceinline__ uint32_t nib_pair_c2(uint32_t w, int j) {
-  const uint32_t sh = j == 0 ? (w << 1) : (w >> (4 * j - 1));
-  const uint32_t x = (sh & 0x001E001Eu) | 0x64016401u;     // 1024 + 2n + 1
-  uint32_t c;
-  asm("sub.f16x2 %0, %1, %2;" : "=r"(c) : "r"(x), "r"(0x64106410u));   // - 1040
-  return c;
+// Same pairs centred on the 4-bit range, (n0 - 8, n1 - 8), exact; w8 = w >> 8 is shared
+// by the four pairs of a word.  A low nibble of a byte goes into the mantissa of fp16
+// 1024 and 1032 is subtracted; a high nibble is masked in place (1024 + 16 n) and one
+// fused multiply-add takes x / 16 - 72: two instructions per pair.
+__device__ __forceinline__ uint32_t nib_pair_c(uint32_t w, uint32_t w8, int j) {
+  const uint32_t src = j < 2 ? w : w8;
+  uint32_t n;
+  if ((j & 1) == 0) {
+    const uint32_t x = (src & 0x000F000Fu) | 0x64006400u;           // 1024 + n
+    asm("sub.f16x2 %0, %1, %2;" : "=r"(n) : "r"(x), "r"(0x64086408u));   // - 1032
+  } else {
+    const uint32_t x = (src & 0x00F000F0u) | 0x64006400u;           // 1024 + 16 n
+    asm("fma.rn.f16x2 %0, %1, %2, %3;"                              // x / 16 - 72
+        : "=r"(n) : "r"(x), "r"(0x2C002C00u), "r"(0xD480D480u));
+  }
+  return n;
 }
 __device__ __forceinline__ float2 h2f(uint32_t h) {
   return __half22float2(*reinterpret_cast<const __half2*>(&h));
@@ -637,12 +645,12 @@ __global__ void __launch_bounds__(128, 3) draft_int4_kernel(const DraftInt4Param
       uint32_t ph[4], pl[4];
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt) split_f16(s[nt][0], s[nt][1], ph[nt], pl[nt]);
-      // B = z + 7.5 s, the value of the middle of each group's grid (the nibbles of V
+      // B = z + 8 s, the value of the middle of each group's grid (the nibbles of V
       // enter centred, so both sums stay of the size of the result: no cancellation)
       auto zmid = [&](int t0) -> uint32_t {
         const int o = (qr * 32 + t0) / 2;
         const float2 z = h2f(vzr[o]), sc = h2f(vsc[o]);
-        return pack_f16x2(fmaf(7.5f, sc.x, z.x), fmaf(7.5f, sc.y, z.y));
+        return pack_f16x2(fmaf(8.f, sc.x, z.x), fmaf(8.f, sc.y, z.y));
       };
 #pragma unroll
       for (int kt = 0; kt < 2; ++kt) {
@@ -654,23 +662,22 @@ __global__ void __launch_bounds__(128, 3) draft_int4_kernel(const DraftInt4Param
         mma_f16(zacc, ph[2 * kt], pl[2 * kt], ph[2 * kt + 1], pl[2 * kt + 1], z0, z1);
       }
     }
-    // ---- O += (p s / 2) (2N - 15) per channel group, B = exact doubled centred nibbles
-    float sh[4][2];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) { sh[j][0] = 0.5f * s[j][0]; sh[j][1] = 0.5f * s[j][1]; }
+    // ---- O += (p s) (N - 8) per channel group, B = exact centred nibbles
 #pragma unroll
     for (int G = 0; G < NW; ++G) {
       uint32_t pah[4], pal[4];                      // [kt * 2 + half]
 #pragma unroll
       for (int j = 0; j < 4; ++j) {                 // token pair 2qc + 8j: n-tile j
         const float2 sv = h2f(vsc[(G * 32 + 2 * qc + 8 * j) / 2]);
-        split_f16(sh[j][0] * sv.x, sh[j][1] * sv.y, pah[j], pal[j]);
+        split_f16(s[j][0] * sv.x, s[j][1] * sv.y, pah[j], pal[j]);
       }
 #pragma unroll
       for (int nn = 4 * G; nn < 4 * G + 4; ++nn) {
-        const uint32_t wv = vw[(nn * 8 + qr) * 4 + qc];
-        mma_f16(o[nn], pah[0], pal[0], pah[1], pal[1], nib_pair_c2(wv, 0), nib_pair_c2(wv, 1));
-        mma_f16(o[nn], pah[2], pal[2], pah[3], pal[3], nib_pair_c2(wv, 2), nib_pair_c2(wv, 3));
+        const uint32_t wv = vw[(nn * 8 + qr) * 4 + qc], wv8 = wv >> 8;
+        mma_f16(o[nn], pah[0], pal[0], pah[1], pal[1], nib_pair_c(wv, wv8, 0),
+                nib_pair_c(wv, wv8, 1));
+        mma_f16(o[nn], pah[2], pal[2], pah[3], pal[3], nib_pair_c(wv, wv8, 2),
+                nib_pair_c(wv, wv8, 3));
       }
     }
     __syncwarp();
