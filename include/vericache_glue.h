@@ -76,9 +76,13 @@ vc_status vc_glue_append_slots(int32_t* idx, int32_t* deg, int Hkv, int S_cap, i
  * [>= cap] with positions[i] = i.  Work buffers for rows_cap rows: x fp32 [rows, d], h
  * bf16 [rows, d], qkv fp32 [rows, (Hq + 2 Hkv) D], q, att bf16 [rows, Hq, D], gu fp32
  * [rows, 2 ffn], act bf16 [rows, ffn], logits fp32 [rows, vocab].  ws: device workspace
- * for the attention calls of one pass (large enough for vc_draft_workspace_size of every
- * draft cache and vc_verify_workspace_size(1, min(rows_cap, 1024 / g), Hq, Hkv, D, 0,
- * cap)).
+ * for the attention calls of one pass, at least vc_glue_workspace_size(m) bytes and
+ * vc_draft_workspace_size of every draft cache.
+ *
+ * Verify attention of blocks of at most tail_cap tokens (a greedy step, a block of k + 1)
+ * splits the keys into windows chosen from Hkv and cap only (the largest power of two
+ * <= 4096, >= 256, giving two CTAs per SM), so a block and the same tokens stepped one at
+ * a time agree bit for bit; longer blocks (the prefill) use 4096-key windows.
  * -------------------------------------------------------------------------------- */
 typedef struct vc_tinylm {
   int32_t n_layers, d_model, Hq, Hkv, D, ffn, vocab;
@@ -108,6 +112,10 @@ typedef struct vc_tinylm {
   void* ws;
   size_t ws_bytes;
 } vc_tinylm;
+
+/* Device workspace the verify calls of vc_glue_forward_full / vc_glue_greedy_steps need
+ * for this model (its Hq, Hkv, D, cap, rows_cap and tail_cap); 0 if those are invalid. */
+size_t vc_glue_workspace_size(const vc_tinylm* m);
 
 /* Tokens ids[0 .. n-1] (device int32) at positions pos0 .. pos0+n-1 through the whole
  * model over the full cache (their K/V stored at their positions, rows attending

@@ -29,7 +29,7 @@ EXPORTS = (
 GLUE_EXPORTS = (
     "vc_glue_embed", "vc_glue_rmsnorm", "vc_glue_gemm", "vc_glue_rope_store",
     "vc_glue_swiglu", "vc_glue_append_slots", "vc_glue_forward_full", "vc_glue_draft_steps",
-    "vc_glue_greedy_steps",
+    "vc_glue_greedy_steps", "vc_glue_workspace_size",
 )
 
 _p = ctypes.c_void_p
@@ -147,6 +147,8 @@ def lib() -> ctypes.CDLL:
                                            ctypes.c_int, _p]
         L.vc_glue_draft_steps.argtypes = [ctypes.POINTER(TinyLM), ctypes.POINTER(CompCache), _p,
                                           ctypes.c_int, ctypes.c_int, _p]
+        L.vc_glue_workspace_size.restype = _sz
+        L.vc_glue_workspace_size.argtypes = [ctypes.POINTER(TinyLM)]
         L.vc_glue_greedy_steps.argtypes = [ctypes.POINTER(TinyLM), _p, ctypes.c_int,
                                            ctypes.c_int, _p]
         _lib = L

@@ -134,6 +134,18 @@ vc_status vc_verify_attn(const void* q, int B, int n_q, int Hq, int Hkv, int D, 
                          const void* v, int64_t L_cap, int64_t kv_start, int64_t kv_len,
                          int64_t P, float* m, float* l, float* acc, int flags, float scale,
                          void* out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  return verify_checked(q, B, n_q, Hq, Hkv, D, k, v, L_cap, kv_start, kv_len, P, m, l, acc,
+                        flags, scale, out, ws, ws_bytes, stream, kVerifySplitKeys);
+}
+
+}  // extern "C"
+
+namespace vc {
+vc_status verify_checked(const void* q, int B, int n_q, int Hq, int Hkv, int D, const void* k,
+                         const void* v, int64_t L_cap, int64_t kv_start, int64_t kv_len,
+                         int64_t P, float* m, float* l, float* acc, int flags, float scale,
+                         void* out, void* ws, size_t ws_bytes, cudaStream_t stream,
+                         int split_keys) {
   if (B <= 0 || n_q <= 0 || Hq <= 0 || Hkv <= 0) return fail(VC_ERR_INVALID, "verify: sizes");
   if (Hq % Hkv) return fail(VC_ERR_INVALID, "verify: Hq %% Hkv != 0");
   if (D != 64 && D != 128) return fail(VC_ERR_UNSUPPORTED, "verify: D must be 64 or 128");
@@ -164,8 +176,12 @@ vc_status vc_verify_attn(const void* q, int B, int n_q, int Hq, int Hkv, int D, 
   if (out && !aligned16(out)) return fail(VC_ERR_INVALID, "verify: out misaligned");
   if (scale <= 0.f) scale = 1.0f / sqrtf((float)D);
   return launch_verify(q, B, n_q, Hq, Hkv, D, k, v, L_cap, kv_start, kv_len, P, m, l, acc,
-                       flags, scale, out, ws, ws_bytes, stream);
+                       flags, scale, out, ws, ws_bytes, stream, split_keys);
 }
+}  // namespace vc
+
+extern "C" {
+
 
 vc_status vc_accept(const float* logits, const int32_t* drafts, int B, int n_q, int V,
                     int32_t* target, int32_t* accept_len, int32_t* commit, int32_t* n_commit,

@@ -35,53 +35,73 @@ __global__ void rmsnorm_kernel(const float* __restrict__ x, int n, int d, float 
   for (int j = lane; j < d; j += 32) out[(int64_t)row * d + j] = __float2bfloat16_rn(xr[j] * inv);
 }
 
-// c[16 x 64 tile] (+)= a[16 x K] @ w[K x 64]: 4 warps x (16 rows x 16 cols), k-steps of 16
-// in order; the w tile rows stream through a 3-stage cp.async ring (128-byte rows,
-// XOR-swizzled) and enter the mma as transposed ldmatrix fragments.
-constexpr int kGemmNst = 3;
+// c[16 x 64 tile] (+)= a[16 x K] @ w[K x 64]: 4 warps x (16 rows x 16 cols), k-steps of
+// 16 in order.  A stage holds 64 k-rows of w (128-byte rows) and the same 64 k-columns of
+// the 16 a rows, both XOR-swizzled, copied by cp.async into a 4-stage ring, so three
+// stages (30 KB) are in flight while one is multiplied; a and w fragments come from
+// shared memory by ldmatrix (w transposed).  Rows past M read as zero.  The k-steps and
+// their order are the same whatever M, so a row's result does not depend on M.
+constexpr int kGemmNst = 4;
+constexpr int kGemmKs = 64;                  // k-rows per stage
 __global__ void __launch_bounds__(128) gemm_kernel(const __nv_bfloat16* __restrict__ a,
                                                    const __nv_bfloat16* __restrict__ w, int M,
                                                    int K, int N, float* __restrict__ c,
                                                    int accumulate) {
-  __shared__ __align__(128) uint8_t sw[kGemmNst][16 * 128];
+  __shared__ __align__(128) uint8_t sw[kGemmNst][kGemmKs * 128];
+  __shared__ __align__(128) uint8_t sa[kGemmNst][16 * 128];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qr = lane >> 2, qc = lane & 3;
   const int n0 = blockIdx.x * 64, m0 = blockIdx.y * 16;
   const int ksteps = K / 16;
-  auto issue = [&](int ks, int st) {
-    const int row = threadIdx.x >> 3, ch = threadIdx.x & 7;
-    const __nv_bfloat16* src = w + (int64_t)(ks * 16 + row) * N + n0 + ch * 8;
-    cp_async16(smem_u32(&sw[st][row * 128 + ((ch ^ (row & 7)) << 4)]), src, 16u);
+  const int nstage = (K + kGemmKs - 1) / kGemmKs;
+  auto issue = [&](int sg, int st) {
+    const int kb = sg * kGemmKs;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {                     // w: 64 rows x 8 chunks
+      const int e = threadIdx.x + 128 * i;
+      const int row = e >> 3, ch = e & 7;
+      const bool ok = kb + row < K;
+      const __nv_bfloat16* src = w + (int64_t)(ok ? kb + row : 0) * N + n0 + ch * 8;
+      cp_async16(smem_u32(&sw[st][row * 128 + ((ch ^ (row & 7)) << 4)]), src, ok ? 16u : 0u);
+    }
+    {                                                 // a: 16 rows x 8 chunks
+      const int row = threadIdx.x >> 3, ch = threadIdx.x & 7;
+      const bool ok = m0 + row < M && kb + ch * 8 < K;
+      const __nv_bfloat16* src = a + (int64_t)(ok ? m0 + row : 0) * K + (ok ? kb + ch * 8 : 0);
+      cp_async16(smem_u32(&sa[st][row * 128 + ((ch ^ (row & 7)) << 4)]), src, ok ? 16u : 0u);
+    }
   };
-  const bool r0 = m0 + qr < M, r1 = m0 + qr + 8 < M;
-  const uint32_t* a0p = reinterpret_cast<const uint32_t*>(a + (int64_t)(r0 ? m0 + qr : 0) * K);
-  const uint32_t* a1p = reinterpret_cast<const uint32_t*>(a + (int64_t)(r1 ? m0 + qr + 8 : 0) * K);
   float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
   for (int st = 0; st < kGemmNst - 1; ++st) {
-    if (st < ksteps) issue(st, st);
+    if (st < nstage) issue(st, st);
     cp_async_commit();
   }
-  for (int ks = 0; ks < ksteps; ++ks) {
-    if (ks + kGemmNst - 1 < ksteps) issue(ks + kGemmNst - 1, (ks + kGemmNst - 1) % kGemmNst);
+  const int mi = lane >> 3;
+  const int arow = (lane & 7) + 8 * (mi & 1), achk = mi >> 1;   // a: rows 0-15, k chunk 0/1
+  const int krow = (mi & 1) * 8 + (lane & 7);                 // w: k rows of the step
+  const int wch = warp * 2 + (mi >> 1);                       // w: 8-column chunk
+  for (int sg = 0; sg < nstage; ++sg) {
+    if (sg + kGemmNst - 1 < nstage) issue(sg + kGemmNst - 1, (sg + kGemmNst - 1) % kGemmNst);
     cp_async_commit();
     cp_async_wait<kGemmNst - 1>();
     __syncthreads();
-    const int k0 = ks * 16;
-    const uint32_t A0 = r0 ? __ldg(a0p + (k0 + 2 * qc) / 2) : 0u;
-    const uint32_t A1 = r1 ? __ldg(a1p + (k0 + 2 * qc) / 2) : 0u;
-    const uint32_t A2 = r0 ? __ldg(a0p + (k0 + 8 + 2 * qc) / 2) : 0u;
-    const uint32_t A3 = r1 ? __ldg(a1p + (k0 + 8 + 2 * qc) / 2) : 0u;
-    const int mi = lane >> 3;
-    const int krow = (mi & 1) * 8 + (lane & 7);
-    const int ch = warp * 2 + (mi >> 1);
-    uint32_t b0, b1, b2, b3;
-    ldsm_x4_t(smem_u32(&sw[ks % kGemmNst][krow * 128 + ((ch ^ (krow & 7)) << 4)]), b0, b1, b2, b3);
-    mma_bf16(acc[0], A0, A1, A2, A3, b0, b1);
-    mma_bf16(acc[1], A0, A1, A2, A3, b2, b3);
+    const int st = sg % kGemmNst;
+#pragma unroll
+    for (int kk = 0; kk < kGemmKs / 16; ++kk) {
+      if (sg * (kGemmKs / 16) + kk >= ksteps) break;
+      uint32_t A0, A1, A2, A3, b0, b1, b2, b3;
+      const int ac = 2 * kk + achk;
+      ldsm_x4(smem_u32(&sa[st][arow * 128 + ((ac ^ (arow & 7)) << 4)]), A0, A1, A2, A3);
+      const int wr = kk * 16 + krow;
+      ldsm_x4_t(smem_u32(&sw[st][wr * 128 + ((wch ^ (wr & 7)) << 4)]), b0, b1, b2, b3);
+      mma_bf16(acc[0], A0, A1, A2, A3, b0, b1);
+      mma_bf16(acc[1], A0, A1, A2, A3, b2, b3);
+    }
     __syncthreads();
   }
   cp_async_wait<0>();
+  const bool r0 = m0 + qr < M, r1 = m0 + qr + 8 < M;
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
     const int col = n0 + warp * 16 + nt * 8 + 2 * qc;
@@ -264,8 +284,21 @@ vc_status logits_of(const vc_tinylm* m, int n, cudaStream_t s) {
   return vc_glue_gemm(m->h, m->lm_head, n, m->d_model, m->vocab, m->logits, 0, s);
 }
 
+// Key window of the verify calls of decode-sized blocks (at most tail_cap tokens: a
+// single greedy step or a block of k + 1): the largest power of two <= 4096, and >= 256,
+// that still gives two CTAs per SM over the model's kv heads and cache capacity.  It
+// depends on the model only, so a k + 1 block and k + 1 single steps use the same window
+// and agree bit for bit.  Longer blocks (the prefill) use the library's default window.
+int decode_split_keys(const vc_tinylm* m) {
+  const int64_t want = 2 * (int64_t)num_sms();
+  int w = kVerifySplitKeys;
+  while (w > 256 && (int64_t)m->Hkv * ((m->cap + w - 1) / w) < want) w >>= 1;
+  return w;
+}
+
 vc_status forward_full(const vc_tinylm* m, const int32_t* ids, int n, int pos0, cudaStream_t s) {
   vc_status st;
+  const int split = n <= m->tail_cap ? decode_split_keys(m) : kVerifySplitKeys;
   if ((st = vc_glue_embed(m->embed, ids, n, m->d_model, m->x, s))) return st;
   const int g = m->Hq / m->Hkv;
   const int chunk = 1024 / g;
@@ -277,10 +310,10 @@ vc_status forward_full(const vc_tinylm* m, const int32_t* ids, int n, int pos0, 
       const int r1 = n < r0 + chunk ? n : r0 + chunk;
       const int nq = r1 - r0;
       const int64_t P = pos0 + r0;
-      st = vc_verify_attn(static_cast<const char*>(m->q) + r0 * qrow, 1, nq, m->Hq, m->Hkv,
+      st = verify_checked(static_cast<const char*>(m->q) + r0 * qrow, 1, nq, m->Hq, m->Hkv,
                           m->D, m->k_full[l], m->v_full[l], m->cap, 0, P + nq, P, nullptr,
                           nullptr, nullptr, 0, 0.f, static_cast<char*>(m->att) + r0 * qrow,
-                          m->ws, m->ws_bytes, s);
+                          m->ws, m->ws_bytes, s, split);
       if (st) return st;
     }
     if ((st = layer_tail(m, l, n, s))) return st;
@@ -289,6 +322,20 @@ vc_status forward_full(const vc_tinylm* m, const int32_t* ids, int n, int pos0, 
 }
 
 }  // namespace
+
+size_t vc_glue_workspace_size(const vc_tinylm* m) {
+  if (!m || m->Hkv <= 0 || m->Hq <= 0 || m->Hq % m->Hkv || m->cap <= 0 || m->rows_cap <= 0)
+    return 0;
+  const int g = m->Hq / m->Hkv;
+  const int rows = m->rows_cap < 1024 / g ? m->rows_cap : 1024 / g;
+  size_t need = verify_workspace_bytes(1, rows, m->Hq, m->Hkv, m->D, 0, m->cap);
+  if (m->tail_cap > 0) {
+    const size_t dec = verify_workspace_bytes(1, m->tail_cap, m->Hq, m->Hkv, m->D, 0, m->cap,
+                                              decode_split_keys(m));
+    if (dec > need) need = dec;
+  }
+  return need;
+}
 
 vc_status vc_glue_forward_full(const vc_tinylm* m, const int32_t* ids, int n, int pos0,
                                cudaStream_t stream) {

@@ -29,12 +29,23 @@ vc_status launch_draft_int4(const void* q, const vc_comp_cache* c, float scale, 
                             void* out, float* lse, void* ws, size_t ws_bytes,
                             cudaStream_t stream);
 
+// Verify attention splits the keys into absolute windows of split_keys positions (a
+// multiple of 64); calls whose rows must agree bit for bit use the same window.  The
+// public entry point uses kVerifySplitKeys.
+constexpr int kVerifySplitKeys = 4096;
 size_t verify_workspace_bytes(int B, int n_q, int Hq, int Hkv, int D, int64_t kv_start,
-                              int64_t kv_len);
+                              int64_t kv_len, int split_keys = kVerifySplitKeys);
 vc_status launch_verify(const void* q, int B, int n_q, int Hq, int Hkv, int D, const void* k,
                         const void* v, int64_t L_cap, int64_t kv_start, int64_t kv_len,
                         int64_t P, float* m, float* l, float* acc, int flags, float scale,
-                        void* out, void* ws, size_t ws_bytes, cudaStream_t stream);
+                        void* out, void* ws, size_t ws_bytes, cudaStream_t stream,
+                        int split_keys = kVerifySplitKeys);
+// vc_verify_attn's argument checks and launch with a chosen window.
+vc_status verify_checked(const void* q, int B, int n_q, int Hq, int Hkv, int D, const void* k,
+                         const void* v, int64_t L_cap, int64_t kv_start, int64_t kv_len,
+                         int64_t P, float* m, float* l, float* acc, int flags, float scale,
+                         void* out, void* ws, size_t ws_bytes, cudaStream_t stream,
+                         int split_keys);
 
 vc_status read_device_error(int32_t* value, int clear);
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;   // 2 s

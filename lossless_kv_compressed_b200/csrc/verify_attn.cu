@@ -46,7 +46,6 @@ namespace vc {
 
 __device__ int g_vc_dev_error;   // bit 0: a bounded wait in the verify kernel expired
 
-constexpr int kSplitKeys = 4096;
 constexpr int kBN = 64;
 constexpr int kVThreads = 384;
 constexpr int kNSt = 6;
@@ -57,6 +56,7 @@ struct VerifyParams {
   int n_q, Hq, Hkv, g, R;   // R = n_q * g rows per pair
   int64_t kv_start, kv_len, P;
   int split0, n_split;
+  int split_keys;           // window of one split (absolute positions, multiple of kBN)
   float qk_scale2;          // scale * log2(e)
   float* ws_o;              // [pairs, n_split, R, D]
   float* ws_ml;             // [pairs, n_split, R, 2]
@@ -105,9 +105,9 @@ __global__ void __launch_bounds__(kVThreads, 1)
   const int64_t part = (int64_t)pair * p.n_split + s_local;
 
   // key range of this split seen by this row group
-  const int64_t win = (int64_t)(p.split0 + s_local) * kSplitKeys;
+  const int64_t win = (int64_t)(p.split0 + s_local) * p.split_keys;
   const int64_t a0 = max(p.kv_start, win);
-  int64_t a1 = min(p.kv_start + p.kv_len, win + kSplitKeys);
+  int64_t a1 = min(p.kv_start + p.kv_len, win + p.split_keys);
   a1 = min(a1, p.P + (row0 + rows_here - 1) / p.g + 1);
   const int n_tiles = a1 > a0 ? (int)((a1 - 1) / kBN - a0 / kBN + 1) : 0;
   const int64_t tile0 = a0 / kBN;
@@ -558,13 +558,14 @@ struct Plan {
   size_t ws_bytes;
 };
 
-Plan plan(int B, int n_q, int Hq, int Hkv, int D, int64_t kv_start, int64_t kv_len) {
+Plan plan(int B, int n_q, int Hq, int Hkv, int D, int64_t kv_start, int64_t kv_len,
+          int split_keys) {
   Plan pl;
   pl.pairs = B * Hkv;
   pl.g = Hq / Hkv;
   pl.R = n_q * pl.g;
-  pl.split0 = (int)(kv_start / kSplitKeys);
-  pl.n_split = (int)((kv_start + kv_len - 1) / kSplitKeys) - pl.split0 + 1;
+  pl.split0 = (int)(kv_start / split_keys);
+  pl.n_split = (int)((kv_start + kv_len - 1) / split_keys) - pl.split0 + 1;
   pl.n_rg = (pl.R + 255) / 256;
   pl.ws_bytes = (size_t)pl.pairs * pl.n_split * pl.R * ((size_t)D + 2) * sizeof(float);
   return pl;
@@ -573,8 +574,8 @@ Plan plan(int B, int n_q, int Hq, int Hkv, int D, int64_t kv_start, int64_t kv_l
 }  // namespace
 
 size_t verify_workspace_bytes(int B, int n_q, int Hq, int Hkv, int D, int64_t kv_start,
-                              int64_t kv_len) {
-  return plan(B, n_q, Hq, Hkv, D, kv_start, kv_len).ws_bytes + 256;
+                              int64_t kv_len, int split_keys) {
+  return plan(B, n_q, Hq, Hkv, D, kv_start, kv_len, split_keys).ws_bytes + 256;
 }
 
 template <int D>
@@ -611,8 +612,10 @@ uint64_t set_verify_wait_ns(uint64_t ns) { return g_verify_wait_ns.exchange(ns);
 vc_status launch_verify(const void* q, int B, int n_q, int Hq, int Hkv, int D, const void* k,
                         const void* v, int64_t L_cap, int64_t kv_start, int64_t kv_len,
                         int64_t P, float* m, float* l, float* acc, int flags, float scale,
-                        void* out, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  const Plan pl = plan(B, n_q, Hq, Hkv, D, kv_start, kv_len);
+                        void* out, void* ws, size_t ws_bytes, cudaStream_t stream,
+                        int split_keys) {
+  if (split_keys < kBN || split_keys % kBN) return fail(VC_ERR_INVALID, "verify: split window");
+  const Plan pl = plan(B, n_q, Hq, Hkv, D, kv_start, kv_len, split_keys);
   if (ws_bytes < pl.ws_bytes) return fail(VC_ERR_INVALID, "verify workspace too small");
   if (P + n_q > (int64_t)1 << 31) return fail(VC_ERR_UNSUPPORTED, "verify: positions >= 2^31");
   CUtensorMap mk, mv;
@@ -631,6 +634,7 @@ vc_status launch_verify(const void* q, int B, int n_q, int Hq, int Hkv, int D, c
   vp.P = P;
   vp.split0 = pl.split0;
   vp.n_split = pl.n_split;
+  vp.split_keys = split_keys;
   vp.qk_scale2 = scale * kLog2e;
   vp.ws_o = static_cast<float*>(ws);
   vp.ws_ml = vp.ws_o + (size_t)pl.pairs * pl.n_split * pl.R * D;

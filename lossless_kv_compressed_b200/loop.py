@@ -31,7 +31,7 @@ import torch
 
 from . import _lib
 from .api import (IndexedCache, accept, csm_compress, draft_attn, draft_workspace_size,
-                  evict_scores, evict_select, verify_attn, verify_workspace_size)
+                  evict_scores, evict_select, verify_attn)
 from ._lib import check, lib
 
 
@@ -193,14 +193,6 @@ class GpuTinyLM:
         c = self.cfg
         P = ctypes.c_void_p
         arr = lambda ts: (P * len(ts))(*[t.data_ptr() for t in ts])
-        g = c.Hq // c.Hkv
-        need = verify_workspace_size(1, min(self.rows, 1024 // g), c.Hq, c.Hkv, c.D, 0,
-                                     self.max_len)
-        probe = IndexedCache(k=self.K[0], v=self.V[0], S=self.s_cap, Hq=c.Hq,
-                             idx=self.idx[0], k_tail=self.KT[0], v_tail=self.VT[0],
-                             n_tail=self.k + 1)
-        need = max(need, draft_workspace_size(probe))
-        self._nat_ws = torch.empty(need, dtype=torch.uint8, device=self.dev)
         self._nat_arrays = [arr(self.wqkv), arr(self.wo), arr(self.wgu), arr(self.wdown),
                             arr(self.K), arr(self.V), arr(self.KT), arr(self.VT)]
         a = self._nat_arrays
@@ -217,6 +209,11 @@ class GpuTinyLM:
         m.att, m.gu, m.act, m.logits = (self.att.data_ptr(), self.gu.data_ptr(),
                                         self.act.data_ptr(), self.logits.data_ptr())
         m.rows_cap = self.rows
+        probe = IndexedCache(k=self.K[0], v=self.V[0], S=self.s_cap, Hq=c.Hq,
+                             idx=self.idx[0], k_tail=self.KT[0], v_tail=self.VT[0],
+                             n_tail=self.k + 1)
+        need = max(lib().vc_glue_workspace_size(ctypes.byref(m)), draft_workspace_size(probe))
+        self._nat_ws = torch.empty(need, dtype=torch.uint8, device=self.dev)
         m.ws, m.ws_bytes = self._nat_ws.data_ptr(), self._nat_ws.numel()
         self._nat, self._nat_key = m, key
         return m

@@ -30,6 +30,23 @@ def test_library_exports_every_declared_function():
     assert sorted(os.listdir(os.path.join(ROOT, "include"))) == ["vericache.h", "vericache_glue.h"]
 
 
+def test_glue_workspace_covers_both_verify_windows():
+    """vc_glue_workspace_size is host arithmetic: the prefill's 4096-key windows over
+    min(rows_cap, 1024 / g) rows and the decode blocks' smaller windows over tail_cap rows
+    (more splits), whichever is larger; 0 for an invalid descriptor."""
+    L = vc.lib()
+    m = _lib.TinyLM()
+    m.n_layers, m.d_model, m.Hq, m.Hkv, m.D = 4, 512, 8, 2, 64
+    m.cap, m.rows_cap, m.tail_cap = 8738, 8192, 33
+    need = L.vc_glue_workspace_size(ctypes.byref(m))
+    prefill = L.vc_verify_workspace_size(1, 256, 8, 2, 64, 0, 8738)
+    assert need >= prefill > 0
+    # decode blocks: 33 rows x 4 heads over windows of at most 4096 keys
+    assert need >= L.vc_verify_workspace_size(1, 33, 8, 2, 64, 0, 8738)
+    m.Hkv = 3
+    assert L.vc_glue_workspace_size(ctypes.byref(m)) == 0
+
+
 def test_status_strings_and_version():
     L = vc.lib()
     assert L.vc_abi_version() == 1
