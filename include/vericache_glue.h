@@ -39,9 +39,22 @@ vc_status vc_glue_rmsnorm(const float* x, int n, int d, float eps, void* out,
 
 /* c[M, N] (+)= a[M, K] @ w[K, N]: a, w bf16 row-major, c fp32, fp32 accumulation in a
  * fixed K order.  accumulate != 0 adds into c (residual connections).
- * K % 16 == 0, N % 64 == 0. */
+ * K % 16 == 0, K <= 4096, N % 64 == 0. */
 vc_status vc_glue_gemm(const void* a, const void* w, int M, int K, int N, float* c,
                        int accumulate, cudaStream_t stream);
+
+/* vc_glue_gemm with a = the RMSNorm of x's rows (as vc_glue_rmsnorm, the same rounding:
+ * bf16(x * 1 / sqrt(mean(x^2) + eps))) formed inside the kernel: x fp32 [M, K],
+ * K % 256 == 0, K <= 4096.  The same result as vc_glue_rmsnorm then vc_glue_gemm, bit for
+ * bit, in one launch. */
+vc_status vc_glue_rmsnorm_gemm(const float* x, float eps, const void* w, int M, int K, int N,
+                               float* c, int accumulate, cudaStream_t stream);
+
+/* vc_glue_gemm with a = SwiGLU of gu (as vc_glue_swiglu) formed inside the kernel: gu fp32
+ * [M, 2F] (gate | up), w bf16 [F, N], F % 16 == 0, F <= 4096.  The same result as
+ * vc_glue_swiglu then vc_glue_gemm, bit for bit, in one launch. */
+vc_status vc_glue_swiglu_gemm(const float* gu, const void* w, int M, int F, int N, float* c,
+                              int accumulate, cudaStream_t stream);
 
 /* Split fused projections qkv fp32 [n, (Hq + 2 Hkv) * D] (q | k | v), rotate q and k by
  * rotate-half RoPE at positions pos[i] (theta base), write q_out bf16 [n, Hq, D], and store

@@ -29,7 +29,8 @@ EXPORTS = (
 GLUE_EXPORTS = (
     "vc_glue_embed", "vc_glue_rmsnorm", "vc_glue_gemm", "vc_glue_rope_store",
     "vc_glue_swiglu", "vc_glue_append_slots", "vc_glue_forward_full", "vc_glue_draft_steps",
-    "vc_glue_greedy_steps", "vc_glue_workspace_size",
+    "vc_glue_greedy_steps", "vc_glue_workspace_size", "vc_glue_rmsnorm_gemm",
+    "vc_glue_swiglu_gemm",
 )
 
 _p = ctypes.c_void_p
@@ -138,6 +139,10 @@ def lib() -> ctypes.CDLL:
         L.vc_glue_rmsnorm.argtypes = [_p, ctypes.c_int, ctypes.c_int, ctypes.c_float, _p, _p]
         L.vc_glue_gemm.argtypes = [_p, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _p,
                                    ctypes.c_int, _p]
+        L.vc_glue_rmsnorm_gemm.argtypes = [_p, ctypes.c_float, _p, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, _p, ctypes.c_int, _p]
+        L.vc_glue_swiglu_gemm.argtypes = [_p, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _p,
+                                          ctypes.c_int, _p]
         L.vc_glue_rope_store.argtypes = [_p, _p, _p] + [ctypes.c_int] * 4 + [ctypes.c_float,
                                                                              _p, _p, _p,
                                                                              ctypes.c_int, _p]

@@ -3,6 +3,8 @@
 // number of rows, so a block of k+1 tokens and k+1 single tokens agree bit for bit.
 #include <math.h>
 
+#include <atomic>
+
 #include "vc_common.cuh"
 #include "vc_internal.h"
 #include "vericache_glue.h"
@@ -35,20 +37,36 @@ __global__ void rmsnorm_kernel(const float* __restrict__ x, int n, int d, float 
   for (int j = lane; j < d; j += 32) out[(int64_t)row * d + j] = __float2bfloat16_rn(xr[j] * inv);
 }
 
-// c[16 x 64 tile] (+)= a[16 x K] @ w[K x 64]: 4 warps x (16 rows x 16 cols), k-steps of
-// 16 in order.  A stage holds 64 k-rows of w (128-byte rows) and the same 64 k-columns of
-// the 16 a rows, both XOR-swizzled, copied by cp.async into a 4-stage ring, so three
-// stages (30 KB) are in flight while one is multiplied; a and w fragments come from
-// shared memory by ldmatrix (w transposed).  Rows past M read as zero.  The k-steps and
-// their order are the same whatever M, so a row's result does not depend on M.
+// c[16 x 64 tile] (+)= A[16 x K] @ w[K x 64]: 4 warps x (16 rows x 16 cols), k-steps of
+// 16 in order.  The CTA's 16 rows of A are built once in shared memory (K * 32 bytes,
+// 16-byte chunks XOR-swizzled within each group of 8), from
+//   kGemmBf16:    a bf16 matrix (cp.async),
+//   kGemmRmsNorm: RMSNorm of fp32 rows x (a row staged in shared memory by all threads,
+//                 then the rmsnorm kernel's sum of squares, order and rounding by one
+//                 warp, so the product is the same as normalising first),
+//   kGemmSwiGLU:  bf16(silu(g) u) of fp32 rows gu = (g | u), as the swiglu kernel,
+// while w streams through a 4-stage cp.async ring of 64 k-rows (128-byte rows, swizzled);
+// fragments by ldmatrix (w transposed).  The k-steps and their
+// order are the same whatever M, so a row's result does not depend on M.
 constexpr int kGemmNst = 4;
 constexpr int kGemmKs = 64;                  // k-rows per stage
-__global__ void __launch_bounds__(128) gemm_kernel(const __nv_bfloat16* __restrict__ a,
+constexpr int kGemmBf16 = 0, kGemmRmsNorm = 1, kGemmSwiGLU = 2;
+constexpr int kGemmWBytes = kGemmNst * kGemmKs * 128;
+
+__device__ __forceinline__ uint32_t gemm_a_off(int row, int chunk, int K) {
+  const int nch = K >> 3;
+  const int c = (chunk | 7) < nch ? (chunk & ~7) | ((chunk ^ row) & 7) : chunk;
+  return (uint32_t)(row * K * 2 + c * 16);
+}
+
+template <int AMODE>
+__global__ void __launch_bounds__(128) gemm_kernel(const void* __restrict__ a_src, float eps,
                                                    const __nv_bfloat16* __restrict__ w, int M,
                                                    int K, int N, float* __restrict__ c,
                                                    int accumulate) {
-  __shared__ __align__(128) uint8_t sw[kGemmNst][kGemmKs * 128];
-  __shared__ __align__(128) uint8_t sa[kGemmNst][16 * 128];
+  extern __shared__ __align__(128) uint8_t gsm[];
+  uint8_t* sw = gsm;                                   // [kGemmNst][64 rows x 128 B]
+  uint8_t* sa = gsm + kGemmWBytes;                     // [16][K] bf16, swizzled
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qr = lane >> 2, qc = lane & 3;
   const int n0 = blockIdx.x * 64, m0 = blockIdx.y * 16;
@@ -62,21 +80,69 @@ __global__ void __launch_bounds__(128) gemm_kernel(const __nv_bfloat16* __restri
       const int row = e >> 3, ch = e & 7;
       const bool ok = kb + row < K;
       const __nv_bfloat16* src = w + (int64_t)(ok ? kb + row : 0) * N + n0 + ch * 8;
-      cp_async16(smem_u32(&sw[st][row * 128 + ((ch ^ (row & 7)) << 4)]), src, ok ? 16u : 0u);
-    }
-    {                                                 // a: 16 rows x 8 chunks
-      const int row = threadIdx.x >> 3, ch = threadIdx.x & 7;
-      const bool ok = m0 + row < M && kb + ch * 8 < K;
-      const __nv_bfloat16* src = a + (int64_t)(ok ? m0 + row : 0) * K + (ok ? kb + ch * 8 : 0);
-      cp_async16(smem_u32(&sa[st][row * 128 + ((ch ^ (row & 7)) << 4)]), src, ok ? 16u : 0u);
+      cp_async16(smem_u32(sw + st * (kGemmKs * 128) + row * 128 + ((ch ^ (row & 7)) << 4)), src,
+                 ok ? 16u : 0u);
     }
   };
-  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  // ---- A rows: bf16 copies join the first copy group; the fp32 modes are computed while
+  //      the first w stages are in flight
+  if constexpr (AMODE == kGemmBf16) {
+    const __nv_bfloat16* a = static_cast<const __nv_bfloat16*>(a_src);
+    const int nch = K >> 3;
+    for (int e = threadIdx.x; e < 16 * nch; e += 128) {
+      const int row = e / nch, ch = e - row * nch;
+      const bool ok = m0 + row < M;
+      cp_async16(smem_u32(sa + gemm_a_off(row, ch, K)),
+                 a + (int64_t)(ok ? m0 + row : 0) * K + ch * 8, ok ? 16u : 0u);
+    }
+  }
 #pragma unroll
   for (int st = 0; st < kGemmNst - 1; ++st) {
     if (st < nstage) issue(st, st);
     cp_async_commit();
   }
+  if constexpr (AMODE != kGemmBf16) {
+    // all 128 threads build the rows (independent loads in flight together).  Rows past
+    // M are left as they are: a row of the product depends on its own row of A only, and
+    // rows past M are never stored.
+    const float* x = static_cast<const float*>(a_src);
+    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(sa);
+    const int rows = min(16, M - m0);
+    auto put = [&](int rr, int j, float v) {
+      dst[(gemm_a_off(rr, j >> 3, K) >> 1) + (j & 7)] = __float2bfloat16_rn(v);
+    };
+    if constexpr (AMODE == kGemmRmsNorm) {
+      float* xs = reinterpret_cast<float*>(sa + 32 * K);   // one row of x, fp32
+      float* inv_s = xs + K;
+      for (int rr = 0; rr < rows; ++rr) {
+        const float* xr = x + (int64_t)(m0 + rr) * K;
+#pragma unroll 4
+        for (int j = threadIdx.x; j < K; j += 128) xs[j] = xr[j];
+        __syncthreads();
+        if (warp == 0) {                               // the rmsnorm kernel's sum, order
+          float ss = 0.f;                              // and rounding
+          for (int j = lane; j < K; j += 32) ss = fmaf(xs[j], xs[j], ss);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+          if (lane == 0) *inv_s = 1.0f / sqrtf(ss / (float)K + eps);
+        }
+        __syncthreads();
+        const float inv = *inv_s;
+        for (int j = threadIdx.x; j < K; j += 128) put(rr, j, xs[j] * inv);
+        __syncthreads();
+      }
+    } else {
+      for (int rr = 0; rr < rows; ++rr) {
+        const float* gr = x + (int64_t)(m0 + rr) * 2 * K;
+#pragma unroll 4
+        for (int j = threadIdx.x; j < K; j += 128) {
+          const float g = gr[j], u = gr[K + j];
+          put(rr, j, g / (1.0f + expf(-g)) * u);
+        }
+      }
+    }
+  }
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   const int mi = lane >> 3;
   const int arow = (lane & 7) + 8 * (mi & 1), achk = mi >> 1;   // a: rows 0-15, k chunk 0/1
   const int krow = (mi & 1) * 8 + (lane & 7);                 // w: k rows of the step
@@ -86,15 +152,15 @@ __global__ void __launch_bounds__(128) gemm_kernel(const __nv_bfloat16* __restri
     cp_async_commit();
     cp_async_wait<kGemmNst - 1>();
     __syncthreads();
-    const int st = sg % kGemmNst;
+    const uint8_t* sws = sw + (sg % kGemmNst) * (kGemmKs * 128);
 #pragma unroll
     for (int kk = 0; kk < kGemmKs / 16; ++kk) {
-      if (sg * (kGemmKs / 16) + kk >= ksteps) break;
+      const int ks = sg * (kGemmKs / 16) + kk;
+      if (ks >= ksteps) break;
       uint32_t A0, A1, A2, A3, b0, b1, b2, b3;
-      const int ac = 2 * kk + achk;
-      ldsm_x4(smem_u32(&sa[st][arow * 128 + ((ac ^ (arow & 7)) << 4)]), A0, A1, A2, A3);
+      ldsm_x4(smem_u32(sa + gemm_a_off(arow, 2 * ks + achk, K)), A0, A1, A2, A3);
       const int wr = kk * 16 + krow;
-      ldsm_x4_t(smem_u32(&sw[st][wr * 128 + ((wch ^ (wr & 7)) << 4)]), b0, b1, b2, b3);
+      ldsm_x4_t(smem_u32(sws + wr * 128 + ((wch ^ (wr & 7)) << 4)), b0, b1, b2, b3);
       mma_bf16(acc[0], A0, A1, A2, A3, b0, b1);
       mma_bf16(acc[1], A0, A1, A2, A3, b2, b3);
     }
@@ -175,6 +241,32 @@ __global__ void append_slots_kernel(int32_t* idx, int32_t* deg, int Hkv, int S_c
 int blocks_for(int64_t n, int t) { return (int)((n + t - 1) / t); }
 
 }  // namespace
+
+template <int AMODE>
+static vc_status launch_gemm(const void* a, float eps, const void* w, int M, int K, int N,
+                             float* c, int accumulate, cudaStream_t stream) {
+  if (!a || !w || !c || M <= 0 || K <= 0 || N <= 0) return fail(VC_ERR_INVALID, "gemm: args");
+  if (K % 16 || N % 64) return fail(VC_ERR_UNSUPPORTED, "gemm: K %% 16 and N %% 64 must be 0");
+  if (K > 4096) return fail(VC_ERR_UNSUPPORTED, "gemm: K > 4096");
+  if (!al16(a) || !al16(w)) return fail(VC_ERR_INVALID, "gemm: misaligned");
+  // w ring, A rows (bf16), and for the RMSNorm one fp32 row and its scale
+  const int smem = kGemmWBytes + 32 * K + (AMODE == kGemmRmsNorm ? 4 * K + 16 : 0);
+  // the largest dynamic shared memory granted so far, per device
+  static std::atomic<int> granted[64];
+  int dev = 0;
+  VC_CUDA(cudaGetDevice(&dev));
+  if (smem > 48 * 1024 && (dev >= 64 || granted[dev].load() < smem)) {
+    VC_CUDA(cudaFuncSetAttribute(gemm_kernel<AMODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem));
+    if (dev < 64) granted[dev].store(smem);
+  }
+  dim3 grid(N / 64, (M + 15) / 16);
+  gemm_kernel<AMODE><<<grid, 128, smem, stream>>>(a, eps, static_cast<const __nv_bfloat16*>(w),
+                                                  M, K, N, c, accumulate);
+  VC_CUDA(cudaGetLastError());
+  return VC_OK;
+}
+
 }  // namespace vc
 
 using namespace vc;
@@ -199,17 +291,21 @@ vc_status vc_glue_rmsnorm(const float* x, int n, int d, float eps, void* out,
   return VC_OK;
 }
 
+
 vc_status vc_glue_gemm(const void* a, const void* w, int M, int K, int N, float* c,
                        int accumulate, cudaStream_t stream) {
-  if (!a || !w || !c || M <= 0 || K <= 0 || N <= 0) return fail(VC_ERR_INVALID, "gemm: args");
-  if (K % 16 || N % 64) return fail(VC_ERR_UNSUPPORTED, "gemm: K %% 16 and N %% 64 must be 0");
-  if (!al16(a) || !al16(w)) return fail(VC_ERR_INVALID, "gemm: misaligned");
-  dim3 grid(N / 64, (M + 15) / 16);
-  gemm_kernel<<<grid, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(a),
-                                        static_cast<const __nv_bfloat16*>(w), M, K, N, c,
-                                        accumulate);
-  VC_CUDA(cudaGetLastError());
-  return VC_OK;
+  return launch_gemm<kGemmBf16>(a, 0.f, w, M, K, N, c, accumulate, stream);
+}
+
+vc_status vc_glue_rmsnorm_gemm(const float* x, float eps, const void* w, int M, int K, int N,
+                               float* c, int accumulate, cudaStream_t stream) {
+  if (K % 256) return fail(VC_ERR_UNSUPPORTED, "rmsnorm_gemm: K %% 256 must be 0");
+  return launch_gemm<kGemmRmsNorm>(x, eps, w, M, K, N, c, accumulate, stream);
+}
+
+vc_status vc_glue_swiglu_gemm(const float* gu, const void* w, int M, int F, int N, float* c,
+                              int accumulate, cudaStream_t stream) {
+  return launch_gemm<kGemmSwiGLU>(gu, 0.f, w, M, F, N, c, accumulate, stream);
 }
 
 vc_status vc_glue_rope_store(const float* qkv, const int32_t* pos, const int32_t* dst_row,
@@ -262,26 +358,26 @@ vc_status check_model(const vc_tinylm* m) {
 vc_status layer_tail(const vc_tinylm* m, int l, int n, cudaStream_t s) {
   vc_status st;
   if ((st = vc_glue_gemm(m->att, m->wo[l], n, m->Hq * m->D, m->d_model, m->x, 1, s))) return st;
-  if ((st = vc_glue_rmsnorm(m->x, n, m->d_model, m->rms_eps, m->h, s))) return st;
-  if ((st = vc_glue_gemm(m->h, m->wgu[l], n, m->d_model, 2 * m->ffn, m->gu, 0, s))) return st;
-  if ((st = vc_glue_swiglu(m->gu, n, m->ffn, m->act, s))) return st;
-  return vc_glue_gemm(m->act, m->wdown[l], n, m->ffn, m->d_model, m->x, 1, s);
+  if ((st = vc_glue_rmsnorm_gemm(m->x, m->rms_eps, m->wgu[l], n, m->d_model, 2 * m->ffn, m->gu,
+                                 0, s)))
+    return st;
+  return vc_glue_swiglu_gemm(m->gu, m->wdown[l], n, m->ffn, m->d_model, m->x, 1, s);
 }
 
 vc_status layer_head(const vc_tinylm* m, int l, int n, const int32_t* pos, const int32_t* dst,
                      void* kc, void* vcache, int cap, cudaStream_t s) {
   vc_status st;
   const int nqkv = (m->Hq + 2 * m->Hkv) * m->D;
-  if ((st = vc_glue_rmsnorm(m->x, n, m->d_model, m->rms_eps, m->h, s))) return st;
-  if ((st = vc_glue_gemm(m->h, m->wqkv[l], n, m->d_model, nqkv, m->qkv, 0, s))) return st;
+  if ((st = vc_glue_rmsnorm_gemm(m->x, m->rms_eps, m->wqkv[l], n, m->d_model, nqkv, m->qkv, 0,
+                                 s)))
+    return st;
   return vc_glue_rope_store(m->qkv, pos, dst, n, m->Hq, m->Hkv, m->D, m->rope_theta, m->q, kc,
                             vcache, cap, s);
 }
 
 vc_status logits_of(const vc_tinylm* m, int n, cudaStream_t s) {
-  vc_status st;
-  if ((st = vc_glue_rmsnorm(m->x, n, m->d_model, m->rms_eps, m->h, s))) return st;
-  return vc_glue_gemm(m->h, m->lm_head, n, m->d_model, m->vocab, m->logits, 0, s);
+  return vc_glue_rmsnorm_gemm(m->x, m->rms_eps, m->lm_head, n, m->d_model, m->vocab, m->logits,
+                              0, s);
 }
 
 // Key window of the verify calls of decode-sized blocks (at most tail_cap tokens: a

@@ -433,8 +433,9 @@ __global__ void __launch_bounds__(kVThreads, 1)
 
 // Merge split partials (plus the carried state) for one query row: one warp per row,
 // lanes holding D/32 output channels each.  The lanes load the splits' (max, sum) at
-// once; the unnormalised outputs of 8 splits are loaded together before any is used,
-// so a row costs a few L2 round trips, not one per split.  The sums run in split order
+// once (kept in registers for up to 64 splits); the unnormalised outputs of 32 (D 64) or
+// 16 (D 128) splits are loaded together before any is used, so a row costs a few L2
+// round trips, not one per split.  The sums run in split order
 // after the carried state, the same order whatever the number of rows, which keeps a
 // verify row bit-identical to the same position decoded alone.
 constexpr int kVCombWarps = 8;
@@ -447,7 +448,7 @@ __global__ void __launch_bounds__(kVCombWarps * 32) verify_combine_kernel(
   pdl_wait();
   pdl_trigger();
   constexpr int DPL = D / 32;
-  constexpr int CH = 8;
+  constexpr int CH = 64 / DPL;                    // splits whose outputs are loaded at once
   const int lane = threadIdx.x & 31;
   const int gr = blockIdx.x * kVCombWarps + (threadIdx.x >> 5);
   if (gr >= rows) return;
@@ -457,8 +458,16 @@ __global__ void __launch_bounds__(kVCombWarps * 32) verify_combine_kernel(
   const int64_t sidx = ((int64_t)b * n_q + i) * Hq + kvh * g + hl;
   const bool carry = m_state != nullptr && !(flags & VC_VERIFY_FIRST);
   const int64_t pr0 = (int64_t)pair * n_split * R + row;   // split s: pr0 + s * R
+  // (max, sum) of up to 64 splits stay in registers (lane: splits lane and 32 + lane);
+  // more splits are read again group by group below
+  float2 mlr[2] = {make_float2(-INFINITY, 0.f), make_float2(-INFINITY, 0.f)};
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+    if (32 * h + lane < n_split)
+      mlr[h] = *reinterpret_cast<const float2*>(ws_ml + (pr0 + (int64_t)(32 * h + lane) * R) * 2);
   float M = carry ? m_state[sidx] : -INFINITY;
-  for (int s = lane; s < n_split; s += 32) M = fmaxf(M, ws_ml[(pr0 + (int64_t)s * R) * 2]);
+  M = fmaxf(M, fmaxf(mlr[0].x, mlr[1].x));
+  for (int s = 64 + lane; s < n_split; s += 32) M = fmaxf(M, ws_ml[(pr0 + (int64_t)s * R) * 2]);
   M = warp_max_xor(M, 5);
   float Ls = 0.f, O[DPL];
 #pragma unroll
@@ -472,15 +481,19 @@ __global__ void __launch_bounds__(kVCombWarps * 32) verify_combine_kernel(
       for (int t = 0; t < DPL; ++t) O[t] = acc_state[sidx * D + lane * DPL + t] * f;
     }
   }
+  // the splits in order: weight exp2(m_s - M), sums and outputs added one split at a time
   for (int s0 = 0; s0 < n_split; s0 += 32) {
     const int cnt32 = min(32, n_split - s0);
+    float2 ml = make_float2(-INFINITY, 0.f);
+    if (s0 < 64) {
+      ml = s0 == 0 ? mlr[0] : mlr[1];
+    } else if (lane < cnt32) {
+      ml = *reinterpret_cast<const float2*>(ws_ml + (pr0 + (int64_t)(s0 + lane) * R) * 2);
+    }
     float wl = 0.f, ll = 0.f;
-    if (lane < cnt32) {
-      const float2 ml = *reinterpret_cast<const float2*>(ws_ml + (pr0 + (int64_t)(s0 + lane) * R) * 2);
-      if (ml.x > -INFINITY) {
-        wl = ex2(ml.x - M);
-        ll = ml.y;
-      }
+    if (lane < cnt32 && ml.x > -INFINITY) {
+      wl = ex2(ml.x - M);
+      ll = ml.y;
     }
     for (int c0 = 0; c0 < cnt32; c0 += CH) {
       float v[CH][DPL];
@@ -496,10 +509,11 @@ __global__ void __launch_bounds__(kVCombWarps * 32) verify_combine_kernel(
           v[j][0] = t.x; v[j][1] = t.y;
         }
       }
+      asm volatile("" ::: "memory");              // every load of the batch issued first
 #pragma unroll
       for (int j = 0; j < CH; ++j) {
-        const float w = __shfl_sync(0xffffffffu, wl, c0 + j);
-        const float lj = __shfl_sync(0xffffffffu, ll, c0 + j);
+        const float w = __shfl_sync(0xffffffffu, wl, (c0 + j) & 31);
+        const float lj = __shfl_sync(0xffffffffu, ll, (c0 + j) & 31);
         if (c0 + j < cnt32 && w != 0.f) {         // warp-uniform
           Ls = fmaf(lj, w, Ls);
 #pragma unroll

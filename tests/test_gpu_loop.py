@@ -11,6 +11,8 @@ outputs identical to full-KV greedy decoding).
 """
 import dataclasses
 
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -26,6 +28,37 @@ from synth.configs import LoopConfig, get_config
 
 pytestmark = pytest.mark.gpu
 S = lambda: torch.cuda.current_stream().cuda_stream
+
+
+@pytest.mark.parametrize("M", [1, 37])
+def test_fused_norm_and_swiglu_gemms_equal_the_two_step_forms(M):
+    """vc_glue_rmsnorm_gemm == vc_glue_rmsnorm then vc_glue_gemm, and vc_glue_swiglu_gemm ==
+    vc_glue_swiglu then vc_glue_gemm, bit for bit (accumulating into a residual too)."""
+    torch.manual_seed(M)
+    d, F = 512, 1408
+    x = torch.randn(M, d, device="cuda") * 3
+    w1 = (torch.randn(d, 2 * F, device="cuda") * 0.02).bfloat16()
+    h = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+    two = torch.empty(M, 2 * F, device="cuda")
+    one = torch.empty(M, 2 * F, device="cuda")
+    check(lib().vc_glue_rmsnorm(x.data_ptr(), M, d, ctypes.c_float(1e-5), h.data_ptr(), S()), "rmsnorm")
+    check(lib().vc_glue_gemm(h.data_ptr(), w1.data_ptr(), M, d, 2 * F, two.data_ptr(), 0, S()), "gemm")
+    check(lib().vc_glue_rmsnorm_gemm(x.data_ptr(), ctypes.c_float(1e-5), w1.data_ptr(), M, d,
+                                     2 * F, one.data_ptr(), 0, S()), "rmsnorm_gemm")
+    torch.cuda.synchronize()
+    assert torch.equal(one, two)
+    gu = two
+    w2 = (torch.randn(F, d, device="cuda") * 0.02).bfloat16()
+    act = torch.empty(M, F, dtype=torch.bfloat16, device="cuda")
+    res = torch.randn(M, d, device="cuda")
+    a2, b2 = res.clone(), res.clone()
+    check(lib().vc_glue_swiglu(gu.data_ptr(), M, F, act.data_ptr(), S()), "swiglu")
+    check(lib().vc_glue_gemm(act.data_ptr(), w2.data_ptr(), M, F, d, a2.data_ptr(), 1, S()), "gemm")
+    check(lib().vc_glue_swiglu_gemm(gu.data_ptr(), w2.data_ptr(), M, F, d, b2.data_ptr(), 1, S()),
+          "swiglu_gemm")
+    torch.cuda.synchronize()
+    assert torch.equal(a2, b2)
+    assert not torch.equal(a2, res)
 
 
 @pytest.mark.parametrize("K,N", [(512, 1408 * 2), (1408, 512), (80, 128)])
