@@ -77,29 +77,6 @@ struct DraftSmem {
 
 template <int D, int NST>
 __global__ void __launch_bounds__(128, 2) draft_indexed_kernel(const DraftIndexedParams p) {
-  // While the previous kernel on the stream may still run: an L2 prefetch of the K and V
-  // rows of this warp's first two tiles.  Nothing is read into the SM: the slot codes are
-  // read around L1 (ld.global.cg) and clamped into the cache, and only steer the prefetch,
-  // so a code the previous kernel is still writing costs a wasted prefetch, never a wrong
-  // value.  Tail rows (which the previous kernel may be writing) are not prefetched.
-  {
-    const int64_t gw0 = (int64_t)blockIdx.x * kDraftWarps + (threadIdx.x >> 5);
-    const int64_t xb = warp_begin(gw0, p.T, p.W);
-    const int nn = (int)(warp_begin(gw0 + 1, p.T, p.W) - xb);
-    const int t = (threadIdx.x & 31) >> 4;                // tile 0 or 1 of the warp
-    if (t < nn) {
-      const int64_t x = xb + t;
-      const int64_t pair = x / p.tpp;
-      const int s = (int)(x - pair * p.tpp) * kTile + (threadIdx.x & 15);
-      if (s < p.S) {
-        int64_t code = p.idx ? (int64_t)__ldcg(p.idx + pair * p.S_cap + s) : s;
-        code = code < 0 ? 0 : (code >= p.T_cap ? p.T_cap - 1 : code);
-        const int64_t row = (pair * p.T_cap + code) * D;
-        bulk_prefetch_l2(p.k + row, D * 2);
-        bulk_prefetch_l2(p.v + row, D * 2);
-      }
-    }
-  }
   pdl_wait();
   pdl_trigger();
   using SM = DraftSmem<D>;
