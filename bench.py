@@ -416,7 +416,8 @@ class Round:
 
 def e2e_measure(rnd, steps: int, warmup: int, device) -> dict:
     """Same metric through the public Python API, with every step's inputs copied
-    from pinned host memory and its results read back inside the timed region."""
+    from pinned host memory and its results read back inside the timed region (the
+    copies on a side stream, each kernel waiting for its own inputs only)."""
     import torch
     vc = rnd.vc
     cfg = rnd.cfg
@@ -432,19 +433,41 @@ def e2e_measure(rnd, steps: int, warmup: int, device) -> dict:
     d2h = sum(x.numel() * x.element_size() for x in (o_d, o_v, o_c, o_n))
     n_q = cfg.k + 1
 
+    # The step's inputs go host -> device on a copy stream in the order the round needs
+    # them (queries and tail first, then each draft step's logits, then the verify
+    # logits); each consumer waits for its own copy only, so the PCIe transfer overlaps
+    # the drafting and the verify instead of preceding them.
+    cs = torch.cuda.Stream(device=device)
+    ev_in = torch.cuda.Event()
+    ev_dl = [torch.cuda.Event() for _ in range(cfg.k)]
+    ev_qv = torch.cuda.Event()
+    ev_lg = torch.cuda.Event()
+
     def one():
-        rnd.q_draft.copy_(h_qd, non_blocking=True)
-        rnd.q_verify.copy_(h_qv, non_blocking=True)
-        rnd.draft_logits.copy_(h_dl, non_blocking=True)
-        rnd.logits.copy_(h_lg, non_blocking=True)
-        rnd.drafts.copy_(h_dr, non_blocking=True)
-        rnd.KT[0].copy_(h_kt, non_blocking=True)
-        rnd.VT[0].copy_(h_vt, non_blocking=True)
+        cur = torch.cuda.current_stream()
+        cs.wait_stream(cur)                      # the previous step's reads are done
+        with torch.cuda.stream(cs):
+            rnd.q_draft.copy_(h_qd, non_blocking=True)
+            rnd.KT[0].copy_(h_kt, non_blocking=True)
+            rnd.VT[0].copy_(h_vt, non_blocking=True)
+            ev_in.record(cs)
+            for j in range(cfg.k):
+                rnd.draft_logits[j].copy_(h_dl[j], non_blocking=True)
+                ev_dl[j].record(cs)
+            rnd.q_verify.copy_(h_qv, non_blocking=True)
+            rnd.drafts.copy_(h_dr, non_blocking=True)
+            ev_qv.record(cs)
+            rnd.logits.copy_(h_lg, non_blocking=True)
+            ev_lg.record(cs)
+        cur.wait_event(ev_in)
         for j in range(cfg.k):
             vc.draft_attn(rnd.q_draft[j], rnd.caches[j], out=rnd.d_out[j], ws=rnd.ws_d)
+            cur.wait_event(ev_dl[j])
             vc.accept(rnd.draft_logits[j], None, target=rnd.d_target[j], err_flag=rnd.d_err[j])
+        cur.wait_event(ev_qv)
         vc.verify_attn(rnd.q_verify, rnd.K[cfg.k % N_COPIES], rnd.V[cfg.k % N_COPIES], cfg.P,
                        out=rnd.v_out, ws=rnd.ws_v)
+        cur.wait_event(ev_lg)
         vc.accept(rnd.logits, rnd.drafts, target=rnd.target, accept_len=rnd.alen,
                   commit=rnd.commit, n_commit=rnd.ncommit, err_flag=rnd.err)
         o_d.copy_(rnd.d_out, non_blocking=True)
