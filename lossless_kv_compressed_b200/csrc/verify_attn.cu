@@ -14,19 +14,20 @@
 //
 // Per CTA (384 threads):
 //   warp 0      TMA producer: K and V tiles [64 keys x D] (128-byte swizzle) into a
-//               6-stage ring, one mbarrier per stage with the transaction byte count.
+//               5-stage ring, one mbarrier per stage with the transaction byte count.
 //   warp 1      TMEM allocator; one thread of warp 1 (M-tile 0) and one of warp 2
 //   warp 2      (M-tile 1) issue the UMMAs: the tile's next S = Q K^T as soon as its
 //               softmax has copied the current S out of TMEM, then O += P V once its
-//               P is in.  Q of M-tile 0 is read from TMEM, Q of M-tile 1 from shared
-//               memory; P from TMEM, K and V from shared memory (V as an N-major B).
+//               P is in.  Q of both M-tiles, K and V are read from shared memory (V as
+//               an N-major B), P from TMEM.  (Q of M-tile 0 read from TMEM contended
+//               with the softmax's TMEM loads: Q K^T took ~3x the time of P V.)
 //   warps 4-7   softmax of M-tile 0, warps 8-11 of M-tile 1: one thread per query row
 //               (TMEM lane); M-tile 1 keeps row r in lane (r + 64) % 128, so a part-
 //               filled second tile lands on sub-partitions 2-3.  Scores in the log2
 //               domain, running max kept unless it grows by more than 2^8 (then O in
 //               TMEM is rescaled after the previous P.V), P written as bf16 into the
 //               M-tile's P columns once the previous P.V has read them.
-// TMEM columns: O0 [0,D), O1 [D,2D), S0, S1 (64 each), P0, P1 (32 each), Q0 (D/2).
+// TMEM columns: O0 [0,D), O1 [D,2D), S0, S1 (64 each), P0, P1 (32 each).
 // Every mbarrier wait is bounded in time (pipeline waits by a launch parameter, 2 s
 // unless vc_set_wait_limit changed it; teardown waits by 1 s); on expiry the CTA raises
 // the library's device error word, lets its copies and products in flight land,
@@ -48,7 +49,7 @@ __device__ int g_vc_dev_error;   // bit 0: a bounded wait in the verify kernel e
 
 constexpr int kBN = 64;
 constexpr int kVThreads = 384;
-constexpr int kNSt = 6;
+constexpr int kNSt = 5;
 constexpr float kRescaleLog2 = 8.f;
 
 struct VerifyParams {
@@ -65,9 +66,10 @@ struct VerifyParams {
 
 template <int D>
 struct VLayout {
-  static constexpr int kQTile = 128 * D * 2;        // Q of M-tile 1 (128-byte swizzle)
+  static constexpr int kQTile = 128 * D * 2;        // Q of one M-tile (128-byte swizzle)
   static constexpr int kKVTile = kBN * D * 2;
-  static constexpr int kQ1 = 0;
+  static constexpr int kQ0 = 0;
+  static constexpr int kQ1 = kQ0 + kQTile;
   static constexpr int kK = kQ1 + kQTile;
   static constexpr int kV = kK + kNSt * kKVTile;
   static constexpr int kBar = kV + kNSt * kKVTile;
@@ -79,9 +81,8 @@ struct VLayout {
   static constexpr uint32_t kColO = 0;
   static constexpr uint32_t kColS = 2 * D;
   static constexpr uint32_t kColP = 2 * D + 2 * kBN;
-  static constexpr uint32_t kColQ0 = kColP + 2 * (kBN / 2);
   static constexpr uint32_t kTmemCols = 512;
-  static_assert(kColQ0 + D / 2 <= kTmemCols, "TMEM columns");
+  static_assert(kColP + 2 * (kBN / 2) <= kTmemCols, "TMEM columns");
   static_assert(kQTile % 1024 == 0 && kKVTile % 1024 == 0, "align");
 };
 
@@ -157,9 +158,8 @@ __global__ void __launch_bounds__(kVThreads, 1)
   tc::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlot);
 
-  // Q rows of this group: M-tile 0 into TMEM (row r in lane r, two bf16 per column), M-tile
-  // 1 into shared memory (K-major, 128-byte swizzle, row r at row (r + 64) % 128);
-  // padding rows are zero.
+  // Q rows of this group into shared memory (K-major, 128-byte swizzle; M-tile 0 row r at
+  // row r, M-tile 1 row r at row (r + 64) % 128); padding rows are zero.
   if (warp >= 4) {
     const int mt = (warp - 4) >> 2, q4 = warp & 3;
     const int rl = 32 * q4 + lane;                       // TMEM lane / UMMA row
@@ -170,25 +170,13 @@ __global__ void __launch_bounds__(kVThreads, 1)
       const int i = grow / p.g, hl = grow - i * p.g;
       src = reinterpret_cast<const uint4*>(p.q + (((int64_t)b * p.n_q + i) * p.Hq + kvh * p.g + hl) * D);
     }
-    if (mt == 0) {
-      const uint32_t q_t = tmem + ((uint32_t)(32 * q4) << 16) + L::kColQ0;
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t w[32];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint4 v = ok ? __ldg(src + 8 * c + u) : make_uint4(0u, 0u, 0u, 0u);
-          w[4 * u] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
-        }
-        tc::tmem_st32(q_t + 32 * c, w);
-      }
-      tc::tmem_wait_st();
-    } else {
+    {
+      const int qbase = mt == 0 ? L::kQ0 : L::kQ1;
 #pragma unroll
       for (int ch = 0; ch < D / 8; ++ch) {
         const uint4 v = ok ? __ldg(src + ch) : make_uint4(0u, 0u, 0u, 0u);
         const int cb = ch >> 3, cc = ch & 7;
-        *reinterpret_cast<uint4*>(smem + L::kQ1 + cb * (128 * 128) + rl * 128 +
+        *reinterpret_cast<uint4*>(smem + qbase + cb * (128 * 128) + rl * 128 +
                                   ((cc ^ (rl & 7)) << 4)) = v;
       }
       tc::fence_proxy_async();
@@ -245,13 +233,10 @@ __global__ void __launch_bounds__(kVThreads, 1)
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t bb = sb + L::kK + st * L::kKVTile + (ks >> 2) * (kBN * 128) + (ks & 3) * 32;
           const uint64_t bdesc = tc::sdesc_sw128(bb, 16, 1024);
-          if (mt == 0) {
-            tc::umma_ts(tmem + L::kColS, tmem + L::kColQ0 + ks * 8, bdesc, id_qk, ks > 0 ? 1u : 0u);
-          } else {
-            const uint32_t a = sb + L::kQ1 + (ks >> 2) * (128 * 128) + (ks & 3) * 32;
-            tc::umma_ss(tmem + L::kColS + kBN, tc::sdesc_sw128(a, 16, 1024), bdesc, id_qk,
-                        ks > 0 ? 1u : 0u);
-          }
+          const uint32_t a = sb + (mt == 0 ? L::kQ0 : L::kQ1) + (ks >> 2) * (128 * 128) +
+                             (ks & 3) * 32;
+          tc::umma_ss(tmem + L::kColS + mt * kBN, tc::sdesc_sw128(a, 16, 1024), bdesc, id_qk,
+                      ks > 0 ? 1u : 0u);
         }
       };
       auto pv = [&](int t) {
