@@ -39,6 +39,27 @@ int num_sms() {
   return cache[dev];
 }
 
+cudaError_t grant_smem(const void* func, int bytes) {
+  struct Granted { const void* func; int dev; int bytes; };
+  static std::mutex mu;
+  static std::vector<Granted> granted;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  for (Granted& g : granted) {
+    if (g.func == func && g.dev == dev) {
+      if (g.bytes >= bytes) return cudaSuccess;
+      e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+      if (e == cudaSuccess) g.bytes = bytes;
+      return e;
+    }
+  }
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) granted.push_back({func, dev, bytes});
+  return e;
+}
+
 vc_status stage_full_kv(void* dst, const void* src, size_t bytes, size_t chunk,
                         cudaStream_t stream, cudaEvent_t* done, int n_events);
 vc_status event_wait(cudaEvent_t ev, double timeout_s);

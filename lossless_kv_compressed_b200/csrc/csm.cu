@@ -441,13 +441,11 @@ vc_status launch_csm(const void* k, const void* v, const int32_t* deg, int pairs
   p.out_len = (int)csm_out_len(T, n_sinks, n_recent, chunk, r);
   const dim3 grid(p.n_chunks + 1, pairs);
   if (D == 128) {
-    VC_CUDA(cudaFuncSetAttribute(csm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 CsmSmem<128>::kTotal));
+    VC_CUDA(grant_smem((const void*)csm_kernel<128>, CsmSmem<128>::kTotal));
     VC_CUDA(launch_pdl(csm_kernel<128>, grid, dim3(kCsmThreads), CsmSmem<128>::kTotal, stream,
                        1, p));
   } else {
-    VC_CUDA(cudaFuncSetAttribute(csm_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 CsmSmem<64>::kTotal));
+    VC_CUDA(grant_smem((const void*)csm_kernel<64>, CsmSmem<64>::kTotal));
     VC_CUDA(launch_pdl(csm_kernel<64>, grid, dim3(kCsmThreads), CsmSmem<64>::kTotal, stream, 1,
                        p));
   }

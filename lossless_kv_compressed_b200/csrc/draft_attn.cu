@@ -896,8 +896,7 @@ DraftIndexedParams indexed_params(const void* q, const vc_comp_cache* c, int S, 
 template <int D>
 vc_status run_indexed(const DraftIndexedParams& p, cudaStream_t stream) {
   const size_t sm = draft_indexed_smem<D>();
-  VC_CUDA(cudaFuncSetAttribute(draft_indexed_kernel<D, kNStage>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+  VC_CUDA(grant_smem((const void*)draft_indexed_kernel<D, kNStage>, (int)sm));
   VC_CUDA(launch_pdl(draft_indexed_kernel<D, kNStage>, dim3(p.W / kDraftWarps), dim3(128), sm,
                      stream, 1, p));
   VC_CUDA(cudaGetLastError());
@@ -907,8 +906,7 @@ vc_status run_indexed(const DraftIndexedParams& p, cudaStream_t stream) {
 template <int D>
 vc_status run_int4(const DraftInt4Params& p, cudaStream_t stream) {
   const size_t sm = draft_int4_smem<D>();
-  VC_CUDA(cudaFuncSetAttribute(draft_int4_kernel<D, kNStageInt4>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+  VC_CUDA(grant_smem((const void*)draft_int4_kernel<D, kNStageInt4>, (int)sm));
   VC_CUDA(launch_pdl(draft_int4_kernel<D, kNStageInt4>, dim3(p.W / kDraftWarps), dim3(128), sm,
                      stream, 1, p));
   VC_CUDA(cudaGetLastError());

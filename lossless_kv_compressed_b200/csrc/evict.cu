@@ -280,8 +280,7 @@ static vc_status run_evict_scores(const EvictParams& p, int B, cudaStream_t stre
   const int pairs = B * p.Hkv;
   VC_CUDA(launch_pdl(evict_lse_kernel<D>, dim3(p.W, pairs), dim3(kEvThreads), 0, stream, 1, p));
   const size_t sm = ((size_t)p.W * p.g * D + (size_t)p.W * p.g) * sizeof(float);
-  VC_CUDA(cudaFuncSetAttribute(evict_score_kernel<D>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+  VC_CUDA(grant_smem((const void*)evict_score_kernel<D>, (int)sm));
   const unsigned nb = (unsigned)((p.n + kEvThreads - 1) / kEvThreads);
   VC_CUDA(launch_pdl(evict_score_kernel<D>, dim3(nb, pairs), dim3(kEvThreads), sm, stream, 1, p));
   VC_CUDA(cudaGetLastError());

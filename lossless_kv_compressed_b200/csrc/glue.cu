@@ -251,15 +251,7 @@ static vc_status launch_gemm(const void* a, float eps, const void* w, int M, int
   if (!al16(a) || !al16(w)) return fail(VC_ERR_INVALID, "gemm: misaligned");
   // w ring, A rows (bf16), and for the RMSNorm one fp32 row and its scale
   const int smem = kGemmWBytes + 32 * K + (AMODE == kGemmRmsNorm ? 4 * K + 16 : 0);
-  // the largest dynamic shared memory granted so far, per device
-  static std::atomic<int> granted[64];
-  int dev = 0;
-  VC_CUDA(cudaGetDevice(&dev));
-  if (smem > 48 * 1024 && (dev >= 64 || granted[dev].load() < smem)) {
-    VC_CUDA(cudaFuncSetAttribute(gemm_kernel<AMODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 smem));
-    if (dev < 64) granted[dev].store(smem);
-  }
+  if (smem > 48 * 1024) VC_CUDA(grant_smem((const void*)gemm_kernel<AMODE>, smem));
   dim3 grid(N / 64, (M + 15) / 16);
   gemm_kernel<AMODE><<<grid, 128, smem, stream>>>(a, eps, static_cast<const __nv_bfloat16*>(w),
                                                   M, K, N, c, accumulate);

@@ -12,6 +12,9 @@ namespace vc {
 vc_status fail(vc_status st, const char* fmt, ...);
 // Number of SMs of the current device (cached per device).
 int num_sms();
+// Raise a kernel's dynamic shared memory limit to at least bytes on the current device;
+// the attribute call is made only when the limit granted so far is smaller.
+cudaError_t grant_smem(const void* func, int bytes);
 
 #define VC_CUDA(call)                                                                \
   do {                                                                               \

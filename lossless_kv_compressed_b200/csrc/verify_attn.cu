@@ -582,8 +582,7 @@ static vc_status run_verify(const Plan& pl, const VerifyParams& vp, const CUtens
                             const CUtensorMap& mv, int flags, float* m, float* l, float* acc,
                             void* out, cudaStream_t stream) {
   using L = VLayout<D>;
-  VC_CUDA(cudaFuncSetAttribute(verify_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               L::kAlloc));
+  VC_CUDA(grant_smem((const void*)verify_kernel<D>, L::kAlloc));
   dim3 grid(pl.n_split, pl.n_rg, pl.pairs);
   VC_CUDA(launch_pdl(verify_kernel<D>, grid, dim3(kVThreads), L::kAlloc, stream, 1, mk, mv, vp));
   VC_CUDA(cudaGetLastError());

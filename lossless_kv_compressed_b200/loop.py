@@ -31,7 +31,7 @@ import torch
 
 from . import _lib
 from .api import (IndexedCache, accept, csm_compress, draft_attn, draft_workspace_size,
-                  evict_scores, evict_select, verify_attn)
+                  evict_scores, evict_select, verify_attn, verify_workspace_size)
 from ._lib import check, lib
 
 
@@ -145,11 +145,7 @@ class GpuTinyLM:
                 draft_attn(self.q[:1].view(1, c.Hq, c.D), cache,
                            out=self.att[:1].view(1, c.Hq, c.D))
             else:
-                for r0 in range(0, n, self.PREFILL_ROWS):
-                    r1 = min(n, r0 + self.PREFILL_ROWS)
-                    verify_attn(self.q[r0:r1].view(1, r1 - r0, c.Hq, c.D), self.K[l],
-                                self.V[l], pos0 + r0, out=self.att[r0:r1].view(1, r1 - r0,
-                                                                                c.Hq, c.D))
+                self._attend_full(n, pos0, l)
             self._gemm(self.att.view(self.rows, -1), self.wo[l], n, self.x, accumulate=True)
             self._norm(self.x, n, self.h)
             self._gemm(self.h, self.wgu[l], n, self.gu)
@@ -159,6 +155,37 @@ class GpuTinyLM:
         self._norm(self.x, n, self.h)
         self._gemm(self.h, self.lm_head, n, self.logits)
         return self.logits[:n]
+
+    PREFILL_STREAMS = 4
+
+    def _attend_full(self, n: int, pos0: int, l: int) -> None:
+        """Causal attention of rows [0, n) at positions pos0.. over layer l's full cache, in
+        blocks of PREFILL_ROWS positions.  The blocks are independent (disjoint rows of q
+        and att, the cache only read), so a long prompt's blocks run on a few side streams
+        at once, each with its own workspace; the caller's stream waits for all of them."""
+        c = self.cfg
+        blocks = list(range(0, n, self.PREFILL_ROWS))
+        def one(r0, ws=None):
+            r1 = min(n, r0 + self.PREFILL_ROWS)
+            verify_attn(self.q[r0:r1].view(1, r1 - r0, c.Hq, c.D), self.K[l], self.V[l],
+                        pos0 + r0, out=self.att[r0:r1].view(1, r1 - r0, c.Hq, c.D), ws=ws)
+        if len(blocks) == 1:
+            one(0)
+            return
+        if getattr(self, "_pf", None) is None:
+            need = verify_workspace_size(1, self.PREFILL_ROWS, c.Hq, c.Hkv, c.D, 0, self.max_len)
+            self._pf = [(torch.cuda.Stream(device=self.dev),
+                         torch.empty(need, dtype=torch.uint8, device=self.dev))
+                        for _ in range(self.PREFILL_STREAMS)]
+        cur = torch.cuda.current_stream(self.dev)
+        for st, _ in self._pf:
+            st.wait_stream(cur)
+        for i, r0 in enumerate(blocks):
+            st, ws = self._pf[i % len(self._pf)]
+            with torch.cuda.stream(st):
+                one(r0, ws)
+        for st, _ in self._pf:
+            cur.wait_stream(st)
 
     # ---------------------------------------------------------------- prefill
     def prefill(self, prompt: np.ndarray, score_window: int = 0):
