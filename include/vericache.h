@@ -177,8 +177,11 @@ vc_status vc_draft_attn_noalloc(const void* q, const vc_comp_cache* cache, float
  *         resets the state before adding this range; VC_VERIFY_LAST writes out after
  *         adding it.  Ranges must tile [0, P + n_q) exactly, in order.
  *   Results do not depend on n_q or on other rows: key tiles and split boundaries sit
- *   at fixed absolute positions, and splits are merged in a fixed order.
- *   ws: vc_verify_workspace_size(...) bytes of device memory.
+ *   at fixed absolute positions, and splits are merged in a fixed order.  The split
+ *   window (a multiple of 64 keys in [2048, 4096]; 4096 when B * Hkv * L_cap / 4096 is
+ *   under one CTA per SM) is chosen from B * Hkv and L_cap only, so that the CTAs fill the
+ *   SMs' last wave; every call on one cache uses the same one.
+ *   ws: vc_verify_workspace_size(...) bytes of device memory (enough for any window).
  *   Supported: D in {64, 128}, g <= 8, n_q * g <= 1024.
  * ---------------------------------------------------------------------------- */
 #define VC_VERIFY_FIRST 1

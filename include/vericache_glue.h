@@ -95,7 +95,8 @@ vc_status vc_glue_append_slots(int32_t* idx, int32_t* deg, int Hkv, int S_cap, i
  * Verify attention of blocks of at most tail_cap tokens (a greedy step, a block of k + 1)
  * splits the keys into windows chosen from Hkv and cap only (the largest power of two
  * <= 4096, >= 256, giving two CTAs per SM), so a block and the same tokens stepped one at
- * a time agree bit for bit; longer blocks (the prefill) use 4096-key windows.
+ * a time agree bit for bit; longer blocks (the prefill) use the window vc_verify_attn
+ * chooses for a cache of Hkv pairs and capacity cap.
  * -------------------------------------------------------------------------------- */
 typedef struct vc_tinylm {
   int32_t n_layers, d_model, Hq, Hkv, D, ffn, vocab;

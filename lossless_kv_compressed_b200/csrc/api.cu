@@ -148,7 +148,7 @@ size_t vc_verify_workspace_size(int B, int n_q, int Hq, int Hkv, int D, int64_t 
                                 int64_t kv_len) {
   if (B <= 0 || n_q <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || kv_start < 0 || kv_len <= 0)
     return 0;
-  return verify_workspace_bytes(B, n_q, Hq, Hkv, D, kv_start, kv_len);
+  return verify_workspace_bytes_any(B, n_q, Hq, Hkv, D, kv_start, kv_len);
 }
 
 vc_status vc_verify_attn(const void* q, int B, int n_q, int Hq, int Hkv, int D, const void* k,
@@ -156,7 +156,8 @@ vc_status vc_verify_attn(const void* q, int B, int n_q, int Hq, int Hkv, int D, 
                          int64_t P, float* m, float* l, float* acc, int flags, float scale,
                          void* out, void* ws, size_t ws_bytes, cudaStream_t stream) {
   return verify_checked(q, B, n_q, Hq, Hkv, D, k, v, L_cap, kv_start, kv_len, P, m, l, acc,
-                        flags, scale, out, ws, ws_bytes, stream, kVerifySplitKeys);
+                        flags, scale, out, ws, ws_bytes, stream,
+                        verify_window((int64_t)B * Hkv, L_cap));
 }
 
 }  // extern "C"

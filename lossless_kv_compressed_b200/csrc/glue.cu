@@ -376,7 +376,8 @@ vc_status logits_of(const vc_tinylm* m, int n, cudaStream_t s) {
 // single greedy step or a block of k + 1): the largest power of two <= 4096, and >= 256,
 // that still gives two CTAs per SM over the model's kv heads and cache capacity.  It
 // depends on the model only, so a k + 1 block and k + 1 single steps use the same window
-// and agree bit for bit.  Longer blocks (the prefill) use the library's default window.
+// and agree bit for bit.  Longer blocks (the prefill) use the window vc_verify_attn
+// chooses for this cache.
 int decode_split_keys(const vc_tinylm* m) {
   const int64_t want = 2 * (int64_t)num_sms();
   int w = kVerifySplitKeys;
@@ -386,7 +387,7 @@ int decode_split_keys(const vc_tinylm* m) {
 
 vc_status forward_full(const vc_tinylm* m, const int32_t* ids, int n, int pos0, cudaStream_t s) {
   vc_status st;
-  const int split = n <= m->tail_cap ? decode_split_keys(m) : kVerifySplitKeys;
+  const int split = n <= m->tail_cap ? decode_split_keys(m) : verify_window(m->Hkv, m->cap);
   if ((st = vc_glue_embed(m->embed, ids, n, m->d_model, m->x, s))) return st;
   const int g = m->Hq / m->Hkv;
   const int chunk = 1024 / g;
@@ -416,7 +417,7 @@ size_t vc_glue_workspace_size(const vc_tinylm* m) {
     return 0;
   const int g = m->Hq / m->Hkv;
   const int rows = m->rows_cap < 1024 / g ? m->rows_cap : 1024 / g;
-  size_t need = verify_workspace_bytes(1, rows, m->Hq, m->Hkv, m->D, 0, m->cap);
+  size_t need = verify_workspace_bytes_any(1, rows, m->Hq, m->Hkv, m->D, 0, m->cap);
   if (m->tail_cap > 0) {
     const size_t dec = verify_workspace_bytes(1, m->tail_cap, m->Hq, m->Hkv, m->D, 0, m->cap,
                                               decode_split_keys(m));

@@ -43,6 +43,12 @@ vc_status launch_verify(const void* q, int B, int n_q, int Hq, int Hkv, int D, c
                         int64_t P, float* m, float* l, float* acc, int flags, float scale,
                         void* out, void* ws, size_t ws_bytes, cudaStream_t stream,
                         int split_keys = kVerifySplitKeys);
+// The public entry point's window for a cache of pairs (batch x kv head) and capacity
+// L_cap: a function of those two only, so every call on one cache uses the same one.
+int verify_window(int64_t pairs, int64_t L_cap);
+// Workspace bytes enough for any window verify_window can return.
+size_t verify_workspace_bytes_any(int B, int n_q, int Hq, int Hkv, int D, int64_t kv_start,
+                                  int64_t kv_len);
 // vc_verify_attn's argument checks and launch with a chosen window.
 vc_status verify_checked(const void* q, int B, int n_q, int Hq, int Hkv, int D, const void* k,
                          const void* v, int64_t L_cap, int64_t kv_start, int64_t kv_len,

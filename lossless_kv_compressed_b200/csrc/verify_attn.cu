@@ -37,7 +37,12 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
+#include <climits>
+#include <functional>
+#include <mutex>
+#include <vector>
 
 #include "tc05.cuh"
 #include "vc_common.cuh"
@@ -575,6 +580,60 @@ Plan plan(int B, int n_q, int Hq, int Hkv, int D, int64_t kv_start, int64_t kv_l
 size_t verify_workspace_bytes(int B, int n_q, int Hq, int Hkv, int D, int64_t kv_start,
                               int64_t kv_len, int split_keys) {
   return plan(B, n_q, Hq, Hkv, D, kv_start, kv_len, split_keys).ws_bytes + 256;
+}
+
+constexpr int kWindowMin = 2048;
+
+size_t verify_workspace_bytes_any(int B, int n_q, int Hq, int Hkv, int D, int64_t kv_start,
+                                  int64_t kv_len) {
+  size_t m = 0;
+  for (int w = kVerifySplitKeys; w >= kWindowMin; w -= kBN)
+    m = std::max(m, verify_workspace_bytes(B, n_q, Hq, Hkv, D, kv_start, kv_len, w));
+  return m;
+}
+
+// Among the windows of 2048..4096 keys (multiples of 64), the one whose CTAs, placed in
+// launch order (pair-major, splits in order) on the SMs as each frees up (one resident
+// CTA per SM), finish first, a CTA costing its 64-key tiles plus four for its start; ties
+// go to the larger window.  Fewer, larger splits leave the last wave of CTAs half empty
+// at some sizes (512 CTAs of 64 tiles on 148 SMs), slightly smaller ones fill it.  The
+// choice is cached per (pairs, L_cap, SM count); caches with less than one wave of
+// 4096-key CTAs, or very large ones, keep 4096.
+int verify_window(int64_t pairs, int64_t L_cap) {
+  struct Chosen { int64_t pairs, L_cap; int sms, w; };
+  static std::mutex mu;
+  static std::vector<Chosen> chosen;
+  const int sms = num_sms();
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (const Chosen& c : chosen)
+      if (c.pairs == pairs && c.L_cap == L_cap && c.sms == sms) return c.w;
+  }
+  int best = kVerifySplitKeys;
+  const int64_t ctas4096 = pairs * ((L_cap + kVerifySplitKeys - 1) / kVerifySplitKeys);
+  if (pairs > 0 && L_cap > 0 && ctas4096 >= sms &&
+      pairs * ((L_cap + kWindowMin - 1) / kWindowMin) <= 65536) {
+    int64_t best_t = INT64_MAX;
+    std::vector<int64_t> heap;
+    for (int w = kVerifySplitKeys; w >= kWindowMin; w -= kBN) {
+      heap.assign(sms, 0);                      // min-heap of SM free times
+      const int64_t n_full = L_cap / w, rem = L_cap % w;
+      auto place = [&](int64_t cost) {
+        std::pop_heap(heap.begin(), heap.end(), std::greater<int64_t>());
+        heap.back() += cost;
+        std::push_heap(heap.begin(), heap.end(), std::greater<int64_t>());
+      };
+      for (int64_t pr = 0; pr < pairs; ++pr) {
+        for (int64_t sp = 0; sp < n_full; ++sp) place(w / kBN + 4);
+        if (rem) place((rem + kBN - 1) / kBN + 4);
+      }
+      const int64_t t = *std::max_element(heap.begin(), heap.end());
+      if (t < best_t) { best_t = t; best = w; }
+    }
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  chosen.push_back({pairs, L_cap, sms, best});
+  return best;
 }
 
 template <int D>

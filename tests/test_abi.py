@@ -31,9 +31,10 @@ def test_library_exports_every_declared_function():
 
 
 def test_glue_workspace_covers_both_verify_windows():
-    """vc_glue_workspace_size is host arithmetic: the prefill's 4096-key windows over
-    min(rows_cap, 1024 / g) rows and the decode blocks' smaller windows over tail_cap rows
-    (more splits), whichever is larger; 0 for an invalid descriptor."""
+    """vc_glue_workspace_size is host arithmetic: the prefill's blocks of min(rows_cap,
+    1024 / g) rows under any window vc_verify_attn may choose, and the decode blocks'
+    smaller windows over tail_cap rows (more splits), whichever is larger; 0 for an
+    invalid descriptor."""
     L = vc.lib()
     m = _lib.TinyLM()
     m.n_layers, m.d_model, m.Hq, m.Hkv, m.D = 4, 512, 8, 2, 64
