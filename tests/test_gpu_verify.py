@@ -86,6 +86,26 @@ def test_row_invariance(D, Hq, Hkv, P):
         assert torch.equal(one[:, 0], full[:, i]), f"row {i} differs"
 
 
+def test_row_invariance_at_the_32k_geometry():
+    """The same bit-exact row invariance on a cache large enough for vc_verify_attn to
+    choose a split window other than 4096 keys (64 pairs, 32801 keys of capacity): the
+    window depends on the cache only, so the block and each token alone share it."""
+    from synth import device as sd
+    B, Hq, Hkv, D, P, n_q = 8, 32, 8, 128, 32768, 33
+    g = sd.generator(4321, "cuda")
+    k = sd.normal_bf16((B, Hkv, P + n_q, D), g, "cuda")
+    v = sd.normal_bf16((B, Hkv, P + n_q, D), g, "cuda")
+    q = sd.normal_bf16((B, n_q, Hq, D), g, "cuda")
+    f32 = lambda shape: torch.empty(shape, dtype=torch.float32, device="cuda")
+    full = vc.verify_attn(q, k, v, P, out=f32(q.shape))
+    for i in (0, 15, 31, 32):
+        qi = q[:, i:i + 1].contiguous()
+        one = vc.verify_attn(qi, k, v, P + i, out=f32(qi.shape))
+        torch.cuda.synchronize()
+        assert torch.equal(one[:, 0], full[:, i]), f"row {i} differs"
+    assert torch.isfinite(full).all()
+
+
 @pytest.mark.parametrize("chunk", [4096, 8192, 12288])
 def test_chunked_equals_single_pass(chunk):
     P, n_q = 20000, 41
