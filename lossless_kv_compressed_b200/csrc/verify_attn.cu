@@ -8,9 +8,11 @@
 //
 // Decomposition.  A CTA owns one pair, one group of <= 256 query rows (two M = 128
 // UMMA tiles; row r = i * g + h) and one split of the keys: the intersection of the
-// call's key range with an absolute window [s * 4096, (s + 1) * 4096).  Split windows
-// and 64-key tiles sit at fixed absolute positions, so a row's result does not depend
-// on n_q or on the other rows (a verify row equals the same token decoded alone).
+// call's key range with an absolute window [s * w, (s + 1) * w) (w a launch parameter:
+// 2048-4096 keys chosen from the cache geometry by the entry point, smaller for the
+// loop's decode-sized blocks).  Split windows and 64-key tiles sit at fixed absolute
+// positions, so a row's result does not depend on n_q or on the other rows (a verify
+// row equals the same token decoded alone).
 //
 // Per CTA (384 threads):
 //   warp 0      TMA producer: K and V tiles [64 keys x D] (128-byte swizzle) into a
