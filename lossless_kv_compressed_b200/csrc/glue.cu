@@ -3,7 +3,6 @@
 // number of rows, so a block of k+1 tokens and k+1 single tokens agree bit for bit.
 #include <math.h>
 
-
 #include "vc_common.cuh"
 #include "vc_internal.h"
 #include "vericache_glue.h"
