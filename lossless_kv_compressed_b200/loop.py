@@ -274,24 +274,49 @@ class GpuTinyLM:
                                          self._s()), "vc_glue_greedy_steps")
 
     # ---------------------------------------------------------------- CentroidKV
-    def csm_init(self, n: int):
-        """The compressed cache starts as the prompt's own rows, degree 1."""
+    def _csm_alloc(self, n: int, rounds: int = 0):
         c = self.cfg
         cap = self.s_cap
         if n > cap:
-            raise ValueError(f"compressed-cache capacity {cap} < prompt length {n}")
+            raise ValueError(f"compressed-cache capacity {cap} < {n} rows")
         bf, i32 = torch.bfloat16, torch.int32
         mk = lambda: [(torch.empty((1, c.Hkv, cap, c.D), dtype=bf, device=self.dev),
                        torch.empty((1, c.Hkv, cap, c.D), dtype=bf, device=self.dev),
                        torch.empty((1, c.Hkv, cap), dtype=i32, device=self.dev))
                       for _ in range(c.n_layers)]
-        self.csm = {"cur": mk(), "alt": mk(), "round": 0}
-        for l in range(c.n_layers):
+        self.csm = {"cur": mk(), "alt": mk(), "round": rounds}
+
+    def csm_init(self, n: int):
+        """The compressed cache starts as the prompt's own rows, degree 1."""
+        self._csm_alloc(n)
+        for l in range(self.cfg.n_layers):
             kc, vcc, dc = self.csm["cur"][l]
             kc[:, :, :n].copy_(self.K[l][:, :, :n])
             vcc[:, :, :n].copy_(self.V[l][:, :, :n])
             dc[:, :, :n].fill_(1)
         self.S = n
+
+    def csm_export(self):
+        """The compact cache as three contiguous tensors: K and V [layers, Hkv, S, D] bf16
+        and the degrees [layers, Hkv, S] int32."""
+        cur = self.csm["cur"]
+        S = self.S
+        return (torch.stack([kc[0, :, :S] for kc, _, _ in cur]),
+                torch.stack([vcc[0, :, :S] for _, vcc, _ in cur]),
+                torch.stack([dc[0, :, :S] for _, _, dc in cur]))
+
+    def csm_load(self, k_rows: torch.Tensor, v_rows: torch.Tensor, deg: torch.Tensor,
+                 rounds: int):
+        """Take a compact cache built elsewhere (the layout of csm_export) as this model's
+        compressed cache; ``rounds`` clustering rounds have already run on it."""
+        S = k_rows.shape[2]
+        self._csm_alloc(S, rounds)
+        for l in range(self.cfg.n_layers):
+            kc, vcc, dc = self.csm["cur"][l]
+            kc[0, :, :S].copy_(k_rows[l])
+            vcc[0, :, :S].copy_(v_rows[l])
+            dc[0, :, :S].copy_(deg[l])
+        self.S = S
 
     def csm_round(self, n_sinks: int, n_recent: int, chunk: int, r: float) -> int:
         """One Chunked Soft Matching round (vc_csm_compress) over every layer's compressed
@@ -310,14 +335,45 @@ class GpuTinyLM:
     def csm_append(self, P: int, n: int):
         """The accepted tokens' verify-pass K/V (rows P .. P+n-1 of the full cache) join
         the compressed cache with degree 1."""
+        self.csm_append_rows([self.K[l][0, :, P:P + n] for l in range(self.cfg.n_layers)],
+                             [self.V[l][0, :, P:P + n] for l in range(self.cfg.n_layers)], n)
+
+    def full_rows(self, P: int, n: int) -> torch.Tensor:
+        """Rows P .. P+n-1 of the full cache, every layer: [layers, 2 (K, V), Hkv, n, D]."""
+        return torch.stack([torch.stack([self.K[l][0, :, P:P + n], self.V[l][0, :, P:P + n]])
+                            for l in range(self.cfg.n_layers)])
+
+    def csm_append_rows(self, k_rows, v_rows, n: int):
+        """n rows per layer ([Hkv, n, D] each) join the compressed cache with degree 1."""
         if self.S + n > self.s_cap:
             raise ValueError("compressed cache full")
         for l in range(self.cfg.n_layers):
             kc, vcc, dc = self.csm["cur"][l]
-            kc[:, :, self.S:self.S + n].copy_(self.K[l][:, :, P:P + n])
-            vcc[:, :, self.S:self.S + n].copy_(self.V[l][:, :, P:P + n])
+            kc[0, :, self.S:self.S + n].copy_(k_rows[l])
+            vcc[0, :, self.S:self.S + n].copy_(v_rows[l])
             dc[:, :, self.S:self.S + n].fill_(1)
         self.S += n
+
+
+def csm_step(model: GpuTinyLM, n_sinks: int, n_recent: int, chunk: int, r_init: float,
+             delta_r: float, r_floor: float) -> int:
+    """Clustering round j of the progressive schedule, r_j = max(r_floor, r_init - j
+    delta_r) (CentroidKV summary, "Riassunto Tecnico: CentroidKV", section "Metodologia",
+    item 3); returns the new cache size."""
+    r = max(r_floor, r_init - model.csm["round"] * delta_r)
+    return model.csm_round(n_sinks, n_recent, chunk, r)
+
+
+def csm_fit(model: GpuTinyLM, budget: int, *sched) -> list:
+    """Clustering rounds until the cache fits the budget (or a round removes nothing);
+    returns the size after each round."""
+    sizes = []
+    while model.S > budget:
+        before = model.S
+        sizes.append(csm_step(model, *sched))
+        if model.S == before:
+            break
+    return sizes
 
 
 def greedy_loop(model: GpuTinyLM, prompt: np.ndarray, n_gen: int) -> list:
@@ -381,17 +437,8 @@ def vericache_loop_csm(model: GpuTinyLM, prompt: np.ndarray, n_gen: int, k: int,
     n = len(prompt)
     logits = model.prefill(prompt)
     model.csm_init(n)
-    sizes = []
-
-    def cluster():
-        r = max(r_floor, r_init - model.csm["round"] * delta_r)
-        sizes.append(model.csm_round(n_sinks, n_recent, chunk, r))
-
-    while model.S > budget:
-        before = model.S
-        cluster()
-        if model.S == before:
-            break
+    sched = (n_sinks, n_recent, chunk, r_init, delta_r, r_floor)
+    sizes = csm_fit(model, budget, *sched)
     dev = model.dev
     first = torch.empty((1, 1), dtype=torch.int32, device=dev)
     accept(logits.view(1, 1, -1), target=first)
@@ -419,5 +466,5 @@ def vericache_loop_csm(model: GpuTinyLM, prompt: np.ndarray, n_gen: int, k: int,
         if since >= recluster_every:
             since = 0
             if model.S > budget:
-                cluster()
+                sizes.append(csm_step(model, *sched))
     return out[:n_gen], alens, sizes
