@@ -855,6 +855,16 @@ def workload_loop(dev) -> dict:
         c_model, prompt, cfg.gen_tokens, cfg.k, cfg.budget, cfg.n_sinks, cfg.n_recent,
         chunk=cfg.csm_chunk, r_init=cfg.csm_r_init, delta_r=cfg.csm_delta_r,
         r_floor=cfg.csm_r_floor, recluster_every=cfg.csm_recluster_every))
+    # remote prefix caching: the same CentroidKV loop split into a drafting side (compact
+    # cache only) and a verifying side (full cache), both on this GPU, joined by device
+    # copies -- what the split costs on one device, and the bytes its link would carry
+    from lossless_kv_compressed_b200.remote import DrafterSide, VerifierSide, run_local
+    sched = (cfg.budget, cfg.n_sinks, cfg.n_recent, cfg.csm_chunk, cfg.csm_r_init,
+             cfg.csm_delta_r, cfg.csm_r_floor)
+    r_ver = VerifierSide(GpuTinyLM(w, cfg, max_len, cfg.k, cap, device=dev), cfg.k, sched)
+    r_dra = DrafterSide(GpuTinyLM(w, cfg, max_len, cfg.k, cap, device=dev), cfg.k, sched,
+                        cfg.csm_recluster_every)
+    (rtoks, ralens, link), tr = timed(lambda: run_local(r_dra, r_ver, prompt, cfg.gen_tokens))
     a_us = _events_median(_accept_case(1, cfg.k + 1, cfg.vocab, dev, cfg.seed + 1)) * 1e6
     clk = clocks.stop()
     hist = np.bincount(np.asarray(alens), minlength=cfg.k + 1).tolist()
@@ -875,6 +885,15 @@ def workload_loop(dev) -> dict:
                 "schedule": {"chunk": cfg.csm_chunk, "r_init": cfg.csm_r_init,
                              "delta_r": cfg.csm_delta_r, "r_floor": cfg.csm_r_floor,
                              "recluster_every": cfg.csm_recluster_every}},
+        "remote_split": {"accepted_tokens_per_s": cfg.gen_tokens / tr,
+                         "commits_equal_greedy": rtoks == greedy,
+                         "accept_lens_equal_csm_loop": ralens == calens,
+                         "rounds": len(ralens),
+                         "link_bytes": {"compact_cache_once": link["setup"],
+                                        "to_verifier_per_round": link["to_verifier"] / len(ralens),
+                                        "to_drafter_per_round": link["to_drafter"] / len(ralens)},
+                         "note": "drafting side and verifying side on one GPU, joined by "
+                                 "device copies"},
         "config": {"layers": cfg.n_layers, "d_model": cfg.d_model,
                    "heads": f"{cfg.Hq}/{cfg.Hkv}", "head_dim": cfg.D, "ffn": cfg.ffn,
                    "vocab": cfg.vocab, "prompt": cfg.prompt_len, "generated": cfg.gen_tokens,
