@@ -1142,6 +1142,26 @@ def run_profile_case(kind: str) -> int:
     from synth import gen
     if kind in ("int4", "verify3"):
         return _profile_int4(kind)
+    if kind == "greedy":
+        # the tiny decoder's decode step: prefill the 8192-token prompt, then 4 greedy
+        # steps inside a profiler range (ncu --profile-from-start off captures only those)
+        from lossless_kv_compressed_b200.loop import GpuTinyLM
+        from synth.configs import get_config
+        c = get_config(5)
+        dev = torch.device("cuda", 0)
+        m = GpuTinyLM(gen.tinylm_weights(c), c, c.prompt_len + c.gen_tokens + c.k + 2, c.k,
+                      c.budget + c.gen_tokens + c.k + 2, device=dev)
+        logits = m.prefill(gen.tinylm_prompt(c))
+        ids = torch.empty(8, dtype=torch.int32, device=dev)
+        vc.accept(logits.view(1, 1, -1), target=ids[0:1].view(1, 1))
+        m.greedy_steps(ids, 2, c.prompt_len)            # warm: module load, first launches
+        torch.cuda.synchronize()
+        torch.cuda.cudart().cudaProfilerStart()
+        m.greedy_steps(ids[2:], 4, c.prompt_len + 2)
+        torch.cuda.synchronize()
+        torch.cuda.cudart().cudaProfilerStop()
+        print(json.dumps({"profile_case": kind, "workload": c.name, "ok": True}), flush=True)
+        return 0
     if kind == "csm":
         # one Chunked Soft Matching round over the 32K-context caches (chunk 256, r 0.5),
         # five times: about 2 GB on the device
@@ -1204,7 +1224,7 @@ def main():
     ap.add_argument("--table", action="store_true",
                     help="per-kernel rates at every workload's shapes, one JSON line per row")
     ap.add_argument("--profile-case",
-                    choices=["draft", "verify", "accept", "int4", "verify3", "csm"],
+                    choices=["draft", "verify", "accept", "int4", "verify3", "csm", "greedy"],
                     default=None,
                     help="run five calls of one entry point on the 32K-context inputs (one "
                          "copy) for an ncu capture, and print no bench line")
