@@ -146,7 +146,14 @@ def run_local(drafter, verifier, prompt, n_gen: int):
 
 # ---------------------------------------------------------------- one side per rank
 def _wire_dev(side):
-    return side.dev if dist.get_backend() == "nccl" else torch.device("cpu")
+    """NCCL moves the side's own device tensors (the rank must have made that device
+    current); gloo moves host copies."""
+    if dist.get_backend() == "nccl":
+        if side.dev.type != "cuda" or torch.cuda.current_device() != side.dev.index:
+            raise RuntimeError(f"NCCL rank: make {side.dev} the current device first "
+                               "(torch.cuda.set_device)")
+        return side.dev
+    return torch.device("cpu")
 
 
 def _send(t: torch.Tensor, peer: int, wire) -> None:
