@@ -149,7 +149,8 @@ def _wire_dev(side):
     """NCCL moves the side's own device tensors (the rank must have made that device
     current); gloo moves host copies."""
     if dist.get_backend() == "nccl":
-        if side.dev.type != "cuda" or torch.cuda.current_device() != side.dev.index:
+        idx = side.dev.index if side.dev.index is not None else torch.cuda.current_device()
+        if side.dev.type != "cuda" or torch.cuda.current_device() != idx:
             raise RuntimeError(f"NCCL rank: make {side.dev} the current device first "
                                "(torch.cuda.set_device)")
         return side.dev
