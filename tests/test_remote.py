@@ -167,3 +167,54 @@ def test_two_gloo_ranks_exchange_the_same_rounds():
     assert got[0] == alens                      # the verifier rank's accept lengths
     assert got[1][0] == toks == greedy_stream()  # the drafter rank's committed stream
     assert got[1][1] == sum(a + 1 for a in alens)
+
+
+def _rank_dies(rank, port, q):
+    """Rank 1 takes the compact cache and exits without drafting (a drafter that died
+    between rounds); rank 0 must end with an error from its next receive."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import datetime
+    import time
+    import torch.distributed as dist
+    from lossless_kv_compressed_b200.remote import _recv, run_verifier
+    import test_remote as T
+    dist.init_process_group("gloo", rank=rank, world_size=2,
+                            timeout=datetime.timedelta(seconds=10))
+    if rank == 1:
+        hdr = _recv((4,), torch.int64, 0, torch.device("cpu"), "cpu").tolist()
+        S = hdr[0]
+        for shape, dt in (((L, HKV, S, D), torch.bfloat16), ((L, HKV, S, D), torch.bfloat16),
+                          ((L, HKV, S), torch.int32)):
+            _recv(shape, dt, 0, torch.device("cpu"), "cpu")
+        q.put((1, "left"))
+        q.close()
+        q.join_thread()                               # the message is out before the exit
+        os._exit(0)                                   # no teardown: the peer just vanishes
+    t0 = time.monotonic()
+    try:
+        run_verifier(T.ToyVerifier(), T.PROMPT, T.N_GEN, peer=1)
+        q.put((0, ("no error", time.monotonic() - t0)))
+    except Exception as e:                           # the failure surfaces on the host
+        q.put((0, (type(e).__name__, time.monotonic() - t0)))
+    q.close()
+    q.join_thread()
+    os._exit(0)
+
+
+@pytest.mark.timeout(180)
+def test_a_drafter_rank_that_dies_ends_the_verifier_with_an_error():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_dies, args=(r, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=150) for _ in procs)
+    for p in procs:
+        p.join(timeout=30)
+    assert got[1] == "left"
+    kind, seconds = got[0]
+    assert kind != "no error"
+    assert seconds < 60                               # bounded by the group's timeout
